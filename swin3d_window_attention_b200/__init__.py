@@ -1,0 +1,14 @@
+"""B200-native (sm_100a) Swin3D shifted-window attention and AdaLN + residual.
+
+The compute lives in CUDA kernels behind a C ABI (``include/swin3d_wa.h``); this
+package is the thin ctypes binding over that library.  Importing the package does not
+load the shared library; the first call does, and fails loudly if it is missing.
+"""
+# placeholder until api exists
+if False:
+    from .api import (  # noqa: F401
+    adaln_residual_fwd,
+    library_path,
+    load_library,
+    swin3d_window_attn_fwd,
+)
