@@ -1,0 +1,137 @@
+/*
+ * swin3d_wa.h - C ABI of the B200 (sm_100a) Swin3D shifted-window attention path.
+ *
+ * Two compute calls, both asynchronous on the caller's CUDA stream:
+ *
+ *   swin3d_window_attn_fwd  cyclic shift + pad + 3D window partition, masked per-window
+ *                           multi-head softmax attention, inverse merge + un-shift, all in
+ *                           one kernel launch that reads Q/K/V straight from grid layout
+ *                           and writes O straight back to grid layout.
+ *   adaln_residual_fwd      LayerNorm + FiLM modulation + residual add in one pass, with
+ *                           optional FP32 output.
+ *
+ * Defining passages ("Flash-Aurora: Toward Efficient Inference for Geospatial Foundation
+ * Models"):
+ *   - section "Kernel fusion for backbone memory traffic": cyclic shift, pad, 3D window
+ *     partition and inverse merge fused instead of eager views/copies; LayerNorm, FiLM
+ *     modulation and residual add without a full-width intermediate; FP32 activations
+ *     between blocks (output_fp32).
+ *   - section "CuTe DSL window attention": window (2,6,12) -> N = 144 tokens; logits
+ *     S = scale * Q K^T, the Swin shift mask, row-wise softmax in FP32, O = softmax(S) V,
+ *     no N x N map in global memory; BF16 activations with FP32 softmax (BF16_MIXED).
+ *   - section "Window attention kernels": head_dim 64 on the production shapes.
+ *
+ * Semantics of swin3d_window_attn_fwd (the readings are stated where the pages leave a
+ * step open):
+ *   1. Each axis a of the token grid (T, H, W) is padded up to P_a = ceil(D_a / w_a) * w_a.
+ *   2. The padded grid is rolled by -shift (pad first, then roll); window slot p' of
+ *      axis a holds the original coordinate p = (p' + s_a) mod P_a; the token is real iff
+ *      p < D_a on every axis.
+ *   3. Region label per axis on the shifted grid: 0 if s_a = 0 or p' < P_a - w_a,
+ *      1 if P_a - w_a <= p' < P_a - s_a, else 2.  Query i may attend key j iff j is real
+ *      and the labels agree on every axis (the -infinity limit of Swin's -100 bias).
+ *   4. Per (sample, window, head): S = scale * Q K^T (bf16 inputs, fp32 accumulate),
+ *      masked softmax in fp32, the probabilities rounded to bf16, O = P V / rowsum(P)
+ *      (fp32 accumulate).
+ *   5. O of each real token is written to its original grid position, exactly once;
+ *      padded slots are dropped.
+ *
+ * Memory layout: q, k, v and o are grid layout [B][T][H][W][token stride]; channel
+ * c = head * head_dim + d.  The caller owns every buffer.  The library allocates no
+ * device memory and keeps no state except a per-device error word and a cached SM count.
+ *
+ * Error convention: every argument check runs on the host before any launch; a failed
+ * check returns a non-zero s3w_status and launches nothing.  A failed launch returns
+ * S3W_ERR_CUDA.  A kernel whose bounded wait expired records S3W_ERR_DEVICE_TIMEOUT in
+ * the device error word, which s3w_poll_device_error() reads and clears.
+ */
+#ifndef SWIN3D_WA_H_
+#define SWIN3D_WA_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* s3w_stream_t;
+
+typedef enum {
+  S3W_OK = 0,
+  S3W_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, shift >= window, ...     */
+  S3W_ERR_UNSUPPORTED = 2,   /* valid but not built: head_dim, window size, dtype combo   */
+  S3W_ERR_MISALIGNED = 3,    /* pointer or stride not 16-byte aligned                     */
+  S3W_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed                      */
+  S3W_ERR_DEVICE_TIMEOUT = 5 /* a bounded wait inside a kernel expired                    */
+} s3w_status;
+
+typedef enum { S3W_BF16 = 0, S3W_F32 = 1 } s3w_dtype;
+
+/*
+ * Shifted-window attention forward.
+ *
+ * q, k, v   device pointers, in_dtype elements (S3W_BF16 only), grid layout with
+ *           qkv_token_stride elements between consecutive tokens (>= heads*head_dim, a
+ *           multiple of 8 so that every token row starts on a 16-byte boundary; q, k and v
+ *           may be three slices of one fused [tokens][3C] buffer).  16-byte aligned.
+ * o         device pointer, out_dtype elements (S3W_BF16 or S3W_F32), grid layout with
+ *           o_token_stride elements between tokens (>= heads*head_dim, 16-byte rows).
+ *           Must not overlap q, k or v.  Channels beyond heads*head_dim are not written.
+ * B,T,H,W   batch and unpadded grid sizes, each >= 1.
+ * win_*     window extents, each >= 1; N = win_t*win_h*win_w must satisfy 1 <= N <= 144.
+ * shift_*   0 <= shift < window on each axis.
+ * heads     >= 1.  head_dim: 32 or 64.
+ * scale     logit scale; a value <= 0 selects 1/sqrt(head_dim).
+ * stream    CUDA stream; the call only enqueues work.
+ *
+ * Returns S3W_OK or an s3w_status; on error nothing is launched.
+ */
+int swin3d_window_attn_fwd(const void* q, const void* k, const void* v, void* o,
+                           int B, int T, int H, int W,
+                           int win_t, int win_h, int win_w,
+                           int shift_t, int shift_h, int shift_w,
+                           int heads, int head_dim,
+                           long long qkv_token_stride, long long o_token_stride,
+                           float scale, int in_dtype, int out_dtype,
+                           s3w_stream_t stream);
+
+/*
+ * Fused AdaLN + residual forward ("Kernel fusion for backbone memory traffic").
+ *
+ * For every sample b and token l of x[B][L][C] (contiguous rows of C elements):
+ *   mean = sum_c x / C,  var = sum_c (x - mean)^2 / C        (biased, two passes)
+ *   out  = residual + (x - mean) / sqrt(var + eps) * (1 + scale[b]) + shift[b]
+ * computed in fp32 and stored as out_dtype (S3W_F32 keeps the FP32 residual stream
+ * between blocks; S3W_BF16 rounds to nearest even).
+ *
+ * x         device, x_dtype (S3W_BF16 or S3W_F32), [B][L][C], 16-byte aligned.
+ * residual  device fp32 [B][L][C], 16-byte aligned.  out may alias residual exactly
+ *           (in-place update of the residual stream); no other overlap is allowed.
+ * scale, shift  device fp32 [B][C] per-sample FiLM vectors, 16-byte aligned.
+ * out       device, out_dtype, [B][L][C], 16-byte aligned.
+ * B >= 1, tokens_per_sample >= 0 (0 launches nothing), C a multiple of 8 with
+ * 8 <= C <= 4096; eps >= 0.
+ */
+int adaln_residual_fwd(const void* x, int x_dtype, const float* residual,
+                       const float* scale, const float* shift,
+                       void* out, int out_dtype,
+                       int B, long long tokens_per_sample, int C, float eps,
+                       s3w_stream_t stream);
+
+/* Static English text for a status code (never NULL). */
+const char* s3w_status_string(int status);
+
+/*
+ * Synchronises `stream`, then reads and clears the calling device's error word.
+ * Returns S3W_OK, S3W_ERR_DEVICE_TIMEOUT (a kernel gave up a bounded wait and returned
+ * early; its output is incomplete) or S3W_ERR_CUDA (the synchronisation failed).
+ */
+int s3w_poll_device_error(s3w_stream_t stream);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int s3w_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWIN3D_WA_H_ */

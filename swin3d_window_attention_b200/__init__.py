@@ -4,11 +4,12 @@ The compute lives in CUDA kernels behind a C ABI (``include/swin3d_wa.h``); this
 package is the thin ctypes binding over that library.  Importing the package does not
 load the shared library; the first call does, and fails loudly if it is missing.
 """
-# placeholder until api exists
-if False:
-    from .api import (  # noqa: F401
+from .api import (  # noqa: F401
+    S3WError,
     adaln_residual_fwd,
     library_path,
     load_library,
+    poll_device_error,
+    status_string,
     swin3d_window_attn_fwd,
 )

@@ -1,0 +1,133 @@
+"""ctypes binding of the C ABI in include/swin3d_wa.h.
+
+Argument marshalling only: every step of the computation runs in the CUDA library.
+Tensors are PyTorch CUDA tensors (PyTorch supplies device memory and streams); the
+current stream of the tensors' device is passed to the library.  There is no CPU
+fallback: if the shared library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libswin3d_wa.so"
+
+S3W_OK, S3W_ERR_INVALID_ARG, S3W_ERR_UNSUPPORTED, S3W_ERR_MISALIGNED, S3W_ERR_CUDA, S3W_ERR_DEVICE_TIMEOUT = range(6)
+S3W_BF16, S3W_F32 = 0, 1
+
+_lib = None
+
+
+class S3WError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+def library_path() -> str:
+    return os.path.join(HERE, _LIB_NAME)
+
+
+def load_library():
+    """Load the in-tree shared library; raise if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m swin3d_window_attention_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, LL, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float
+    lib.swin3d_window_attn_fwd.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, I, LL, LL, F, I, I, P]
+    lib.swin3d_window_attn_fwd.restype = I
+    lib.adaln_residual_fwd.argtypes = [P, I, P, P, P, P, I, I, LL, I, F, P]
+    lib.adaln_residual_fwd.restype = I
+    lib.s3w_status_string.argtypes = [I]
+    lib.s3w_status_string.restype = ctypes.c_char_p
+    lib.s3w_poll_device_error.argtypes = [P]
+    lib.s3w_poll_device_error.restype = I
+    lib.s3w_version.argtypes = []
+    lib.s3w_version.restype = I
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().s3w_status_string(int(status)).decode()
+
+
+def _dtype_code(t) -> int:
+    import torch
+
+    if t.dtype == torch.bfloat16:
+        return S3W_BF16
+    if t.dtype == torch.float32:
+        return S3W_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream_of(t) -> int:
+    import torch
+
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _token_stride(t, C: int) -> int:
+    """Elements between consecutive grid tokens of a [B, T, H, W, >=C] view."""
+    if t.dim() != 5:
+        raise ValueError("expected a grid-layout tensor [B, T, H, W, channels]")
+    if t.stride(4) != 1:
+        raise ValueError("channels must be contiguous")
+    ts = t.stride(3)
+    if t.stride(2) != ts * t.shape[3] or t.stride(1) != t.stride(2) * t.shape[2] or t.stride(0) != t.stride(1) * t.shape[1]:
+        raise ValueError("grid tokens must be evenly strided")
+    if t.shape[4] < C:
+        raise ValueError("fewer channels than heads * head_dim")
+    return ts
+
+
+def swin3d_window_attn_fwd(q, k, v, o, heads: int, head_dim: int, window=(2, 6, 12), shift=(0, 0, 0),
+                           scale: float = 0.0, stream=None, check: bool = True) -> int:
+    """Shifted-window attention.  q, k, v: bf16 CUDA tensors [B, T, H, W, >=heads*head_dim]
+    with one token stride; o: bf16 or fp32 [B, T, H, W, >=heads*head_dim].  Returns the
+    status (raises S3WError on a non-zero status when ``check``)."""
+    lib = load_library()
+    C = heads * head_dim
+    B, T, H, W = q.shape[:4]
+    ts = _token_stride(q, C)
+    if _token_stride(k, C) != ts or _token_stride(v, C) != ts:
+        raise ValueError("q, k and v must share one token stride")
+    if tuple(o.shape[:4]) != (B, T, H, W) or tuple(k.shape[:4]) != (B, T, H, W) or tuple(v.shape[:4]) != (B, T, H, W):
+        raise ValueError("q, k, v and o must have the same grid shape")
+    ots = _token_stride(o, C)
+    st = _stream_of(q) if stream is None else stream
+    rc = lib.swin3d_window_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), B, T, H, W,
+                                    *window, *shift, heads, head_dim, ts, ots, float(scale),
+                                    _dtype_code(q), _dtype_code(o), st)
+    if check and rc != S3W_OK:
+        raise S3WError(rc, "swin3d_window_attn_fwd")
+    return rc
+
+
+def adaln_residual_fwd(x, residual, scale, shift, out, eps: float = 1e-5, stream=None, check: bool = True) -> int:
+    """AdaLN + residual.  x: bf16/fp32 [B, L, C]; residual: fp32 [B, L, C]; scale, shift:
+    fp32 [B, C]; out: fp32/bf16 [B, L, C] (may be ``residual`` itself)."""
+    lib = load_library()
+    B, L, C = x.shape
+    for t in (x, residual, out):
+        if not t.is_contiguous():
+            raise ValueError("x, residual and out must be contiguous")
+    st = _stream_of(x) if stream is None else stream
+    rc = lib.adaln_residual_fwd(x.data_ptr(), _dtype_code(x), residual.data_ptr(), scale.data_ptr(),
+                                shift.data_ptr(), out.data_ptr(), _dtype_code(out), B, L, C, float(eps), st)
+    if check and rc != S3W_OK:
+        raise S3WError(rc, "adaln_residual_fwd")
+    return rc
+
+
+def poll_device_error(stream=None) -> int:
+    import torch
+
+    st = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    return load_library().s3w_poll_device_error(st)

@@ -1,0 +1,163 @@
+// C ABI of the shifted-window attention library: host-side argument checks, the
+// per-device error word, and kernel dispatch.  Every check runs before any launch; a
+// failed check returns a status and enqueues nothing.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/swin3d_wa.h"
+#include "s3w_internal.h"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// One error word per device; kernels get its device address.
+__device__ int g_s3w_error_word;
+
+struct DeviceState {
+  int* err = nullptr;
+  int num_sms = 0;
+  bool ready = false;
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mu;
+
+int device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return S3W_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& s = g_dev[dev];
+  if (!s.ready) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_s3w_error_word) != cudaSuccess) return S3W_ERR_CUDA;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return S3W_ERR_CUDA;
+    s.err = static_cast<int*>(p);
+    s.num_sms = sms;
+    s.ready = true;
+  }
+  *out = &s;
+  return S3W_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+long long g_spin_limit = 1ll << 26;  // bounded-wait iterations inside kernels
+
+}  // namespace
+
+extern "C" {
+
+const char* s3w_status_string(int status) {
+  switch (status) {
+    case S3W_OK: return "ok";
+    case S3W_ERR_INVALID_ARG: return "invalid argument";
+    case S3W_ERR_UNSUPPORTED: return "unsupported configuration";
+    case S3W_ERR_MISALIGNED: return "pointer or stride not 16-byte aligned";
+    case S3W_ERR_CUDA: return "CUDA runtime error";
+    case S3W_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel expired";
+    default: return "unknown status";
+  }
+}
+
+int s3w_version(void) { return 100; }
+
+int s3w_poll_device_error(s3w_stream_t stream) {
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != S3W_OK) return rc;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return S3W_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, ds->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return S3W_ERR_CUDA;
+  if (word != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(ds->err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return S3W_ERR_CUDA;
+    return S3W_ERR_DEVICE_TIMEOUT;
+  }
+  return S3W_OK;
+}
+
+int swin3d_window_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int T, int H, int W,
+                           int win_t, int win_h, int win_w, int shift_t, int shift_h, int shift_w, int heads,
+                           int head_dim, long long qkv_token_stride, long long o_token_stride, float scale,
+                           int in_dtype, int out_dtype, s3w_stream_t stream) {
+  if (!q || !k || !v || !o) return S3W_ERR_INVALID_ARG;
+  if (B < 1 || T < 1 || H < 1 || W < 1 || heads < 1 || head_dim < 1) return S3W_ERR_INVALID_ARG;
+  if (win_t < 1 || win_h < 1 || win_w < 1) return S3W_ERR_INVALID_ARG;
+  if (shift_t < 0 || shift_h < 0 || shift_w < 0 || shift_t >= win_t || shift_h >= win_h || shift_w >= win_w)
+    return S3W_ERR_INVALID_ARG;
+  if (!(scale == scale) || std::isinf(scale)) return S3W_ERR_INVALID_ARG;
+  if ((in_dtype != S3W_BF16 && in_dtype != S3W_F32) || (out_dtype != S3W_BF16 && out_dtype != S3W_F32))
+    return S3W_ERR_INVALID_ARG;
+  const long long C = static_cast<long long>(heads) * head_dim;
+  if (qkv_token_stride < C || o_token_stride < C) return S3W_ERR_INVALID_ARG;
+  const long long N = static_cast<long long>(win_t) * win_h * win_w;
+  if (N > 144) return S3W_ERR_UNSUPPORTED;
+  if (head_dim != 32 && head_dim != 64) return S3W_ERR_UNSUPPORTED;
+  if (in_dtype != S3W_BF16) return S3W_ERR_UNSUPPORTED;
+  const int ob = out_dtype == S3W_F32 ? 4 : 2;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return S3W_ERR_MISALIGNED;
+  if ((qkv_token_stride * 2) % 16 != 0 || (o_token_stride * ob) % 16 != 0) return S3W_ERR_MISALIGNED;
+  // padded grid sizes must stay in int range
+  const long long Pt = (T + win_t - 1) / win_t * static_cast<long long>(win_t);
+  const long long Ph = (H + win_h - 1) / win_h * static_cast<long long>(win_h);
+  const long long Pw = (W + win_w - 1) / win_w * static_cast<long long>(win_w);
+  if (Pt > INT32_MAX / 2 || Ph > INT32_MAX / 2 || Pw > INT32_MAX / 2) return S3W_ERR_UNSUPPORTED;
+  const long long per_sample = (Pt / win_t) * (Ph / win_h) * (Pw / win_w);
+  if (per_sample > INT32_MAX) return S3W_ERR_UNSUPPORTED;
+
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != S3W_OK) return rc;
+
+  s3w::WinGeom g;
+  g.B = B; g.T = T; g.H = H; g.W = W;
+  g.wt = win_t; g.wh = win_h; g.ww = win_w;
+  g.st = shift_t; g.sh = shift_h; g.sw = shift_w;
+  g.Pt = static_cast<int>(Pt); g.Ph = static_cast<int>(Ph); g.Pw = static_cast<int>(Pw);
+  g.nwt = g.Pt / win_t; g.nwh = g.Ph / win_h; g.nww = g.Pw / win_w;
+  g.N = static_cast<int>(N);
+  g.heads = heads;
+  g.head_dim = head_dim;
+  g.windows = per_sample * B;
+  g.qkv_stride = qkv_token_stride;
+  g.o_stride = o_token_stride;
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
+  g.scale_log2 = sc * 1.4426950408889634f;  // log2(e): softmax is evaluated with exp2
+  if (g.windows * heads > (1ll << 31) - 1) return S3W_ERR_UNSUPPORTED;
+
+  cudaError_t e = s3w::launch_window_attn_mma(g, q, k, v, o, out_dtype == S3W_F32,
+                                              reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? S3W_OK : S3W_ERR_CUDA;
+}
+
+int adaln_residual_fwd(const void* x, int x_dtype, const float* residual, const float* scale, const float* shift,
+                       void* out, int out_dtype, int B, long long tokens_per_sample, int C, float eps,
+                       s3w_stream_t stream) {
+  if (!x || !residual || !scale || !shift || !out) return S3W_ERR_INVALID_ARG;
+  if (B < 1 || tokens_per_sample < 0 || C < 1 || !(eps >= 0.f) || std::isinf(eps)) return S3W_ERR_INVALID_ARG;
+  if ((x_dtype != S3W_BF16 && x_dtype != S3W_F32) || (out_dtype != S3W_BF16 && out_dtype != S3W_F32))
+    return S3W_ERR_INVALID_ARG;
+  if (C % 8 != 0 || C > 4096) return S3W_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(residual) || !aligned16(scale) || !aligned16(shift) || !aligned16(out))
+    return S3W_ERR_MISALIGNED;
+  // out may alias residual exactly; any other overlap with residual is rejected
+  const long long n = static_cast<long long>(B) * tokens_per_sample * C;
+  const char* r0 = reinterpret_cast<const char*>(residual);
+  const char* o0 = reinterpret_cast<const char*>(out);
+  const long long ob = out_dtype == S3W_F32 ? 4 : 2;
+  if (o0 != r0 && o0 < r0 + n * 4 && r0 < o0 + n * ob) return S3W_ERR_INVALID_ARG;
+  if (B * tokens_per_sample > (1ll << 34)) return S3W_ERR_UNSUPPORTED;
+  if (tokens_per_sample == 0) return S3W_OK;
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != S3W_OK) return rc;
+  cudaError_t e = s3w::launch_adaln(x, x_dtype == S3W_BF16, residual, scale, shift, out, out_dtype == S3W_F32, B,
+                                    tokens_per_sample, C, eps, ds->num_sms, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? S3W_OK : S3W_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,25 @@
+// Host-side launch declarations shared between the C-ABI layer (api.cu) and the kernel
+// translation units.  Not part of the public ABI.
+#pragma once
+#include <cuda_runtime.h>
+
+#include "s3w_common.cuh"
+
+namespace s3w {
+
+// Window attention on the tcgen05 / TMEM path (attn_tcgen05.cu).
+cudaError_t launch_window_attn_tc(const WinGeom& g, const void* q, const void* k, const void* v,
+                                  void* o, bool out_f32, int* err, long long spin_limit,
+                                  int num_sms, cudaStream_t stream);
+
+// Window attention on the legacy warp-level mma.sync path (attn_mma.cu); kept as the
+// measured baseline the tcgen05 kernel is compared with.
+cudaError_t launch_window_attn_mma(const WinGeom& g, const void* q, const void* k, const void* v,
+                                   void* o, bool out_f32, cudaStream_t stream);
+
+// AdaLN + residual (adaln.cu).
+cudaError_t launch_adaln(const void* x, bool x_bf16, const float* residual, const float* scale,
+                         const float* shift, void* out, bool out_f32, int B, long long L, int C,
+                         float eps, int num_sms, cudaStream_t stream);
+
+}  // namespace s3w

@@ -1,0 +1,108 @@
+"""C-ABI checks that need no GPU: the library loads, exports every declared entry point,
+and rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import swin3d_window_attention_b200 as s3w
+from swin3d_window_attention_b200 import api
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x10000  # 16-byte aligned dummy address; only used with arguments that are rejected first
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = s3w.load_library()
+    names = declared_functions()
+    assert {"swin3d_window_attn_fwd", "adaln_residual_fwd", "s3w_status_string", "s3w_poll_device_error"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_status_strings():
+    assert s3w.status_string(0) == "ok"
+    for code in range(1, 6):
+        assert s3w.status_string(code) not in ("ok", "unknown status")
+    assert s3w.status_string(99) == "unknown status"
+    assert s3w.load_library().s3w_version() >= 100
+
+
+def _attn(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, B=1, T=4, H=12, W=24, wt=2, wh=6, ww=12, st=1, sh=3, sw=6,
+             heads=8, hd=64, qs=512, os_=512, scale=0.0, ind=0, outd=0, stream=None)
+    a.update(over)
+    return s3w.load_library().swin3d_window_attn_fwd(
+        a["q"], a["k"], a["v"], a["o"], a["B"], a["T"], a["H"], a["W"], a["wt"], a["wh"], a["ww"], a["st"],
+        a["sh"], a["sw"], a["heads"], a["hd"], a["qs"], a["os_"], a["scale"], a["ind"], a["outd"], a["stream"])
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(q=None), api.S3W_ERR_INVALID_ARG),
+    (dict(o=None), api.S3W_ERR_INVALID_ARG),
+    (dict(B=0), api.S3W_ERR_INVALID_ARG),
+    (dict(T=-1), api.S3W_ERR_INVALID_ARG),
+    (dict(st=2), api.S3W_ERR_INVALID_ARG),          # shift == window
+    (dict(sw=-1), api.S3W_ERR_INVALID_ARG),
+    (dict(wh=0), api.S3W_ERR_INVALID_ARG),
+    (dict(qs=100), api.S3W_ERR_INVALID_ARG),        # token stride < heads * head_dim
+    (dict(os_=511), api.S3W_ERR_INVALID_ARG),
+    (dict(outd=7), api.S3W_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), api.S3W_ERR_INVALID_ARG),
+    (dict(ww=13, sw=6), api.S3W_ERR_UNSUPPORTED),   # N = 156 > 144
+    (dict(hd=48, qs=384, os_=384), api.S3W_ERR_UNSUPPORTED),
+    (dict(ind=1), api.S3W_ERR_UNSUPPORTED),         # fp32 Q/K/V not built
+    (dict(q=FAKE + 8), api.S3W_ERR_MISALIGNED),
+    (dict(o=FAKE + 2), api.S3W_ERR_MISALIGNED),
+    (dict(qs=516), api.S3W_ERR_MISALIGNED),         # token rows not on 16-byte boundaries
+])
+def test_attn_rejects_bad_arguments_on_host(over, expect):
+    assert _attn(**over) == expect
+
+
+def _adaln(**over):
+    a = dict(x=FAKE, xd=0, res=FAKE, sc=FAKE, sh=FAKE, out=FAKE, outd=1, B=1, L=16, C=512, eps=1e-5)
+    a.update(over)
+    return s3w.load_library().adaln_residual_fwd(a["x"], a["xd"], a["res"], a["sc"], a["sh"], a["out"], a["outd"],
+                                                 a["B"], a["L"], a["C"], a["eps"], None)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(x=None), api.S3W_ERR_INVALID_ARG),
+    (dict(res=None), api.S3W_ERR_INVALID_ARG),
+    (dict(B=0), api.S3W_ERR_INVALID_ARG),
+    (dict(L=-1), api.S3W_ERR_INVALID_ARG),
+    (dict(eps=-1.0), api.S3W_ERR_INVALID_ARG),
+    (dict(xd=5), api.S3W_ERR_INVALID_ARG),
+    (dict(C=12), api.S3W_ERR_UNSUPPORTED),
+    (dict(C=8192), api.S3W_ERR_UNSUPPORTED),
+    (dict(sc=FAKE + 4), api.S3W_ERR_MISALIGNED),
+    (dict(out=FAKE + 16 * 512), api.S3W_ERR_INVALID_ARG),   # partial overlap with residual
+])
+def test_adaln_rejects_bad_arguments_on_host(over, expect):
+    # the overlap case keeps out != residual while the two ranges intersect
+    if "out" in over:
+        over = dict(over, res=FAKE + 64)
+    assert _adaln(**over) == expect
+
+
+def test_adaln_zero_tokens_is_a_no_op():
+    assert _adaln(L=0) == api.S3W_OK
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(api, "_lib", None)
+    monkeypatch.setattr(api, "HERE", str(tmp_path))
+    with pytest.raises(RuntimeError, match="missing"):
+        api.load_library()
