@@ -191,6 +191,18 @@ def bench_cuda(args):
     attn_ms = [a.elapsed_time(b) for a, b in attn_events]
     attn_avg_ms = sum(attn_ms) / len(attn_ms)
 
+    # For context: the same attention call on the legacy mma.sync baseline kernel.
+    leg = []
+    for i in range(3):
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        s3w.swin3d_window_attn_fwd_legacy_mma(d["q1"], d["k1"], d["v1"], o, HEADS, HD, WINDOW, SHIFTS[1])
+        a1.record(stream)
+        leg.append((a0, a1))
+    torch.cuda.synchronize()
+    legacy_ms = min(a.elapsed_time(b) for a, b in leg)
+
     # End-to-end through the public API with host buffers: every step copies its inputs
     # from pinned host memory and reads the step's result (the residual stream) back.
     pinned = {k: (torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) if v.dtype == np.uint16
@@ -247,7 +259,8 @@ def bench_cuda(args):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "attn": {"avg_launch_ms": attn_avg_ms, "hbm_gbs": attn_gbs, "tflops": attn_tflops,
                  "windows_per_s": N_WIN / (attn_avg_ms * 1e-3),
-                 "hbm_frac": attn_gbs / hbm_peak, "tensor_frac": attn_tflops / tc_peak},
+                 "hbm_frac": attn_gbs / hbm_peak, "tensor_frac": attn_tflops / tc_peak,
+                 "legacy_mma_baseline_ms": legacy_ms},
         "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": hbm_peak, "unit": "GB/s",
                      "frac": attn_gbs / hbm_peak, "traffic": None, "peak_source": peak_src,
                      "kernel": "window attention", "algorithmic_bytes_per_launch": ATTN_BYTES},

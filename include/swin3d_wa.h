@@ -95,6 +95,21 @@ int swin3d_window_attn_fwd(const void* q, const void* k, const void* v, void* o,
                            s3w_stream_t stream);
 
 /*
+ * The same operation and the same arguments, checks and results as
+ * swin3d_window_attn_fwd, computed on the legacy warp-level tensor path (mma.sync,
+ * one CTA per (window, head), loads and math not overlapped).  It is the measured
+ * baseline the tcgen05 path is compared with; it has no bounded waits.
+ */
+int swin3d_window_attn_fwd_legacy_mma(const void* q, const void* k, const void* v, void* o,
+                                      int B, int T, int H, int W,
+                                      int win_t, int win_h, int win_w,
+                                      int shift_t, int shift_h, int shift_w,
+                                      int heads, int head_dim,
+                                      long long qkv_token_stride, long long o_token_stride,
+                                      float scale, int in_dtype, int out_dtype,
+                                      s3w_stream_t stream);
+
+/*
  * Fused AdaLN + residual forward ("Kernel fusion for backbone memory traffic").
  *
  * For every sample b and token l of x[B][L][C] (contiguous rows of C elements):
@@ -126,6 +141,15 @@ const char* s3w_status_string(int status);
  * early; its output is incomplete) or S3W_ERR_CUDA (the synchronisation failed).
  */
 int s3w_poll_device_error(s3w_stream_t stream);
+
+/*
+ * Time limit, in nanoseconds, of every bounded wait inside kernels launched after the
+ * call (process-wide); returns the previous limit.  Default 1e9 (one second).  With 0, a
+ * wait not satisfied at its first poll expires: the kernel unwinds early (copies drained,
+ * tensor memory released), records S3W_ERR_DEVICE_TIMEOUT in the device error word and
+ * leaves the CUDA context usable.  Meant for tests of that failure path.
+ */
+long long s3w_set_wait_limit_ns(long long ns);
 
 /* Library version as major*10000 + minor*100 + patch. */
 int s3w_version(void);

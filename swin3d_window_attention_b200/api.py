@@ -41,6 +41,10 @@ def load_library():
     P, I, LL, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float
     lib.swin3d_window_attn_fwd.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, I, LL, LL, F, I, I, P]
     lib.swin3d_window_attn_fwd.restype = I
+    lib.swin3d_window_attn_fwd_legacy_mma.argtypes = lib.swin3d_window_attn_fwd.argtypes
+    lib.swin3d_window_attn_fwd_legacy_mma.restype = I
+    lib.s3w_set_wait_limit_ns.argtypes = [LL]
+    lib.s3w_set_wait_limit_ns.restype = LL
     lib.adaln_residual_fwd.argtypes = [P, I, P, P, P, P, I, I, LL, I, F, P]
     lib.adaln_residual_fwd.restype = I
     lib.s3w_status_string.argtypes = [I]
@@ -89,9 +93,21 @@ def _token_stride(t, C: int) -> int:
 
 def swin3d_window_attn_fwd(q, k, v, o, heads: int, head_dim: int, window=(2, 6, 12), shift=(0, 0, 0),
                            scale: float = 0.0, stream=None, check: bool = True) -> int:
-    """Shifted-window attention.  q, k, v: bf16 CUDA tensors [B, T, H, W, >=heads*head_dim]
-    with one token stride; o: bf16 or fp32 [B, T, H, W, >=heads*head_dim].  Returns the
-    status (raises S3WError on a non-zero status when ``check``)."""
+    """Shifted-window attention (tcgen05 path).  q, k, v: bf16 CUDA tensors
+    [B, T, H, W, >=heads*head_dim] with one token stride; o: bf16 or fp32
+    [B, T, H, W, >=heads*head_dim].  Returns the status (raises S3WError on a non-zero
+    status when ``check``)."""
+    return _attn("swin3d_window_attn_fwd", q, k, v, o, heads, head_dim, window, shift, scale, stream, check)
+
+
+def swin3d_window_attn_fwd_legacy_mma(q, k, v, o, heads: int, head_dim: int, window=(2, 6, 12), shift=(0, 0, 0),
+                                      scale: float = 0.0, stream=None, check: bool = True) -> int:
+    """The same call on the legacy mma.sync baseline kernel."""
+    return _attn("swin3d_window_attn_fwd_legacy_mma", q, k, v, o, heads, head_dim, window, shift, scale, stream,
+                 check)
+
+
+def _attn(entry, q, k, v, o, heads, head_dim, window, shift, scale, stream, check):
     lib = load_library()
     C = heads * head_dim
     B, T, H, W = q.shape[:4]
@@ -102,11 +118,11 @@ def swin3d_window_attn_fwd(q, k, v, o, heads: int, head_dim: int, window=(2, 6, 
         raise ValueError("q, k, v and o must have the same grid shape")
     ots = _token_stride(o, C)
     st = _stream_of(q) if stream is None else stream
-    rc = lib.swin3d_window_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), B, T, H, W,
+    rc = getattr(lib, entry)(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), B, T, H, W,
                                     *window, *shift, heads, head_dim, ts, ots, float(scale),
                                     _dtype_code(q), _dtype_code(o), st)
     if check and rc != S3W_OK:
-        raise S3WError(rc, "swin3d_window_attn_fwd")
+        raise S3WError(rc, entry)
     return rc
 
 
@@ -131,3 +147,8 @@ def poll_device_error(stream=None) -> int:
 
     st = torch.cuda.current_stream().cuda_stream if stream is None else stream
     return load_library().s3w_poll_device_error(st)
+
+
+def set_wait_limit_ns(ns: int) -> int:
+    """Set the kernels' bounded-wait limit (ns); returns the previous one."""
+    return int(load_library().s3w_set_wait_limit_ns(int(ns)))

@@ -45,7 +45,8 @@ int device_state(DeviceState** out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-long long g_spin_limit = 1ll << 26;  // bounded-wait iterations inside kernels
+// Time limit of every bounded wait inside the kernels (nanoseconds); 1 s by default.
+long long g_wait_limit_ns = 1000000000ll;
 
 }  // namespace
 
@@ -80,10 +81,15 @@ int s3w_poll_device_error(s3w_stream_t stream) {
   return S3W_OK;
 }
 
-int swin3d_window_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int T, int H, int W,
-                           int win_t, int win_h, int win_w, int shift_t, int shift_h, int shift_w, int heads,
-                           int head_dim, long long qkv_token_stride, long long o_token_stride, float scale,
-                           int in_dtype, int out_dtype, s3w_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Host-side checks shared by both attention entry points; fills the kernel geometry.
+int make_geometry(const void* q, const void* k, const void* v, void* o, int B, int T, int H, int W, int win_t,
+                  int win_h, int win_w, int shift_t, int shift_h, int shift_w, int heads, int head_dim,
+                  long long qkv_token_stride, long long o_token_stride, float scale, int in_dtype, int out_dtype,
+                  s3w::WinGeom* out) {
   if (!q || !k || !v || !o) return S3W_ERR_INVALID_ARG;
   if (B < 1 || T < 1 || H < 1 || W < 1 || heads < 1 || head_dim < 1) return S3W_ERR_INVALID_ARG;
   if (win_t < 1 || win_h < 1 || win_w < 1) return S3W_ERR_INVALID_ARG;
@@ -101,19 +107,17 @@ int swin3d_window_attn_fwd(const void* q, const void* k, const void* v, void* o,
   const int ob = out_dtype == S3W_F32 ? 4 : 2;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return S3W_ERR_MISALIGNED;
   if ((qkv_token_stride * 2) % 16 != 0 || (o_token_stride * ob) % 16 != 0) return S3W_ERR_MISALIGNED;
-  // padded grid sizes must stay in int range
+  // grid token indices are 32-bit inside the kernels; padded sizes must stay in int range
+  if (static_cast<long long>(B) * T * H * W > INT32_MAX) return S3W_ERR_UNSUPPORTED;
   const long long Pt = (T + win_t - 1) / win_t * static_cast<long long>(win_t);
   const long long Ph = (H + win_h - 1) / win_h * static_cast<long long>(win_h);
   const long long Pw = (W + win_w - 1) / win_w * static_cast<long long>(win_w);
   if (Pt > INT32_MAX / 2 || Ph > INT32_MAX / 2 || Pw > INT32_MAX / 2) return S3W_ERR_UNSUPPORTED;
   const long long per_sample = (Pt / win_t) * (Ph / win_h) * (Pw / win_w);
   if (per_sample > INT32_MAX) return S3W_ERR_UNSUPPORTED;
+  if (per_sample * B * heads > (1ll << 40)) return S3W_ERR_UNSUPPORTED;
 
-  DeviceState* ds = nullptr;
-  int rc = device_state(&ds);
-  if (rc != S3W_OK) return rc;
-
-  s3w::WinGeom g;
+  s3w::WinGeom& g = *out;
   g.B = B; g.T = T; g.H = H; g.W = W;
   g.wt = win_t; g.wh = win_h; g.ww = win_w;
   g.st = shift_t; g.sh = shift_h; g.sw = shift_w;
@@ -126,9 +130,48 @@ int swin3d_window_attn_fwd(const void* q, const void* k, const void* v, void* o,
   g.qkv_stride = qkv_token_stride;
   g.o_stride = o_token_stride;
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
-  g.scale_log2 = sc * 1.4426950408889634f;  // log2(e): softmax is evaluated with exp2
-  if (g.windows * heads > (1ll << 31) - 1) return S3W_ERR_UNSUPPORTED;
+  g.scale_log2 = sc * 1.4426950408889634f;  // log2(e): the softmax is evaluated with exp2
+  return S3W_OK;
+}
 
+}  // namespace
+
+extern "C" {
+
+long long s3w_set_wait_limit_ns(long long ns) {
+  const long long prev = g_wait_limit_ns;
+  g_wait_limit_ns = ns < 0 ? 0 : ns;
+  return prev;
+}
+
+int swin3d_window_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int T, int H, int W,
+                           int win_t, int win_h, int win_w, int shift_t, int shift_h, int shift_w, int heads,
+                           int head_dim, long long qkv_token_stride, long long o_token_stride, float scale,
+                           int in_dtype, int out_dtype, s3w_stream_t stream) {
+  s3w::WinGeom g;
+  int rc = make_geometry(q, k, v, o, B, T, H, W, win_t, win_h, win_w, shift_t, shift_h, shift_w, heads, head_dim,
+                         qkv_token_stride, o_token_stride, scale, in_dtype, out_dtype, &g);
+  if (rc != S3W_OK) return rc;
+  DeviceState* ds = nullptr;
+  rc = device_state(&ds);
+  if (rc != S3W_OK) return rc;
+  cudaError_t e = s3w::launch_window_attn_tc(g, q, k, v, o, out_dtype == S3W_F32, ds->err, g_wait_limit_ns,
+                                             ds->num_sms, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? S3W_OK : S3W_ERR_CUDA;
+}
+
+int swin3d_window_attn_fwd_legacy_mma(const void* q, const void* k, const void* v, void* o, int B, int T, int H,
+                                      int W, int win_t, int win_h, int win_w, int shift_t, int shift_h, int shift_w,
+                                      int heads, int head_dim, long long qkv_token_stride, long long o_token_stride,
+                                      float scale, int in_dtype, int out_dtype, s3w_stream_t stream) {
+  s3w::WinGeom g;
+  int rc = make_geometry(q, k, v, o, B, T, H, W, win_t, win_h, win_w, shift_t, shift_h, shift_w, heads, head_dim,
+                         qkv_token_stride, o_token_stride, scale, in_dtype, out_dtype, &g);
+  if (rc != S3W_OK) return rc;
+  if (g.windows * heads > (1ll << 31) - 1) return S3W_ERR_UNSUPPORTED;
+  DeviceState* ds = nullptr;
+  rc = device_state(&ds);
+  if (rc != S3W_OK) return rc;
   cudaError_t e = s3w::launch_window_attn_mma(g, q, k, v, o, out_dtype == S3W_F32,
                                               reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? S3W_OK : S3W_ERR_CUDA;

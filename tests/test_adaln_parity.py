@@ -32,9 +32,10 @@ def make_inputs(B, L, C, x_bf16, base, film_sigma=0.1):
 
 def check_bf16(got_bf16, ref):
     got = got_bf16.float().cpu().numpy().astype(np.float64)
-    # one bf16 step at the value's magnitude
+    # one bf16 step at the value's magnitude, plus the fp32 arithmetic error of the kernel
+    # (values near zero have tiny bf16 steps but keep the fp32 rounding of the larger terms)
     step = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 7)
-    assert np.all(np.abs(got - ref) <= step * 1.0001 + 1e-30)
+    assert np.all(np.abs(got - ref) <= step + 1e-5)
 
 
 SHAPES = [

@@ -20,12 +20,14 @@ pytestmark = pytest.mark.gpu
 SENTINEL = 8192.0   # exact in bf16; written into o before the call; must survive outside the real channels
 
 
-def run_gpu(dev_qkv, B, T, H, W, heads, hd, window, shift, out_dtype, o_extra=0):
+IMPLS = {"tcgen05": s3w.swin3d_window_attn_fwd, "legacy_mma": s3w.swin3d_window_attn_fwd_legacy_mma}
+
+
+def run_gpu(dev_qkv, B, T, H, W, heads, hd, window, shift, out_dtype, o_extra=0, impl="tcgen05"):
     C = heads * hd
     o = torch.full((B, T, H, W, C + o_extra), SENTINEL, dtype=out_dtype, device="cuda")
     q, k, v = dev_qkv
-    s3w.swin3d_window_attn_fwd(q[..., :C] if q.shape[-1] != C else q, k[..., :C] if k.shape[-1] != C else k,
-                               v[..., :C] if v.shape[-1] != C else v, o, heads, hd, window, shift)
+    IMPLS[impl](q, k, v, o, heads, hd, window, shift)
     torch.cuda.synchronize()
     assert s3w.poll_device_error() == 0
     return o
@@ -45,14 +47,27 @@ SMALL = [
 ]
 
 
+def case_id(c):
+    return f"B{c[0]}T{c[1]}H{c[2]}W{c[3]}h{c[4]}d{c[5]}w{c[6]}s{c[7]}"
+
+
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32], ids=["o_bf16", "o_f32"])
-@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"B{c[0]}T{c[1]}H{c[2]}W{c[3]}h{c[4]}d{c[5]}w{c[6]}s{c[7]}")
+@pytest.mark.parametrize("case", SMALL, ids=case_id)
 def test_small_grids_full_compare(cuda_ok, case, out_dtype):
+    _small_compare(case, out_dtype, "tcgen05")
+
+
+@pytest.mark.parametrize("case", [SMALL[0], SMALL[2], SMALL[5]], ids=case_id)
+def test_legacy_mma_baseline_small(cuda_ok, case):
+    _small_compare(case, torch.bfloat16, "legacy_mma")
+
+
+def _small_compare(case, out_dtype, impl):
     B, T, H, W, heads, hd, window, shift = case
     C = heads * hd
     bits, dev = make_qkv(B, T, H, W, C, base=10)
     ref = oracle.window_attn_grid(*bits, heads, hd, window, shift)
-    o = run_gpu(dev, B, T, H, W, heads, hd, window, shift, out_dtype, o_extra=8)
+    o = run_gpu(dev, B, T, H, W, heads, hd, window, shift, out_dtype, o_extra=8, impl=impl)
     got = o.float().cpu().numpy().astype(np.float64)
     assert np.all(got[..., C:] == SENTINEL), "channels beyond heads*head_dim were written"
     got = got[..., :C]
@@ -135,3 +150,28 @@ def test_full_size_sampled_windows(cuda_ok, case):
     assert torch.isfinite(o).all()
     vmax = dev[2].float().abs().amax()
     assert float(o.float().abs().amax()) <= float(vmax) * (1 + 2 ** -7)
+
+
+def test_bounded_wait_timeout_is_reported_and_context_survives(cuda_ok):
+    """A zero wait limit makes the kernel's first unsatisfied wait expire: the call must
+    unwind, report S3W_ERR_DEVICE_TIMEOUT through the error word, and leave the context
+    usable for a normal call right after."""
+    B, T, H, W, heads, hd, window, shift = 1, 4, 36, 72, 8, 64, (2, 6, 12), (1, 3, 6)
+    C = heads * hd
+    bits, dev = make_qkv(B, T, H, W, C, base=60)
+    o = torch.zeros((B, T, H, W, C), dtype=torch.bfloat16, device="cuda")
+    assert s3w.poll_device_error() == 0
+    prev = s3w.set_wait_limit_ns(0)
+    try:
+        s3w.swin3d_window_attn_fwd(*dev, o, heads, hd, window, shift)
+        status = s3w.poll_device_error()
+    finally:
+        s3w.set_wait_limit_ns(prev)
+    assert status == 5
+    assert s3w.poll_device_error() == 0          # the word was cleared by the poll
+    s3w.swin3d_window_attn_fwd(*dev, o, heads, hd, window, shift)
+    torch.cuda.synchronize()
+    assert s3w.poll_device_error() == 0
+    ref = oracle.window_attn_grid(*bits, heads, hd, window, shift)
+    mx, rl2 = attn_errors(o.float().cpu().numpy(), ref)
+    assert mx <= ATTN_MAX_ABS and rl2 <= ATTN_REL_L2, (mx, rl2)
