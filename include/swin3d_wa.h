@@ -123,8 +123,9 @@ int swin3d_window_attn_fwd_legacy_mma(const void* q, const void* k, const void* 
  *           (in-place update of the residual stream); no other overlap is allowed.
  * scale, shift  device fp32 [B][C] per-sample FiLM vectors, 16-byte aligned.
  * out       device, out_dtype, [B][L][C], 16-byte aligned.
- * B >= 1, tokens_per_sample >= 0 (0 launches nothing), C a multiple of 8 with
- * 8 <= C <= 4096; eps >= 0.
+ * B >= 1, tokens_per_sample >= 0, C a multiple of 8 with 8 <= C <= 4096; eps >= 0.
+ * With tokens_per_sample == 0 nothing is launched and the pointers are not used (they
+ * may be NULL).
  */
 int adaln_residual_fwd(const void* x, int x_dtype, const float* residual,
                        const float* scale, const float* shift,

@@ -180,11 +180,12 @@ int swin3d_window_attn_fwd_legacy_mma(const void* q, const void* k, const void* 
 int adaln_residual_fwd(const void* x, int x_dtype, const float* residual, const float* scale, const float* shift,
                        void* out, int out_dtype, int B, long long tokens_per_sample, int C, float eps,
                        s3w_stream_t stream) {
-  if (!x || !residual || !scale || !shift || !out) return S3W_ERR_INVALID_ARG;
   if (B < 1 || tokens_per_sample < 0 || C < 1 || !(eps >= 0.f) || std::isinf(eps)) return S3W_ERR_INVALID_ARG;
   if ((x_dtype != S3W_BF16 && x_dtype != S3W_F32) || (out_dtype != S3W_BF16 && out_dtype != S3W_F32))
     return S3W_ERR_INVALID_ARG;
   if (C % 8 != 0 || C > 4096) return S3W_ERR_UNSUPPORTED;
+  if (tokens_per_sample == 0) return S3W_OK;  // nothing to read or write; pointers unused
+  if (!x || !residual || !scale || !shift || !out) return S3W_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(residual) || !aligned16(scale) || !aligned16(shift) || !aligned16(out))
     return S3W_ERR_MISALIGNED;
   // out may alias residual exactly; any other overlap with residual is rejected
@@ -194,7 +195,6 @@ int adaln_residual_fwd(const void* x, int x_dtype, const float* residual, const 
   const long long ob = out_dtype == S3W_F32 ? 4 : 2;
   if (o0 != r0 && o0 < r0 + n * 4 && r0 < o0 + n * ob) return S3W_ERR_INVALID_ARG;
   if (B * tokens_per_sample > (1ll << 34)) return S3W_ERR_UNSUPPORTED;
-  if (tokens_per_sample == 0) return S3W_OK;
   DeviceState* ds = nullptr;
   int rc = device_state(&ds);
   if (rc != S3W_OK) return rc;

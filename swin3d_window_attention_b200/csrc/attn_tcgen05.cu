@@ -181,18 +181,20 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
       named_bar_sync(1, kProducerThreads);
       for (int r = p; r < kN; r += kProducerThreads)
         atomicOr(&tb.mask[tb.lab[r] * kMaskWords + (r >> 5)], 1u << (r & 31));
+      // Each thread copies one 16-byte column c of every (kProducerThreads / CH)-th row, for
+      // Q, K and V: a warp covers whole 128-byte head rows, so every request is coalesced.
       const uint32_t stage = sb + OFF_STAGE + s * kStageBytes;
-      for (int idx = p; idx < 3 * kN * CH; idx += kProducerThreads) {
-        const int tensor = idx / (kN * CH);
-        const int rem = idx - tensor * (kN * CH);
-        const int r = rem / CH;
-        const int c = rem - r * CH;
+      constexpr int kRowsPerPass = kProducerThreads / CH;
+      const int c = p % CH;
+      const long long coff = static_cast<long long>(head) * HD + c * 8;
+#pragma unroll 4
+      for (int r = p / CH; r < kN; r += kRowsPerPass) {
         const int tk = tb.tok[r];
-        const __nv_bfloat16* base = tensor == 0 ? q : (tensor == 1 ? k : v);
-        const __nv_bfloat16* src =
-            base + (tk < 0 ? 0ll : static_cast<long long>(tk) * g.qkv_stride + head * HD + c * 8);
-        const uint32_t dst = stage + tensor * kTileBytes + r * kRowBytes + ((c ^ (r & 7)) << 4);
-        cp_async_16_zfill(dst, src, tk >= 0);
+        const long long off = tk < 0 ? 0ll : static_cast<long long>(tk) * g.qkv_stride + coff;
+        const uint32_t dst = stage + r * kRowBytes + ((c ^ (r & 7)) << 4);
+        cp_async_16_zfill(dst, q + off, tk >= 0);
+        cp_async_16_zfill(dst + kTileBytes, k + off, tk >= 0);
+        cp_async_16_zfill(dst + 2 * kTileBytes, v + off, tk >= 0);
       }
       cp_async_commit();
       if (it > 0) {
@@ -332,60 +334,60 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
       return true;
     };
 
-    // Softmax of one S row already in registers; writes P (bf16) to shared memory.
-    // Returns 1 / rowsum.
-    auto softmax_row = [&](float (&sv)[kN], const uint32_t (&mw)[kMaskWords], bool full_tile, int row,
-                           uint32_t pb0, uint32_t pb1, uint32_t pb2, bool write) -> float {
-      float m = -INFINITY;
+    // Softmax of one S row held in registers: mask, row max, exp2, row sum (8 independent
+    // accumulators each, so the reductions are not one long dependency chain).  The
+    // probabilities stay in sv; returns 1 / rowsum.
+    auto softmax_row = [&](float (&sv)[kN], const uint32_t (&mw)[kMaskWords], bool full_tile) -> float {
+      float mx[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) mx[a] = -INFINITY;
       if (full_tile) {
 #pragma unroll
-        for (int j = 0; j < kN; ++j) m = fmaxf(m, sv[j]);
+        for (int j = 0; j < kN; ++j) mx[j & 7] = fmaxf(mx[j & 7], sv[j]);
       } else {
 #pragma unroll
         for (int j = 0; j < kN; ++j) {
           sv[j] = ((mw[j >> 5] >> (j & 31)) & 1u) ? sv[j] : -INFINITY;
-          m = fmaxf(m, sv[j]);
+          mx[j & 7] = fmaxf(mx[j & 7], sv[j]);
         }
       }
+      float m = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       if (m == -INFINITY) m = 0.f;
       const float mc = m * c;
-      float l = 0.f;
+      float ls[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) ls[a] = 0.f;
 #pragma unroll
       for (int j = 0; j < kN; ++j) {
         sv[j] = ex2(fmaf(sv[j], c, -mc));
-        l += sv[j];
+        ls[j & 7] += sv[j];
       }
-      if (write) {
+      const float l = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+      return l > 0.f ? 1.f / l : 0.f;
+    };
+    // Round a probability row to bf16 and store it as row `row` of the P operand (keys
+    // 0..63 and 64..127 in 128B-swizzled blocks, keys 128..143 in a 32B-swizzled block).
+    auto store_p_row = [&](const float (&sv)[kN], int row, uint32_t pb0, uint32_t pb1, uint32_t pb2) {
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
-          const uint32_t base = (b == 0 ? pb0 : pb1) + row * 128;
+      for (int b = 0; b < 2; ++b) {
+        const uint32_t base = (b == 0 ? pb0 : pb1) + row * 128;
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            const int j0 = 64 * b + 8 * ch;
-            uint4 u;
-            u.x = pack_bf16x2(sv[j0], sv[j0 + 1]);
-            u.y = pack_bf16x2(sv[j0 + 2], sv[j0 + 3]);
-            u.z = pack_bf16x2(sv[j0 + 4], sv[j0 + 5]);
-            u.w = pack_bf16x2(sv[j0 + 6], sv[j0 + 7]);
-            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(base + ((ch ^ (row & 7)) << 4)), "r"(u.x),
-                         "r"(u.y), "r"(u.z), "r"(u.w)
-                         : "memory");
-          }
-        }
-#pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          const int j0 = 128 + 8 * ch;
-          uint4 u;
-          u.x = pack_bf16x2(sv[j0], sv[j0 + 1]);
-          u.y = pack_bf16x2(sv[j0 + 2], sv[j0 + 3]);
-          u.z = pack_bf16x2(sv[j0 + 4], sv[j0 + 5]);
-          u.w = pack_bf16x2(sv[j0 + 6], sv[j0 + 7]);
-          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(pb2 + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4)),
-                       "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w)
+        for (int ch = 0; ch < 8; ++ch) {
+          const int j0 = 64 * b + 8 * ch;
+          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(base + ((ch ^ (row & 7)) << 4)),
+                       "r"(pack_bf16x2(sv[j0], sv[j0 + 1])), "r"(pack_bf16x2(sv[j0 + 2], sv[j0 + 3])),
+                       "r"(pack_bf16x2(sv[j0 + 4], sv[j0 + 5])), "r"(pack_bf16x2(sv[j0 + 6], sv[j0 + 7]))
                        : "memory");
         }
       }
-      return l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        const int j0 = 128 + 8 * ch;
+        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(pb2 + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4)),
+                     "r"(pack_bf16x2(sv[j0], sv[j0 + 1])), "r"(pack_bf16x2(sv[j0 + 2], sv[j0 + 3])),
+                     "r"(pack_bf16x2(sv[j0 + 4], sv[j0 + 5])), "r"(pack_bf16x2(sv[j0 + 6], sv[j0 + 7]))
+                     : "memory");
+      }
     };
 
     for (long long tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
@@ -438,13 +440,14 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
       }
       const bool mfull = ((mw[0] & mw[1] & mw[2] & mw[3]) == 0xffffffffu) && ((mw[4] & 0xffffu) == 0xffffu);
       const bool full_tile = __all_sync(0xffffffffu, mfull);
+      const float inv = softmax_row(sv, mw, full_tile);
       // P may only be overwritten once the previous tile's PV MMA has consumed it.
       ok = mbar_wait_bounded(p_empty, (it & 1) ^ 1, limit_ns);
       if (!__all_sync(0xffffffffu, ok)) {
         aborted = true;
         break;
       }
-      const float inv = softmax_row(sv, mw, full_tile, tid, sb + OFF_P0B0, sb + OFF_P0B1, sb + OFF_P0B2, true);
+      store_p_row(sv, tid, sb + OFF_P0B0, sb + OFF_P0B1, sb + OFF_P0B2);
       float inv_tail = 0.f;
       if (tail_warp) {
 #pragma unroll
@@ -456,7 +459,8 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
         mbar_arrive(s_empty);
         const bool tfull = ((tw[0] & tw[1] & tw[2] & tw[3]) == 0xffffffffu) && ((tw[4] & 0xffffu) == 0xffffu);
         const bool tfull_w = __all_sync(0xffffffffu, tfull || lane >= 16);
-        inv_tail = softmax_row(sv, tw, tfull_w, lane, sb + OFF_P1B0, sb + OFF_P1B1, sb + OFF_P1B2, lane < 16);
+        inv_tail = softmax_row(sv, tw, tfull_w);
+        if (lane < 16) store_p_row(sv, lane, sb + OFF_P1B0, sb + OFF_P1B1, sb + OFF_P1B2);
       }
       fence_proxy_async_smem();
       mbar_arrive(p_full);

@@ -99,6 +99,7 @@ def test_adaln_rejects_bad_arguments_on_host(over, expect):
 
 def test_adaln_zero_tokens_is_a_no_op():
     assert _adaln(L=0) == api.S3W_OK
+    assert _adaln(L=0, x=None, res=None, out=None) == api.S3W_OK
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
