@@ -7,7 +7,7 @@
 #include <cstdint>
 #include <mutex>
 
-#include "../../include/swin3d_wa.h"
+#include "swin3d_wa.h"
 #include "s3w_internal.h"
 
 namespace {

@@ -208,65 +208,73 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
     if (!stopped && it > 0) mbar_arrive(full_bar((it - 1) % kStages));
   } else if (warp == 4) {
     // ------------------------------------------------------------------ MMA issuer
+    // Issue order: S(t+1) goes out as soon as tile t+1 is loaded and S(t) has been read
+    // out of TMEM, before PV(t); the softmax warps then find S(t+1) ready when they finish
+    // tile t, and PV(t) runs underneath the softmax of tile t+1.
     constexpr uint32_t idesc_s = idesc_bf16_f32(128, kN, false, false);
     constexpr uint32_t idesc_o = idesc_bf16_f32(128, HD, false, true);
-    int it = 0;
     bool issued = false;
-    for (long long tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
-      const int s = it % kStages;
-      const uint32_t ph = (it / kStages) & 1;
-      int ok = 1;
-      if (lane == 0) {
-        ok = !*abort_flag;
-        ok = ok && mbar_wait_bounded(full_bar(s), ph, limit_ns) &&
-             mbar_wait_bounded(s_empty, (it & 1) ^ 1, limit_ns);
-        if (ok) {
-          tc_fence_after();
-          const uint32_t stage = sb + OFF_STAGE + s * kStageBytes;
-          const uint32_t qa = stage, ka = stage + kTileBytes, va = stage + 2 * kTileBytes;
+    auto issue_s = [&](int jt) -> bool {   // S(jt) = Q K^T of the tile in stage jt % kStages
+      const int s = jt % kStages;
+      if (!mbar_wait_bounded(full_bar(s), (jt / kStages) & 1, limit_ns)) return false;
+      if (!mbar_wait_bounded(s_empty, (jt & 1) ^ 1, limit_ns)) return false;
+      tc_fence_after();
+      const uint32_t qa = sb + OFF_STAGE + s * kStageBytes, ka = qa + kTileBytes;
 #pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk)
-            umma_bf16_ss(tmem + TM_S0, desc_kmajor_sw128(qa + kk * 32), desc_kmajor_sw128(ka + kk * 32), idesc_s,
-                         kk > 0);
-          if (has_tail) {
+      for (int kk = 0; kk < HD / 16; ++kk)
+        umma_bf16_ss(tmem + TM_S0, desc_kmajor_sw128(qa + kk * 32), desc_kmajor_sw128(ka + kk * 32), idesc_s, kk > 0);
+      if (has_tail) {
 #pragma unroll
-            for (int kk = 0; kk < HD / 16; ++kk)
-              umma_bf16_ss(tmem + TM_S1, desc_kmajor_sw128(qa + 128 * kRowBytes + kk * 32),
-                           desc_kmajor_sw128(ka + kk * 32), idesc_s, kk > 0);
-          }
-          umma_commit(s_full);
-          issued = true;
-          ok = mbar_wait_bounded(p_full, it & 1, limit_ns) && mbar_wait_bounded(o_empty, (it & 1) ^ 1, limit_ns);
-          if (ok) {
-            tc_fence_after();
+        for (int kk = 0; kk < HD / 16; ++kk)
+          umma_bf16_ss(tmem + TM_S1, desc_kmajor_sw128(qa + 128 * kRowBytes + kk * 32),
+                       desc_kmajor_sw128(ka + kk * 32), idesc_s, kk > 0);
+      }
+      umma_commit(s_full);
+      issued = true;
+      return true;
+    };
+    auto issue_pv = [&](int jt) -> bool {  // O(jt) = P V of the tile in stage jt % kStages
+      const int s = jt % kStages;
+      if (!mbar_wait_bounded(p_full, jt & 1, limit_ns)) return false;
+      if (!mbar_wait_bounded(o_empty, (jt & 1) ^ 1, limit_ns)) return false;
+      tc_fence_after();
+      const uint32_t va = sb + OFF_STAGE + s * kStageBytes + 2 * kTileBytes;
 #pragma unroll
-            for (int kk = 0; kk < kN / 16; ++kk) {
-              const uint64_t vd = desc_mnmajor_sw128(va + kk * 2048);
-              const uint64_t pd0 = kk < 8 ? desc_kmajor_sw128(sb + (kk < 4 ? OFF_P0B0 : OFF_P0B1) + (kk & 3) * 32)
-                                          : desc_kmajor_sw32(sb + OFF_P0B2);
-              umma_bf16_ss(tmem + TM_O0, pd0, vd, idesc_o, kk > 0);
-            }
-            if (has_tail) {
+      for (int kk = 0; kk < kN / 16; ++kk) {
+        const uint64_t vd = desc_mnmajor_sw128(va + kk * 2048);
+        const uint64_t pd0 = kk < 8 ? desc_kmajor_sw128(sb + (kk < 4 ? OFF_P0B0 : OFF_P0B1) + (kk & 3) * 32)
+                                    : desc_kmajor_sw32(sb + OFF_P0B2);
+        umma_bf16_ss(tmem + TM_O0, pd0, vd, idesc_o, kk > 0);
+      }
+      if (has_tail) {
 #pragma unroll
-              for (int kk = 0; kk < kN / 16; ++kk) {
-                const uint64_t vd = desc_mnmajor_sw128(va + kk * 2048);
-                const uint64_t pd1 = kk < 8 ? desc_kmajor_sw128(sb + (kk < 4 ? OFF_P1B0 : OFF_P1B1) + (kk & 3) * 32)
-                                            : desc_kmajor_sw32(sb + OFF_P1B2);
-                umma_bf16_ss(tmem + TM_O1, pd1, vd, idesc_o, kk > 0);
-              }
-            }
-            umma_commit(o_full);
-            umma_commit(p_empty);
-            umma_commit(empty_bar(s));
-          }
-        }
-        if (!ok) {
-          record_error(err, kStatusTimeout);
-          *abort_flag = 1;
+        for (int kk = 0; kk < kN / 16; ++kk) {
+          const uint64_t vd = desc_mnmajor_sw128(va + kk * 2048);
+          const uint64_t pd1 = kk < 8 ? desc_kmajor_sw128(sb + (kk < 4 ? OFF_P1B0 : OFF_P1B1) + (kk & 3) * 32)
+                                      : desc_kmajor_sw32(sb + OFF_P1B2);
+          umma_bf16_ss(tmem + TM_O1, pd1, vd, idesc_o, kk > 0);
         }
       }
+      umma_commit(o_full);
+      umma_commit(p_empty);
+      umma_commit(empty_bar(s));
+      return true;
+    };
+    int ok = 1;
+    if (lane == 0 && static_cast<long long>(blockIdx.x) < num_tiles) ok = issue_s(0);
+    int it = 0;
+    for (long long tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
+      if (lane == 0) {
+        ok = !*abort_flag;
+        if (ok && tile + gridDim.x < num_tiles) ok = issue_s(it + 1);
+        if (ok) ok = issue_pv(it);
+      }
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok && lane == 0) {
+      record_error(err, kStatusTimeout);
+      *abort_flag = 1;
     }
     // Drain: wait (bounded, independent of the test limit) until every MMA issued has
     // completed, so TMEM can be released.
