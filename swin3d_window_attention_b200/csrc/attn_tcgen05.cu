@@ -11,21 +11,25 @@
 //    Q/K/V rows straight from grid layout and the scatter of O rows straight back to grid
 //    layout, so none of them costs a global-memory pass.
 //
-// Work unit ("tile"): one (sample, window, head).  Per tile:
-//   producer warps 5-7  gather 3 x 144 token rows (16-byte cp.async, zero-fill for padded
-//                       slots) into a 3-stage shared-memory ring laid out as the 128-byte
-//                       swizzled operand layout of the tensor core; compute the slot ->
-//                       grid-token table, the Swin region label of every slot and one
-//                       key bitmask per label.
-//   MMA warp 4          S0 = Q[0:128] K^T and S1 = Q[128:144] K^T (M = 128, N = 144,
-//                       K = head_dim) into TMEM; after softmax, O0 = P0 V and O1 = P1 V
-//                       (M = 128, N = head_dim, K = 144, V read as an MN-major operand).
-//   softmax warps 0-3   thread t owns TMEM lane t = query row t: load the S row (144 fp32),
-//                       mask by region label / padding, exact row max, exp2, row sum, round
-//                       P to bf16 into shared memory; warp 0 also handles the 16 tail rows.
-//                       Then (one tile later, so the PV MMA overlaps the next softmax) load
-//                       the O row, scale by 1/rowsum, and store it to the query's original
-//                       grid position (padded slots are dropped).
+// Work unit ("tile"): one (sample, window, head).  Roles (warp -> SM sub-partition w % 4):
+//   softmax warps 0-3  thread t owns TMEM lane t = query row t of S0 = Q[0:128] K^T: load
+//                      the row (144 fp32), mask by region label / padding, exact row max,
+//                      exp2, row sum, P rounded to bf16 into shared memory.  Warp 0 also
+//                      owns the 16 tail rows (S1 = Q[128:144] K^T, TMEM lanes 0..15), read
+//                      with the 16x256b shape so all 32 lanes share them.  One tile later
+//                      (the PV MMA overlaps the next softmax) the same thread loads its O
+//                      row, scales by 1/rowsum and stores it to the query's original grid
+//                      position; padded slots are dropped.
+//   MMA warp 5         one thread issues S(t+1) as soon as tile t+1 is loaded and S(t) has
+//                      left TMEM, then PV(t) = P V once P(t) is in shared memory (V read as
+//                      an MN-major operand); completion is signalled by tcgen05.commit.
+//   producer warps 6-7 gather 3 x 144 token rows per tile with 16-byte cp.async (zero fill
+//                      for padded slots) into a 3-stage ring in the tensor core's 128-byte
+//                      swizzled K-major layout, plus the slot -> grid-token table, the
+//                      region label of every slot and one key bitmask per label.  Copy
+//                      completion arrives on the stage's mbarrier asynchronously, so the
+//                      producers run ahead as far as the ring allows.
+//   warp 4             idle after set-up.
 // Synchronisation is by mbarriers only; every wait is bounded by a time limit and a
 // timeout unwinds the whole CTA (error word set, copies drained, TMEM freed).
 #include <cuda_bf16.h>
@@ -39,7 +43,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kN = 144;          // tokens per window slot block (queries and keys)
+constexpr int kN = 144;          // slots per window tile (queries and keys)
 constexpr int kStages = 3;
 constexpr int kRowBytes = 128;   // one token row of one head in shared memory (swizzle width)
 constexpr int kTileBytes = kN * kRowBytes;          // 18432: one of Q / K / V
@@ -48,7 +52,9 @@ constexpr int kLabels = 28;      // 27 region labels + "padded"
 constexpr int kPadLabel = 27;
 constexpr int kMaskWords = 5;    // 144 key bits
 
-// Shared-memory map (offsets from a 1024-byte aligned base).
+// Shared-memory map (offsets from a 1024-byte aligned base).  The tail P blocks only hold
+// 16 rows; the rows 16..127 their M = 128 descriptors also cover fall on the buffers that
+// follow (valid memory, results of those rows are never used).
 constexpr int OFF_P1B0 = 0;        // tail P rows 0..15, keys 0..63   (128B swizzle)
 constexpr int OFF_P1B1 = 2048;     // tail P rows 0..15, keys 64..127 (128B swizzle)
 constexpr int OFF_P1B2 = 4096;     // tail P rows 0..15, keys 128..143 (32B swizzle)
@@ -76,16 +82,25 @@ constexpr uint32_t TM_S0 = 0, TM_S1 = 160, TM_O0 = 320, TM_O1 = 384;
 constexpr uint32_t kTmemCols = 512;
 
 constexpr int kThreads = 256;
-constexpr int kProducerThreads = 96;
+constexpr int kMmaWarp = 5;
+constexpr int kFirstProducerWarp = 6;
+constexpr int kProducerThreads = 64;
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-// Descriptors of the A/B operands (see the layout notes at the top of the file).
+// Operand descriptors.  K-major 128B swizzle: 8-row x 128-byte atoms, 1024 bytes apart.
+// K-major 32B swizzle: 8-row x 32-byte atoms, 256 bytes apart.  MN-major 128B swizzle (V,
+// whose rows are keys = the K dimension): 8-key x 64-element atoms, 1024 bytes apart.
 __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t addr) { return smem_desc(addr, 16, 1024, kSwizzle128B); }
 __device__ __forceinline__ uint64_t desc_kmajor_sw32(uint32_t addr) { return smem_desc(addr, 16, 256, kSwizzle32B); }
 __device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t addr) { return smem_desc(addr, 16, 1024, kSwizzle128B); }
+
+__device__ __forceinline__ bool mask_all(const uint32_t (&m)[kMaskWords]) {
+  return ((m[0] & m[1] & m[2] & m[3]) == 0xffffffffu) && ((m[4] & 0xffffu) == 0xffffu);
+}
+__device__ __forceinline__ bool mask_bit(const uint32_t (&m)[kMaskWords], int j) { return (m[j >> 5] >> (j & 31)) & 1u; }
 
 template <int HD, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -132,7 +147,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tmem_alloc(sb + OFF_MISC, kTmemCols);
     tmem_relinquish();
   }
@@ -141,12 +156,12 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp >= 5) {
+  if (warp >= kFirstProducerWarp) {
     // ------------------------------------------------------------------ producers
-    const int p = tid - 160;
+    const int p = tid - kFirstProducerWarp * 32;
     constexpr int CH = HD / 8;                   // 16-byte chunks per head row
+    constexpr int kRowsPerPass = kProducerThreads / CH;
     int it = 0;
-    bool stopped = false;
     for (long long tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int s = it % kStages;
       const uint32_t ph = (it / kStages) & 1;
@@ -159,10 +174,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
         *prod_stop = (!ok || *abort_flag) ? 1 : 0;
       }
       named_bar_sync(1, kProducerThreads);
-      if (*prod_stop) {
-        stopped = true;
-        break;
-      }
+      if (*prod_stop) break;
       const long long win = tile / g.heads;
       const int head = static_cast<int>(tile - win * g.heads);
       Table& tb = tables[s];
@@ -181,13 +193,12 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
       named_bar_sync(1, kProducerThreads);
       for (int r = p; r < kN; r += kProducerThreads)
         atomicOr(&tb.mask[tb.lab[r] * kMaskWords + (r >> 5)], 1u << (r & 31));
-      // Each thread copies one 16-byte column c of every (kProducerThreads / CH)-th row, for
-      // Q, K and V: a warp covers whole 128-byte head rows, so every request is coalesced.
+      // Each thread copies one 16-byte column c of every kRowsPerPass-th row, for Q, K and
+      // V: a warp covers whole 128-byte head rows, so every request is coalesced.
       const uint32_t stage = sb + OFF_STAGE + s * kStageBytes;
-      constexpr int kRowsPerPass = kProducerThreads / CH;
       const int c = p % CH;
       const long long coff = static_cast<long long>(head) * HD + c * 8;
-#pragma unroll 4
+#pragma unroll 6
       for (int r = p / CH; r < kN; r += kRowsPerPass) {
         const int tk = tb.tok[r];
         const long long off = tk < 0 ? 0ll : static_cast<long long>(tk) * g.qkv_stride + coff;
@@ -197,16 +208,11 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
         cp_async_16_zfill(dst + 2 * kTileBytes, v + off, tk >= 0);
       }
       cp_async_commit();
-      if (it > 0) {
-        cp_async_wait_1();
-        fence_proxy_async_smem();
-        mbar_arrive(full_bar((it - 1) % kStages));
-      }
+      cp_async_arrive(full_bar(s));   // fires when this thread's copies have landed
+      mbar_arrive(full_bar(s));       // table written (release)
     }
     cp_async_wait_0();
-    fence_proxy_async_smem();
-    if (!stopped && it > 0) mbar_arrive(full_bar((it - 1) % kStages));
-  } else if (warp == 4) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     // Issue order: S(t+1) goes out as soon as tile t+1 is loaded and S(t) has been read
     // out of TMEM, before PV(t); the softmax warps then find S(t+1) ready when they finish
@@ -218,6 +224,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
       const int s = jt % kStages;
       if (!mbar_wait_bounded(full_bar(s), (jt / kStages) & 1, limit_ns)) return false;
       if (!mbar_wait_bounded(s_empty, (jt & 1) ^ 1, limit_ns)) return false;
+      fence_proxy_async_smem();
       tc_fence_after();
       const uint32_t qa = sb + OFF_STAGE + s * kStageBytes, ka = qa + kTileBytes;
 #pragma unroll
@@ -262,6 +269,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
     };
     int ok = 1;
     if (lane == 0 && static_cast<long long>(blockIdx.x) < num_tiles) ok = issue_s(0);
+    ok = __shfl_sync(0xffffffffu, ok, 0);   // every lane takes the same path from here on
     int it = 0;
     for (long long tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
       if (lane == 0) {
@@ -271,7 +279,6 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
     }
-    ok = __shfl_sync(0xffffffffu, ok, 0);
     if (!ok && lane == 0) {
       record_error(err, kStatusTimeout);
       *abort_flag = 1;
@@ -283,94 +290,122 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
       if (!mbar_wait_bounded(drain_bar, 0, 2000000000ull)) record_error(err, kStatusTimeout);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 4) {
     // ------------------------------------------------------------------ softmax + epilogue
     const float c = g.scale_log2;
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const bool tail_warp = (warp == 0) && has_tail;
+    // Tail rows seen by this lane through the 16x256b shape: ra and ra + 8, columns
+    // 8j + 2*qd and 8j + 2*qd + 1 of every 8-column chunk j.
+    const int ra = lane >> 2, qd = lane & 3;
     int it = 0;
     // state of the previous tile, finished one iteration later
     bool have_prev = false;
-    int prev_it = 0, prev_head = 0, prev_tok = -1, prev_tok_tail = -1;
-    float prev_inv = 0.f, prev_inv_tail = 0.f;
+    int prev_it = 0, prev_head = 0, prev_tok = -1, prev_tok_a = -1, prev_tok_b = -1;
+    float prev_inv = 0.f, prev_inv_a = 0.f, prev_inv_b = 0.f;
     bool aborted = false;
 
-    auto epilogue = [&](int pit, int head, int tok, int tok_tail, float inv, float inv_tail) -> bool {
+    auto store8 = [&](int tk, int head, int col, const float* vals, float scl) {
+      // 8 consecutive outputs of one row starting at column `col`.
+      if constexpr (OUT_F32) {
+        float* dst = static_cast<float*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD + col;
+        if (g.o_rows_32b) {
+          uint32_t u[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) u[e] = __float_as_uint(vals[e] * scl);
+          st_global_v8(dst, u);
+        } else {
+          *reinterpret_cast<float4*>(dst) = make_float4(vals[0] * scl, vals[1] * scl, vals[2] * scl, vals[3] * scl);
+          *reinterpret_cast<float4*>(dst + 4) = make_float4(vals[4] * scl, vals[5] * scl, vals[6] * scl, vals[7] * scl);
+        }
+      } else {
+        __nv_bfloat16* dst =
+            static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD + col;
+        uint4 u;
+        u.x = pack_bf16x2(vals[0] * scl, vals[1] * scl);
+        u.y = pack_bf16x2(vals[2] * scl, vals[3] * scl);
+        u.z = pack_bf16x2(vals[4] * scl, vals[5] * scl);
+        u.w = pack_bf16x2(vals[6] * scl, vals[7] * scl);
+        *reinterpret_cast<uint4*>(dst) = u;
+      }
+    };
+    auto store2 = [&](int tk, int head, int col, float a, float b, float scl) {
+      if constexpr (OUT_F32) {
+        float* dst = static_cast<float*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD + col;
+        *reinterpret_cast<float2*>(dst) = make_float2(a * scl, b * scl);
+      } else {
+        __nv_bfloat16* dst =
+            static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD + col;
+        *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(a * scl, b * scl);
+      }
+    };
+
+    auto epilogue = [&](int pit, int head, int tok, int tok_a, int tok_b, float inv, float inv_a,
+                        float inv_b) -> bool {
       bool ok = mbar_wait_bounded(o_full, pit & 1, limit_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) return false;
       tc_fence_after();
-      float ov[HD], ov1[HD];
+      float ov[HD];
+      float ot[HD / 2];   // tail: (row ra, row ra+8) x 2 columns per 8-column chunk
 #pragma unroll
       for (int j = 0; j < HD / 16; ++j) tmem_ld16(tmem + lane_base + TM_O0 + 16 * j, ov + 16 * j);
       if (tail_warp) {
 #pragma unroll
-        for (int j = 0; j < HD / 16; ++j) tmem_ld16(tmem + lane_base + TM_O1 + 16 * j, ov1 + 16 * j);
+        for (int j = 0; j < HD / 8; ++j) tmem_ld_16x256b(tmem + TM_O1 + 8 * j, ot + 4 * j);
       }
       tmem_wait_ld();
 #pragma unroll
       for (int j = 0; j < HD / 16; ++j) reg_fence16(ov + 16 * j);
       if (tail_warp) {
 #pragma unroll
-        for (int j = 0; j < HD / 16; ++j) reg_fence16(ov1 + 16 * j);
+        for (int j = 0; j < HD / 8; ++j) reg_fence4(ot + 4 * j);
       }
       tc_fence_before();
       mbar_arrive(o_empty);
-      auto store_row = [&](const float* vals, float scl, int tk) {
-        if (tk < 0) return;
-        if constexpr (OUT_F32) {
-          float* dst = static_cast<float*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD;
+      if (tok >= 0) {
 #pragma unroll
-          for (int j = 0; j < HD; j += 4)
-            *reinterpret_cast<float4*>(dst + j) =
-                make_float4(vals[j] * scl, vals[j + 1] * scl, vals[j + 2] * scl, vals[j + 3] * scl);
-        } else {
-          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD;
+        for (int j = 0; j < HD; j += 8) store8(tok, head, j, ov + j, inv);
+      }
+      if (tail_warp) {
 #pragma unroll
-          for (int j = 0; j < HD; j += 8) {
-            uint4 u;
-            u.x = pack_bf16x2(vals[j] * scl, vals[j + 1] * scl);
-            u.y = pack_bf16x2(vals[j + 2] * scl, vals[j + 3] * scl);
-            u.z = pack_bf16x2(vals[j + 4] * scl, vals[j + 5] * scl);
-            u.w = pack_bf16x2(vals[j + 6] * scl, vals[j + 7] * scl);
-            *reinterpret_cast<uint4*>(dst + j) = u;
-          }
+        for (int j = 0; j < HD / 8; ++j) {
+          if (tok_a >= 0) store2(tok_a, head, 8 * j + 2 * qd, ot[4 * j], ot[4 * j + 1], inv_a);
+          if (tok_b >= 0) store2(tok_b, head, 8 * j + 2 * qd, ot[4 * j + 2], ot[4 * j + 3], inv_b);
         }
-      };
-      store_row(ov, inv, tok);
-      if (tail_warp && lane < 16) store_row(ov1, inv_tail, tok_tail);
+      }
       return true;
     };
 
-    // Softmax of one S row held in registers: mask, row max, exp2, row sum (8 independent
-    // accumulators each, so the reductions are not one long dependency chain).  The
-    // probabilities stay in sv; returns 1 / rowsum.
+    // Softmax of one S row held in registers (thread = row): mask, row max, exp2 and row
+    // sum, with independent partial accumulators and packed fp32x2 arithmetic.  The
+    // probabilities replace the logits in sv; returns 1 / rowsum.
     auto softmax_row = [&](float (&sv)[kN], const uint32_t (&mw)[kMaskWords], bool full_tile) -> float {
       float mx[8];
 #pragma unroll
       for (int a = 0; a < 8; ++a) mx[a] = -INFINITY;
-      if (full_tile) {
+      if (!full_tile) {
 #pragma unroll
-        for (int j = 0; j < kN; ++j) mx[j & 7] = fmaxf(mx[j & 7], sv[j]);
-      } else {
-#pragma unroll
-        for (int j = 0; j < kN; ++j) {
-          sv[j] = ((mw[j >> 5] >> (j & 31)) & 1u) ? sv[j] : -INFINITY;
-          mx[j & 7] = fmaxf(mx[j & 7], sv[j]);
-        }
+        for (int j = 0; j < kN; ++j) sv[j] = mask_bit(mw, j) ? sv[j] : -INFINITY;
       }
+#pragma unroll
+      for (int j = 0; j < kN; ++j) mx[j & 7] = fmaxf(mx[j & 7], sv[j]);
       float m = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       if (m == -INFINITY) m = 0.f;
-      const float mc = m * c;
-      float ls[8];
+      const float2 cc = make_float2(c, c), nm = make_float2(-m * c, -m * c);
+      float2 ls[4];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) ls[a] = 0.f;
+      for (int a = 0; a < 4; ++a) ls[a] = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int j = 0; j < kN; ++j) {
-        sv[j] = ex2(fmaf(sv[j], c, -mc));
-        ls[j & 7] += sv[j];
+      for (int j = 0; j < kN; j += 2) {
+        const float2 x = fma2(make_float2(sv[j], sv[j + 1]), cc, nm);
+        const float2 pr = make_float2(ex2(x.x), ex2(x.y));
+        ls[(j >> 1) & 3] = add2(ls[(j >> 1) & 3], pr);
+        sv[j] = pr.x;
+        sv[j + 1] = pr.y;
       }
-      const float l = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+      const float2 l2 = add2(add2(ls[0], ls[1]), add2(ls[2], ls[3]));
+      const float l = l2.x + l2.y;
       return l > 0.f ? 1.f / l : 0.f;
     };
     // Round a probability row to bf16 and store it as row `row` of the P operand (keys
@@ -397,6 +432,83 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
                      : "memory");
       }
     };
+    // The 16 tail rows, spread over the warp with the 16x256b shape: st[4j + 0..1] holds
+    // columns 8j + 2qd + {0, 1} of row ra, st[4j + 2..3] the same columns of row ra + 8.
+    // Row max / sum finish with two shuffles among the four lanes (qd = 0..3) that share a
+    // row.  Writes both rows' probabilities (bf16) into the tail P blocks and returns the
+    // two 1/rowsum values.
+    auto softmax_tail = [&](float* st, const uint32_t (&ma)[kMaskWords], const uint32_t (&mb)[kMaskWords],
+                            float& inv_a, float& inv_b) {
+      const bool full = __all_sync(0xffffffffu, mask_all(ma) && mask_all(mb));
+      if (!full) {
+#pragma unroll
+        for (int j = 0; j < kN / 8; ++j) {
+          const int col = 8 * j + 2 * qd;
+          st[4 * j + 0] = mask_bit(ma, col) ? st[4 * j + 0] : -INFINITY;
+          st[4 * j + 1] = mask_bit(ma, col + 1) ? st[4 * j + 1] : -INFINITY;
+          st[4 * j + 2] = mask_bit(mb, col) ? st[4 * j + 2] : -INFINITY;
+          st[4 * j + 3] = mask_bit(mb, col + 1) ? st[4 * j + 3] : -INFINITY;
+        }
+      }
+      float xa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      float xb[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int j = 0; j < kN / 8; ++j) {
+        xa[j & 3] = fmaxf(xa[j & 3], fmaxf(st[4 * j], st[4 * j + 1]));
+        xb[j & 3] = fmaxf(xb[j & 3], fmaxf(st[4 * j + 2], st[4 * j + 3]));
+      }
+      float m_a = fmaxf(fmaxf(xa[0], xa[1]), fmaxf(xa[2], xa[3]));
+      float m_b = fmaxf(fmaxf(xb[0], xb[1]), fmaxf(xb[2], xb[3]));
+      m_a = fmaxf(m_a, __shfl_xor_sync(0xffffffffu, m_a, 1));
+      m_a = fmaxf(m_a, __shfl_xor_sync(0xffffffffu, m_a, 2));
+      m_b = fmaxf(m_b, __shfl_xor_sync(0xffffffffu, m_b, 1));
+      m_b = fmaxf(m_b, __shfl_xor_sync(0xffffffffu, m_b, 2));
+      if (m_a == -INFINITY) m_a = 0.f;
+      if (m_b == -INFINITY) m_b = 0.f;
+      const float2 cc = make_float2(c, c);
+      const float2 na = make_float2(-m_a * c, -m_a * c), nb = make_float2(-m_b * c, -m_b * c);
+      float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < kN / 8; ++j) {
+        const float2 x = fma2(make_float2(st[4 * j], st[4 * j + 1]), cc, na);
+        const float2 y = fma2(make_float2(st[4 * j + 2], st[4 * j + 3]), cc, nb);
+        const float2 pa = make_float2(ex2(x.x), ex2(x.y));
+        const float2 pb = make_float2(ex2(y.x), ex2(y.y));
+        la = add2(la, pa);
+        lb = add2(lb, pb);
+        st[4 * j] = pa.x;
+        st[4 * j + 1] = pa.y;
+        st[4 * j + 2] = pb.x;
+        st[4 * j + 3] = pb.y;
+      }
+      float sa = la.x + la.y, sbm = lb.x + lb.y;
+      sa += __shfl_xor_sync(0xffffffffu, sa, 1);
+      sa += __shfl_xor_sync(0xffffffffu, sa, 2);
+      sbm += __shfl_xor_sync(0xffffffffu, sbm, 1);
+      sbm += __shfl_xor_sync(0xffffffffu, sbm, 2);
+      inv_a = sa > 0.f ? 1.f / sa : 0.f;
+      inv_b = sbm > 0.f ? 1.f / sbm : 0.f;
+      // bf16 pairs into the tail P blocks (4-byte stores; conflict-free across the warp)
+      const int rb = ra + 8;
+#pragma unroll
+      for (int j = 0; j < kN / 8; ++j) {
+        const uint32_t wa = pack_bf16x2(st[4 * j], st[4 * j + 1]);
+        const uint32_t wb = pack_bf16x2(st[4 * j + 2], st[4 * j + 3]);
+        uint32_t addr_a, addr_b;
+        if (j < 16) {
+          const uint32_t blk = sb + (j < 8 ? OFF_P1B0 : OFF_P1B1);
+          const int ch = j & 7;
+          addr_a = blk + ra * 128 + ((ch ^ (ra & 7)) << 4) + 4 * qd;
+          addr_b = blk + rb * 128 + ((ch ^ (rb & 7)) << 4) + 4 * qd;
+        } else {
+          const int ch = j - 16;
+          addr_a = sb + OFF_P1B2 + ra * 32 + ((ch ^ ((ra >> 2) & 1)) << 4) + 4 * qd;
+          addr_b = sb + OFF_P1B2 + rb * 32 + ((ch ^ ((rb >> 2) & 1)) << 4) + 4 * qd;
+        }
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr_a), "r"(wa) : "memory");
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr_b), "r"(wb) : "memory");
+      }
+    };
 
     for (long long tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int s = it % kStages;
@@ -414,19 +526,22 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
       const int head = static_cast<int>(tile - win * g.heads);
       const Table& tb = tables[s];
       const int tok = tb.tok[tid];
-      uint32_t mw[kMaskWords], tw[kMaskWords];
+      uint32_t mw[kMaskWords], ma[kMaskWords], mb[kMaskWords];
       {
         const int lab = tb.lab[tid];
 #pragma unroll
         for (int w = 0; w < kMaskWords; ++w) mw[w] = tb.mask[lab * kMaskWords + w];
       }
-      int tok_tail = -1;
+      int tok_a = -1, tok_b = -1;
       if (tail_warp) {
-        const int r = 128 + (lane & 15);
-        tok_tail = lane < 16 ? tb.tok[r] : -1;
-        const int lab = tb.lab[r];
+        tok_a = tb.tok[128 + ra];
+        tok_b = tb.tok[136 + ra];
+        const int la = tb.lab[128 + ra], lb = tb.lab[136 + ra];
 #pragma unroll
-        for (int w = 0; w < kMaskWords; ++w) tw[w] = tb.mask[lab * kMaskWords + w];
+        for (int w = 0; w < kMaskWords; ++w) {
+          ma[w] = tb.mask[la * kMaskWords + w];
+          mb[w] = tb.mask[lb * kMaskWords + w];
+        }
       }
       mbar_arrive(empty_bar(s));
 
@@ -444,11 +559,12 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
       for (int j = 0; j < kN / 16; ++j) reg_fence16(sv + 16 * j);
       if (!tail_warp) {
         tc_fence_before();
-        mbar_arrive(s_empty);
+        mbar_arrive(s_empty);   // S(t) is in registers: the next tile's S may be written
       }
-      const bool mfull = ((mw[0] & mw[1] & mw[2] & mw[3]) == 0xffffffffu) && ((mw[4] & 0xffffu) == 0xffffu);
-      const bool full_tile = __all_sync(0xffffffffu, mfull);
+
+      const bool full_tile = __all_sync(0xffffffffu, mask_all(mw));
       const float inv = softmax_row(sv, mw, full_tile);
+      float inv_a = 0.f, inv_b = 0.f;
       // P may only be overwritten once the previous tile's PV MMA has consumed it.
       ok = mbar_wait_bounded(p_empty, (it & 1) ^ 1, limit_ns);
       if (!__all_sync(0xffffffffu, ok)) {
@@ -456,24 +572,22 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
         break;
       }
       store_p_row(sv, tid, sb + OFF_P0B0, sb + OFF_P0B1, sb + OFF_P0B2);
-      float inv_tail = 0.f;
       if (tail_warp) {
+        // the tail rows are loaded only now, so that the main row's registers are free
+        float st[kN / 2];
 #pragma unroll
-        for (int j = 0; j < kN / 16; ++j) tmem_ld16(tmem + lane_base + TM_S1 + 16 * j, sv + 16 * j);
+        for (int j = 0; j < kN / 8; ++j) tmem_ld_16x256b(tmem + TM_S1 + 8 * j, st + 4 * j);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < kN / 16; ++j) reg_fence16(sv + 16 * j);
+        for (int j = 0; j < kN / 8; ++j) reg_fence4(st + 4 * j);
         tc_fence_before();
         mbar_arrive(s_empty);
-        const bool tfull = ((tw[0] & tw[1] & tw[2] & tw[3]) == 0xffffffffu) && ((tw[4] & 0xffffu) == 0xffffu);
-        const bool tfull_w = __all_sync(0xffffffffu, tfull || lane >= 16);
-        inv_tail = softmax_row(sv, tw, tfull_w);
-        if (lane < 16) store_p_row(sv, lane, sb + OFF_P1B0, sb + OFF_P1B1, sb + OFF_P1B2);
+        softmax_tail(st, ma, mb, inv_a, inv_b);
       }
       fence_proxy_async_smem();
       mbar_arrive(p_full);
       if (have_prev) {
-        if (!epilogue(prev_it, prev_head, prev_tok, prev_tok_tail, prev_inv, prev_inv_tail)) {
+        if (!epilogue(prev_it, prev_head, prev_tok, prev_tok_a, prev_tok_b, prev_inv, prev_inv_a, prev_inv_b)) {
           aborted = true;
           have_prev = false;
           break;
@@ -483,12 +597,15 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
       prev_it = it;
       prev_head = head;
       prev_tok = tok;
-      prev_tok_tail = tok_tail;
+      prev_tok_a = tok_a;
+      prev_tok_b = tok_b;
       prev_inv = inv;
-      prev_inv_tail = inv_tail;
+      prev_inv_a = inv_a;
+      prev_inv_b = inv_b;
     }
     if (have_prev && !aborted) {
-      if (!epilogue(prev_it, prev_head, prev_tok, prev_tok_tail, prev_inv, prev_inv_tail)) aborted = true;
+      if (!epilogue(prev_it, prev_head, prev_tok, prev_tok_a, prev_tok_b, prev_inv, prev_inv_a, prev_inv_b))
+        aborted = true;
     }
     if (aborted) {
       if (lane == 0) record_error(err, kStatusTimeout);
@@ -499,7 +616,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 4) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
 template <int HD, bool OUT_F32>

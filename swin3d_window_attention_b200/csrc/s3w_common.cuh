@@ -32,6 +32,7 @@ struct WinGeom {
   long long qkv_stride;    // elements between tokens in q/k/v
   long long o_stride;      // elements between tokens in o
   float scale_log2;        // scale * log2(e)
+  int o_rows_32b;          // 1 if every output row start is 32-byte aligned
 };
 
 // Per-axis region label on the shifted, padded grid.

@@ -94,6 +94,19 @@ def test_fused_qkv_buffer_token_stride(cuda_ok):
     assert mx <= ATTN_MAX_ABS and rl2 <= ATTN_REL_L2, (mx, rl2)
 
 
+def test_f32_output_rows_only_16_byte_aligned(cuda_ok):
+    """o token stride C + 4 floats: rows start on 16- but not 32-byte boundaries."""
+    B, T, H, W, heads, hd, window, shift = 1, 4, 13, 25, 2, 64, (2, 6, 12), (1, 3, 6)
+    C = heads * hd
+    bits, dev = make_qkv(B, T, H, W, C, base=25)
+    o = run_gpu(dev, B, T, H, W, heads, hd, window, shift, torch.float32, o_extra=4)
+    got = o.cpu().numpy().astype(np.float64)
+    assert np.all(got[..., C:] == SENTINEL)
+    ref = oracle.window_attn_grid(*bits, heads, hd, window, shift)
+    mx, rl2 = attn_errors(got[..., :C], ref)
+    assert mx <= ATTN_MAX_ABS and rl2 <= ATTN_REL_L2, (mx, rl2)
+
+
 def test_explicit_scale(cuda_ok):
     B, T, H, W, heads, hd, window, shift = 1, 2, 12, 24, 2, 64, (2, 6, 12), (1, 3, 6)
     C = heads * hd
