@@ -115,7 +115,7 @@ int make_geometry(const void* q, const void* k, const void* v, void* o, int B, i
   if (Pt > INT32_MAX / 2 || Ph > INT32_MAX / 2 || Pw > INT32_MAX / 2) return S3W_ERR_UNSUPPORTED;
   const long long per_sample = (Pt / win_t) * (Ph / win_h) * (Pw / win_w);
   if (per_sample > INT32_MAX) return S3W_ERR_UNSUPPORTED;
-  if (per_sample * B * heads > (1ll << 40)) return S3W_ERR_UNSUPPORTED;
+  if (per_sample * B * heads > INT32_MAX) return S3W_ERR_UNSUPPORTED;  // tile index is 32-bit
 
   s3w::WinGeom& g = *out;
   g.B = B; g.T = T; g.H = H; g.W = W;

@@ -25,8 +25,9 @@
 //                      an MN-major operand); completion is signalled by tcgen05.commit.
 //   producer warps 6-7 gather 3 x 144 token rows per tile with 16-byte cp.async (zero fill
 //                      for padded slots) into a 3-stage ring in the tensor core's 128-byte
-//                      swizzled K-major layout, plus the slot -> grid-token table, the
-//                      region label of every slot and one key bitmask per label.  Copy
+//                      swizzled K-major layout, plus the slot -> grid-token table, a
+//                      bitmask of the real slots and the window's "last along a shifted
+//                      axis" flags (the mask of a query follows from these).  Copy
 //                      completion arrives on the stage's mbarrier asynchronously, so the
 //                      producers run ahead as far as the ring allows.
 //   warp 4             idle after set-up.
@@ -48,8 +49,6 @@ constexpr int kStages = 3;
 constexpr int kRowBytes = 128;   // one token row of one head in shared memory (swizzle width)
 constexpr int kTileBytes = kN * kRowBytes;          // 18432: one of Q / K / V
 constexpr int kStageBytes = 3 * kTileBytes;         // 55296
-constexpr int kLabels = 28;      // 27 region labels + "padded"
-constexpr int kPadLabel = 27;
 constexpr int kMaskWords = 5;    // 144 key bits
 
 // Shared-memory map (offsets from a 1024-byte aligned base).  The tail P blocks only hold
@@ -64,13 +63,24 @@ constexpr int OFF_P0B2 = OFF_P0B1 + 16384;   // keys 128..143, 32B swizzle, 4 KB
 constexpr int OFF_STAGE = OFF_P0B2 + 4096;   // 41984 (1024-aligned)
 constexpr int OFF_TABLE = OFF_STAGE + kStages * kStageBytes;
 
+// Per tile: grid token of every slot (-1 = padded), which slots are real, and along which
+// shifted axes the window is the last one (where Swin's mask splits it in two regions).
 struct Table {
-  int tok[kN];                       // flat grid token of each slot, -1 = padded
-  uint32_t mask[kLabels * kMaskWords];
-  uint8_t lab[kN];                   // region label of each slot (kPadLabel = padded)
+  int tok[kN];
+  uint32_t real[kMaskWords];
+  uint32_t last;
 };
 constexpr int kTableBytes = (static_cast<int>(sizeof(Table)) + 15) & ~15;
-constexpr int OFF_BARS = OFF_TABLE + kStages * kTableBytes;
+// Per CTA, the same for every tile: the (t, h, w) offset of each slot inside the window
+// and, per axis, the slots of the wrapped-around part (offset >= window - shift).  A query
+// in the last window along a shifted axis may only see keys on its own side of that split.
+struct SlotConst {
+  uint32_t coord[kN];                 // rt | rh << 8 | rw << 16
+  uint32_t hi[3][kMaskWords];
+  uint32_t all[kMaskWords];           // slots < N
+};
+constexpr int OFF_SLOTC = OFF_TABLE + kStages * kTableBytes;
+constexpr int OFF_BARS = OFF_SLOTC + ((static_cast<int>(sizeof(SlotConst)) + 15) & ~15);
 // barriers: full[3], empty[3], s_full, s_empty, p_full, p_empty, o_full, o_empty, drain
 constexpr int kNumBars = 2 * kStages + 7;
 constexpr int OFF_MISC = OFF_BARS + kNumBars * 8;   // tmem address, abort flag, producer stop
@@ -97,6 +107,20 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t addr) { return sm
 __device__ __forceinline__ uint64_t desc_kmajor_sw32(uint32_t addr) { return smem_desc(addr, 16, 256, kSwizzle32B); }
 __device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t addr) { return smem_desc(addr, 16, 1024, kSwizzle128B); }
 
+// Keys visible to a query in slot r: real slots, restricted on every axis where the window
+// is the last one of a shifted axis to the query's side of the wrap-around split.
+// hi_bits: bit a set iff slot r is in the wrapped-around part of axis a.
+__device__ __forceinline__ void build_mask(const Table& tb, const SlotConst& sc, uint32_t last, uint32_t hi_bits,
+                                           uint32_t (&m)[kMaskWords]) {
+#pragma unroll
+  for (int w = 0; w < kMaskWords; ++w) {
+    uint32_t x = tb.real[w];
+#pragma unroll
+    for (int a = 0; a < 3; ++a)
+      if ((last >> a) & 1u) x &= ((hi_bits >> a) & 1u) ? sc.hi[a][w] : (sc.all[w] & ~sc.hi[a][w]);
+    m[w] = x;
+  }
+}
 __device__ __forceinline__ bool mask_all(const uint32_t (&m)[kMaskWords]) {
   return ((m[0] & m[1] & m[2] & m[3]) == 0xffffffffu) && ((m[4] & 0xffffu) == 0xffffu);
 }
@@ -147,6 +171,30 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
     fence_barrier_init();
     fence_proxy_async_smem();
   }
+  SlotConst* slotc = reinterpret_cast<SlotConst*>(sm + OFF_SLOTC);
+  {
+    auto split_at = [&](int a) { return a == 0 ? g.wt - g.st : (a == 1 ? g.wh - g.sh : g.ww - g.sw); };
+    auto slot_off = [&](int r, int a) {   // offset of slot r along axis a
+      return a == 2 ? r % g.ww : (a == 1 ? (r / g.ww) % g.wh : r / (g.ww * g.wh));
+    };
+    if (tid < kN) slotc->coord[tid] = tid < g.N ? (slot_off(tid, 0) | slot_off(tid, 1) << 8 | slot_off(tid, 2) << 16) : 0u;
+    if (tid >= 160 && tid < 160 + 3 * kMaskWords) {
+      const int a = (tid - 160) / kMaskWords, w = (tid - 160) % kMaskWords;
+      uint32_t bits = 0;
+      for (int b = 0; b < 32; ++b) {
+        const int r = 32 * w + b;
+        if (r < g.N && slot_off(r, a) >= split_at(a)) bits |= 1u << b;
+      }
+      slotc->hi[a][w] = bits;
+    }
+    if (tid >= 192 && tid < 192 + kMaskWords) {
+      const int w = tid - 192;
+      uint32_t bits = 0;
+      for (int b = 0; b < 32; ++b)
+        if (32 * w + b < g.N) bits |= 1u << b;
+      slotc->all[w] = bits;
+    }
+  }
   if (warp == kMmaWarp) {
     tmem_alloc(sb + OFF_MISC, kTmemCols);
     tmem_relinquish();
@@ -175,24 +223,44 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
       }
       named_bar_sync(1, kProducerThreads);
       if (*prod_stop) break;
-      const long long win = tile / g.heads;
-      const int head = static_cast<int>(tile - win * g.heads);
+      // Window coordinates (32-bit: the tile count is checked on the host).
+      const int t32 = static_cast<int>(tile);
+      const int win = t32 / g.heads;
+      const int head = t32 - win * g.heads;
+      const int per = g.nwt * g.nwh * g.nww;
+      const int bsmp = win / per;
+      int rem = win - bsmp * per;
+      const int iw = rem % g.nww;
+      rem /= g.nww;
+      const int ih = rem % g.nwh;
+      const int itw = rem / g.nwh;
+      // shifted padded coordinate of slot offset 0, plus the shift: slot (rt, rh, rw) of
+      // this window holds the original coordinate (base + offset) mod P on each axis.
+      const int bt = itw * g.wt + g.st, bh = ih * g.wh + g.sh, bw = iw * g.ww + g.sw;
+      auto resolve = [&](int r) -> int {   // grid token of slot r, -1 if padded
+        if (r >= g.N) return -1;
+        const uint32_t cd = slotc->coord[r];
+        int t = bt + static_cast<int>(cd & 0xffu);
+        int h = bh + static_cast<int>((cd >> 8) & 0xffu);
+        int w = bw + static_cast<int>(cd >> 16);
+        t -= t >= g.Pt ? g.Pt : 0;
+        h -= h >= g.Ph ? g.Ph : 0;
+        w -= w >= g.Pw ? g.Pw : 0;
+        if (t >= g.T || h >= g.H || w >= g.W) return -1;
+        return ((bsmp * g.T + t) * g.H + h) * g.W + w;
+      };
       Table& tb = tables[s];
-      for (int r = p; r < kN; r += kProducerThreads) {
-        int lab = kPadLabel;
-        long long tk = -1;
-        if (r < g.N) {
-          int l2;
-          tk = slot_token(g, win, r, &l2);
-          if (tk >= 0) lab = l2;
+      {
+        const int pw = p >> 5;
+        for (int wd = pw; wd < kMaskWords; wd += kProducerThreads / 32) {
+          const int r = 32 * wd + lane;
+          const unsigned m = __ballot_sync(0xffffffffu, r < kN && resolve(r) >= 0);
+          if (lane == 0) tb.real[wd] = m;
         }
-        tb.tok[r] = static_cast<int>(tk);
-        tb.lab[r] = static_cast<uint8_t>(lab);
+        if (p == 0)
+          tb.last = ((itw == g.nwt - 1 && g.st > 0) ? 1u : 0u) | ((ih == g.nwh - 1 && g.sh > 0) ? 2u : 0u) |
+                    ((iw == g.nww - 1 && g.sw > 0) ? 4u : 0u);
       }
-      for (int w = p; w < kLabels * kMaskWords; w += kProducerThreads) tb.mask[w] = 0u;
-      named_bar_sync(1, kProducerThreads);
-      for (int r = p; r < kN; r += kProducerThreads)
-        atomicOr(&tb.mask[tb.lab[r] * kMaskWords + (r >> 5)], 1u << (r & 31));
       // Each thread copies one 16-byte column c of every kRowsPerPass-th row, for Q, K and
       // V: a warp covers whole 128-byte head rows, so every request is coalesced.
       const uint32_t stage = sb + OFF_STAGE + s * kStageBytes;
@@ -200,7 +268,8 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
       const long long coff = static_cast<long long>(head) * HD + c * 8;
 #pragma unroll 6
       for (int r = p / CH; r < kN; r += kRowsPerPass) {
-        const int tk = tb.tok[r];
+        const int tk = resolve(r);
+        if (c == 0) tb.tok[r] = tk;
         const long long off = tk < 0 ? 0ll : static_cast<long long>(tk) * g.qkv_stride + coff;
         const uint32_t dst = stage + r * kRowBytes + ((c ^ (r & 7)) << 4);
         cp_async_16_zfill(dst, q + off, tk >= 0);
@@ -298,6 +367,13 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
     // Tail rows seen by this lane through the 16x256b shape: ra and ra + 8, columns
     // 8j + 2*qd and 8j + 2*qd + 1 of every 8-column chunk j.
     const int ra = lane >> 2, qd = lane & 3;
+    auto hi_bits_of = [&](int r) -> uint32_t {
+      uint32_t h = 0;
+#pragma unroll
+      for (int a = 0; a < 3; ++a) h |= ((slotc->hi[a][r >> 5] >> (r & 31)) & 1u) << a;
+      return h;
+    };
+    const uint32_t my_hi = hi_bits_of(tid), hi_a = hi_bits_of(128 + ra), hi_b = hi_bits_of(136 + ra);
     int it = 0;
     // state of the previous tile, finished one iteration later
     bool have_prev = false;
@@ -389,7 +465,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
         for (int j = 0; j < kN; ++j) sv[j] = mask_bit(mw, j) ? sv[j] : -INFINITY;
       }
 #pragma unroll
-      for (int j = 0; j < kN; ++j) mx[j & 7] = fmaxf(mx[j & 7], sv[j]);
+      for (int j = 0; j < kN; j += 2) mx[(j >> 1) & 7] = max3(mx[(j >> 1) & 7], sv[j], sv[j + 1]);
       float m = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       if (m == -INFINITY) m = 0.f;
       const float2 cc = make_float2(c, c), nm = make_float2(-m * c, -m * c);
@@ -418,8 +494,8 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
         for (int ch = 0; ch < 8; ++ch) {
           const int j0 = 64 * b + 8 * ch;
           asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(base + ((ch ^ (row & 7)) << 4)),
-                       "r"(pack_bf16x2(sv[j0], sv[j0 + 1])), "r"(pack_bf16x2(sv[j0 + 2], sv[j0 + 3])),
-                       "r"(pack_bf16x2(sv[j0 + 4], sv[j0 + 5])), "r"(pack_bf16x2(sv[j0 + 6], sv[j0 + 7]))
+                       "r"(pack_bf16x2_int(sv[j0], sv[j0 + 1])), "r"(pack_bf16x2_int(sv[j0 + 2], sv[j0 + 3])),
+                       "r"(pack_bf16x2_int(sv[j0 + 4], sv[j0 + 5])), "r"(pack_bf16x2_int(sv[j0 + 6], sv[j0 + 7]))
                        : "memory");
         }
       }
@@ -427,8 +503,8 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
       for (int ch = 0; ch < 2; ++ch) {
         const int j0 = 128 + 8 * ch;
         asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(pb2 + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4)),
-                     "r"(pack_bf16x2(sv[j0], sv[j0 + 1])), "r"(pack_bf16x2(sv[j0 + 2], sv[j0 + 3])),
-                     "r"(pack_bf16x2(sv[j0 + 4], sv[j0 + 5])), "r"(pack_bf16x2(sv[j0 + 6], sv[j0 + 7]))
+                     "r"(pack_bf16x2_int(sv[j0], sv[j0 + 1])), "r"(pack_bf16x2_int(sv[j0 + 2], sv[j0 + 3])),
+                     "r"(pack_bf16x2_int(sv[j0 + 4], sv[j0 + 5])), "r"(pack_bf16x2_int(sv[j0 + 6], sv[j0 + 7]))
                      : "memory");
       }
     };
@@ -454,8 +530,8 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
       float xb[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int j = 0; j < kN / 8; ++j) {
-        xa[j & 3] = fmaxf(xa[j & 3], fmaxf(st[4 * j], st[4 * j + 1]));
-        xb[j & 3] = fmaxf(xb[j & 3], fmaxf(st[4 * j + 2], st[4 * j + 3]));
+        xa[j & 3] = max3(xa[j & 3], st[4 * j], st[4 * j + 1]);
+        xb[j & 3] = max3(xb[j & 3], st[4 * j + 2], st[4 * j + 3]);
       }
       float m_a = fmaxf(fmaxf(xa[0], xa[1]), fmaxf(xa[2], xa[3]));
       float m_b = fmaxf(fmaxf(xb[0], xb[1]), fmaxf(xb[2], xb[3]));
@@ -492,8 +568,8 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
       const int rb = ra + 8;
 #pragma unroll
       for (int j = 0; j < kN / 8; ++j) {
-        const uint32_t wa = pack_bf16x2(st[4 * j], st[4 * j + 1]);
-        const uint32_t wb = pack_bf16x2(st[4 * j + 2], st[4 * j + 3]);
+        const uint32_t wa = pack_bf16x2_int(st[4 * j], st[4 * j + 1]);
+        const uint32_t wb = pack_bf16x2_int(st[4 * j + 2], st[4 * j + 3]);
         uint32_t addr_a, addr_b;
         if (j < 16) {
           const uint32_t blk = sb + (j < 8 ? OFF_P1B0 : OFF_P1B1);
@@ -526,22 +602,15 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
       const int head = static_cast<int>(tile - win * g.heads);
       const Table& tb = tables[s];
       const int tok = tb.tok[tid];
+      const uint32_t last = tb.last;
       uint32_t mw[kMaskWords], ma[kMaskWords], mb[kMaskWords];
-      {
-        const int lab = tb.lab[tid];
-#pragma unroll
-        for (int w = 0; w < kMaskWords; ++w) mw[w] = tb.mask[lab * kMaskWords + w];
-      }
+      build_mask(tb, *slotc, last, my_hi, mw);
       int tok_a = -1, tok_b = -1;
       if (tail_warp) {
         tok_a = tb.tok[128 + ra];
         tok_b = tb.tok[136 + ra];
-        const int la = tb.lab[128 + ra], lb = tb.lab[136 + ra];
-#pragma unroll
-        for (int w = 0; w < kMaskWords; ++w) {
-          ma[w] = tb.mask[la * kMaskWords + w];
-          mb[w] = tb.mask[lb * kMaskWords + w];
-        }
+        build_mask(tb, *slotc, last, hi_a, ma);
+        build_mask(tb, *slotc, last, hi_b, mb);
       }
       mbar_arrive(empty_bar(s));
 

@@ -167,6 +167,22 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
   return r;
 }
 
+// max of three fp32 values in one instruction.
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Two finite fp32 values -> packed bf16x2, rounded to nearest with ties away from zero,
+// on the integer pipe (add half an ulp of bf16 to the bit pattern, keep the upper halves).
+// Differs from round-to-nearest-even only on exact ties.
+__device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
+  const uint32_t a = __float_as_uint(lo) + 0x8000u;
+  const uint32_t b = __float_as_uint(hi) + 0x8000u;
+  return __byte_perm(a, b, 0x7632);
+}
+
 // 32-byte global store (one full sector per thread).
 __device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&v)[8]) {
   asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v[0]), "r"(v[1]), "r"(v[2]),
