@@ -23,18 +23,24 @@
 //   MMA warp 5         one thread issues S(t+1) as soon as tile t+1 is loaded and S(t) has
 //                      left TMEM, then PV(t) = P V once P(t) is in shared memory (V read as
 //                      an MN-major operand); completion is signalled by tcgen05.commit.
-//   producer warps 6-7 gather 3 x 144 token rows per tile with 16-byte cp.async (zero fill
-//                      for padded slots) into a 3-stage ring in the tensor core's 128-byte
-//                      swizzled K-major layout, plus the slot -> grid-token table, a
-//                      bitmask of the real slots and the window's "last along a shifted
-//                      axis" flags (the mask of a query follows from these).  Copy
-//                      completion arrives on the stage's mbarrier asynchronously, so the
-//                      producers run ahead as far as the ring allows.
+//   producer warps 6-7 one thread loads the tile's Q, K and V with TMA: one box per
+//                      (t, h) run of window tokens per tensor (two where the run wraps
+//                      around the W seam), straight from grid layout into a 3-stage ring in
+//                      the tensor core's 128-byte swizzled K-major layout; padded
+//                      coordinates are out of bounds and read as zero.  The other threads
+//                      write the slot -> grid-token table, a bitmask of the real slots and
+//                      the window's "last along a shifted axis" flags (the mask of a query
+//                      follows from these).  The producers run ahead as far as the ring
+//                      allows.
 //   warp 4             idle after set-up.
 // Synchronisation is by mbarriers only; every wait is bounded by a time limit and a
 // timeout unwinds the whole CTA (error word set, copies drained, TMEM freed).
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
 
 #include "s3w_internal.h"
 #include "sm100_ptx.cuh"
@@ -126,10 +132,18 @@ __device__ __forceinline__ bool mask_all(const uint32_t (&m)[kMaskWords]) {
 }
 __device__ __forceinline__ bool mask_bit(const uint32_t (&m)[kMaskWords], int j) { return (m[j >> 5] >> (j & 31)) & 1u; }
 
+// Tensor maps of Q, K and V over the grid as a 5-D tensor (channel, W, H, T, sample), one
+// per box height along W: a whole window run (win_w tokens), and the two pieces of a run
+// that wraps around the W seam (win_w - shift_w, then shift_w tokens).  Box width is 64
+// channels (one head of 64; for head_dim 32 the head plus its neighbour, 128 bytes either
+// way), 128-byte swizzle, out-of-bounds elements (padding) read as zero.
+struct TmaMaps {
+  CUtensorMap m[3][3];   // [tensor q/k/v][box: full run, wrap part 1, wrap part 2]
+};
+
 template <int HD, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1)
-window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __restrict__ q,
-                      const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__ TmaMaps maps,
                       void* __restrict__ o, int* __restrict__ err, unsigned long long limit_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -195,6 +209,18 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
       slotc->all[w] = bits;
     }
   }
+  // Slots N..143 are never loaded: keep them zero (finite) for the whole kernel.
+  if (g.N < kN) {
+    for (int i = tid; i < kStages * 3 * (kN - g.N) * (kRowBytes / 16); i += kThreads) {
+      const int chunk = i % (kRowBytes / 16);
+      const int rest = i / (kRowBytes / 16);
+      const int r = g.N + rest % (kN - g.N);
+      const int tile_id = rest / (kN - g.N);   // stage * 3 + tensor
+      *reinterpret_cast<uint4*>(sm + OFF_STAGE + tile_id * kTileBytes + r * kRowBytes + chunk * 16) =
+          make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
+  }
   if (warp == kMmaWarp) {
     tmem_alloc(sb + OFF_MISC, kTmemCols);
     tmem_relinquish();
@@ -207,8 +233,13 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
   if (warp >= kFirstProducerWarp) {
     // ------------------------------------------------------------------ producers
     const int p = tid - kFirstProducerWarp * 32;
-    constexpr int CH = HD / 8;                   // 16-byte chunks per head row
-    constexpr int kRowsPerPass = kProducerThreads / CH;
+    if (p == 0) {
+#pragma unroll
+      for (int a = 0; a < 3; ++a)
+#pragma unroll
+        for (int b = 0; b < 3; ++b) prefetch_tmap(&maps.m[a][b]);
+    }
+    const uint32_t tile_bytes = static_cast<uint32_t>(3 * g.N * kRowBytes);
     int it = 0;
     for (long long tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int s = it % kStages;
@@ -237,6 +268,34 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
       // shifted padded coordinate of slot offset 0, plus the shift: slot (rt, rh, rw) of
       // this window holds the original coordinate (base + offset) mod P on each axis.
       const int bt = itw * g.wt + g.st, bh = ih * g.wh + g.sh, bw = iw * g.ww + g.sw;
+      const uint32_t stage = sb + OFF_STAGE + s * kStageBytes;
+      if (p == 0) {
+        // One TMA box per (t, h) run of win_w tokens and tensor; a run that wraps around the
+        // W seam is loaded as two boxes.  Padded coordinates (>= T, H or W) read as zero.
+        mbar_arrive_expect_tx(full_bar(s), tile_bytes);
+        const bool wrap = bw + g.ww > g.Pw;
+        const int n1 = g.Pw - bw;
+        const int c0 = head * HD;
+        for (int rt = 0; rt < g.wt; ++rt) {
+          int t = bt + rt;
+          t -= t >= g.Pt ? g.Pt : 0;
+          for (int rh = 0; rh < g.wh; ++rh) {
+            int h = bh + rh;
+            h -= h >= g.Ph ? g.Ph : 0;
+            const uint32_t dst = stage + (rt * g.wh + rh) * g.ww * kRowBytes;
+#pragma unroll
+            for (int tsr = 0; tsr < 3; ++tsr) {
+              const uint32_t d = dst + tsr * kTileBytes;
+              if (!wrap) {
+                tma_load_5d(d, &maps.m[tsr][0], c0, bw, h, t, bsmp, full_bar(s));
+              } else {
+                tma_load_5d(d, &maps.m[tsr][1], c0, bw, h, t, bsmp, full_bar(s));
+                tma_load_5d(d + n1 * kRowBytes, &maps.m[tsr][2], c0, 0, h, t, bsmp, full_bar(s));
+              }
+            }
+          }
+        }
+      }
       auto resolve = [&](int r) -> int {   // grid token of slot r, -1 if padded
         if (r >= g.N) return -1;
         const uint32_t cd = slotc->coord[r];
@@ -249,38 +308,32 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
         if (t >= g.T || h >= g.H || w >= g.W) return -1;
         return ((bsmp * g.T + t) * g.H + h) * g.W + w;
       };
+      // Thread 0 only issues the loads (its expect_tx arrival releases nothing else); the
+      // other producer threads write the table and then arrive.
       Table& tb = tables[s];
-      {
-        const int pw = p >> 5;
-        for (int wd = pw; wd < kMaskWords; wd += kProducerThreads / 32) {
+      if (p != 0) {
+        for (int r = p - 1; r < kN; r += kProducerThreads - 1) tb.tok[r] = resolve(r);
+        if (p == 1)
+          tb.last = ((itw == g.nwt - 1 && g.st > 0) ? 1u : 0u) | ((ih == g.nwh - 1 && g.sh > 0) ? 2u : 0u) |
+                    ((iw == g.nww - 1 && g.sw > 0) ? 4u : 0u);
+      }
+      if (warp == kFirstProducerWarp + 1) {
+#pragma unroll
+        for (int wd = 0; wd < kMaskWords; ++wd) {
           const int r = 32 * wd + lane;
           const unsigned m = __ballot_sync(0xffffffffu, r < kN && resolve(r) >= 0);
           if (lane == 0) tb.real[wd] = m;
         }
-        if (p == 0)
-          tb.last = ((itw == g.nwt - 1 && g.st > 0) ? 1u : 0u) | ((ih == g.nwh - 1 && g.sh > 0) ? 2u : 0u) |
-                    ((iw == g.nww - 1 && g.sw > 0) ? 4u : 0u);
       }
-      // Each thread copies one 16-byte column c of every kRowsPerPass-th row, for Q, K and
-      // V: a warp covers whole 128-byte head rows, so every request is coalesced.
-      const uint32_t stage = sb + OFF_STAGE + s * kStageBytes;
-      const int c = p % CH;
-      const long long coff = static_cast<long long>(head) * HD + c * 8;
-#pragma unroll 6
-      for (int r = p / CH; r < kN; r += kRowsPerPass) {
-        const int tk = resolve(r);
-        if (c == 0) tb.tok[r] = tk;
-        const long long off = tk < 0 ? 0ll : static_cast<long long>(tk) * g.qkv_stride + coff;
-        const uint32_t dst = stage + r * kRowBytes + ((c ^ (r & 7)) << 4);
-        cp_async_16_zfill(dst, q + off, tk >= 0);
-        cp_async_16_zfill(dst + kTileBytes, k + off, tk >= 0);
-        cp_async_16_zfill(dst + 2 * kTileBytes, v + off, tk >= 0);
-      }
-      cp_async_commit();
-      cp_async_arrive(full_bar(s));   // fires when this thread's copies have landed
-      mbar_arrive(full_bar(s));       // table written (release)
+      if (p != 0) mbar_arrive(full_bar(s));   // table rows written (release); thread 0 arrived with expect_tx
     }
-    cp_async_wait_0();
+    // Before the CTA may exit, every TMA load issued must have landed.  On the normal path
+    // the MMA warp has consumed them all; after an abort, wait (bounded, independently of
+    // the test limit) for the last stages issued.
+    if (p == 0) {
+      for (int j = it > kStages ? it - kStages : 0; j < it; ++j)
+        if (!mbar_wait_bounded(full_bar(j % kStages), (j / kStages) & 1, 2000000000ull)) record_error(err, kStatusTimeout);
+    }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     // Issue order: S(t+1) goes out as soon as tile t+1 is loaded and S(t) has been read
@@ -688,18 +741,51 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __nv_bfloat16* __
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult qres;
+    void* ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+cudaError_t make_maps(const WinGeom& g, const void* const ptrs[3], TmaMaps* maps) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t es = 2;  // bf16
+  const cuuint64_t C = static_cast<cuuint64_t>(g.heads) * g.head_dim;
+  const cuuint64_t dims[5] = {C, static_cast<cuuint64_t>(g.W), static_cast<cuuint64_t>(g.H),
+                              static_cast<cuuint64_t>(g.T), static_cast<cuuint64_t>(g.B)};
+  const cuuint64_t row = static_cast<cuuint64_t>(g.qkv_stride) * es;
+  const cuuint64_t strides[4] = {row, row * g.W, row * g.W * g.H, row * g.W * g.H * g.T};
+  const cuuint32_t boxw[3] = {static_cast<cuuint32_t>(g.ww), static_cast<cuuint32_t>(g.ww - g.sw),
+                              static_cast<cuuint32_t>(g.sw > 0 ? g.sw : g.ww)};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  for (int t = 0; t < 3; ++t)
+    for (int b = 0; b < 3; ++b) {
+      const cuuint32_t box[5] = {64, boxw[b], 1, 1, 1};
+      CUresult r = enc(&maps->m[t][b], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptrs[t]), dims, strides,
+                       box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    }
+  return cudaSuccess;
+}
+
 template <int HD, bool OUT_F32>
-cudaError_t launch_t(const WinGeom& g, const void* q, const void* k, const void* v, void* o, int* err,
-                     long long limit_ns, int num_sms, cudaStream_t st) {
+cudaError_t launch_t(const WinGeom& g, const TmaMaps& maps, void* o, int* err, long long limit_ns, int num_sms,
+                     cudaStream_t st) {
   auto kern = window_attn_tc_kernel<HD, OUT_F32>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   if (e != cudaSuccess) return e;
   const long long tiles = g.windows * g.heads;
   const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-  kern<<<grid, kThreads, kSmemAlloc, st>>>(g, static_cast<const __nv_bfloat16*>(q),
-                                           static_cast<const __nv_bfloat16*>(k),
-                                           static_cast<const __nv_bfloat16*>(v), o, err,
-                                           static_cast<unsigned long long>(limit_ns < 0 ? 0 : limit_ns));
+  kern<<<grid, kThreads, kSmemAlloc, st>>>(g, maps, o, err, static_cast<unsigned long long>(limit_ns < 0 ? 0 : limit_ns));
   return cudaGetLastError();
 }
 
@@ -707,11 +793,15 @@ cudaError_t launch_t(const WinGeom& g, const void* q, const void* k, const void*
 
 cudaError_t launch_window_attn_tc(const WinGeom& g, const void* q, const void* k, const void* v, void* o,
                                   bool out_f32, int* err, long long spin_limit, int num_sms, cudaStream_t stream) {
+  TmaMaps maps;
+  const void* ptrs[3] = {q, k, v};
+  cudaError_t e = make_maps(g, ptrs, &maps);
+  if (e != cudaSuccess) return e;
   if (g.head_dim == 64)
-    return out_f32 ? launch_t<64, true>(g, q, k, v, o, err, spin_limit, num_sms, stream)
-                   : launch_t<64, false>(g, q, k, v, o, err, spin_limit, num_sms, stream);
-  return out_f32 ? launch_t<32, true>(g, q, k, v, o, err, spin_limit, num_sms, stream)
-                 : launch_t<32, false>(g, q, k, v, o, err, spin_limit, num_sms, stream);
+    return out_f32 ? launch_t<64, true>(g, maps, o, err, spin_limit, num_sms, stream)
+                   : launch_t<64, false>(g, maps, o, err, spin_limit, num_sms, stream);
+  return out_f32 ? launch_t<32, true>(g, maps, o, err, spin_limit, num_sms, stream)
+                 : launch_t<32, false>(g, maps, o, err, spin_limit, num_sms, stream);
 }
 
 }  // namespace s3w
