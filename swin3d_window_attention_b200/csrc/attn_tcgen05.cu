@@ -127,10 +127,6 @@ __device__ __forceinline__ void build_mask(const Table& tb, const SlotConst& sc,
     m[w] = x;
   }
 }
-__device__ __forceinline__ bool mask_all(const uint32_t (&m)[kMaskWords]) {
-  return ((m[0] & m[1] & m[2] & m[3]) == 0xffffffffu) && ((m[4] & 0xffffu) == 0xffffu);
-}
-__device__ __forceinline__ bool mask_bit(const uint32_t (&m)[kMaskWords], int j) { return (m[j >> 5] >> (j & 31)) & 1u; }
 
 // Tensor maps of Q, K and V over the grid as a 5-D tensor (channel, W, H, T, sample), one
 // per box height along W: a whole window run (win_w tokens), and the two pieces of a run
@@ -506,88 +502,152 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       return true;
     };
 
-    // Softmax of one S row held in registers (thread = row): mask, row max, exp2 and row
-    // sum, with independent partial accumulators and packed fp32x2 arithmetic.  The
-    // probabilities replace the logits in sv; returns 1 / rowsum.
-    auto softmax_row = [&](float (&sv)[kN], const uint32_t (&mw)[kMaskWords], bool full_tile) -> float {
-      float mx[8];
+    // Softmax of the main rows (thread = TMEM lane = query row), in two passes over TMEM so
+    // that only one 32-column chunk is live in registers and the loop bodies stay small:
+    // pass 1 takes the masked row max, pass 2 reloads the chunk, evaluates exp2, sums the
+    // row and stores P (bf16) into the 128B-swizzled P blocks.  Masked keys become -inf,
+    // hence weight 0, without a branch.
+    const uint32_t s0_addr = tmem + lane_base + TM_S0;
+    auto sel = [](uint32_t w, int e, float x) { return ((w >> e) & 1u) ? x : -INFINITY; };
+    auto main_row_max = [&](const uint32_t (&mw)[kMaskWords]) -> float {
+      float m = -INFINITY;
+      uint32_t w0 = mw[0], w1 = mw[1], w2 = mw[2], w3 = mw[3];
+#pragma unroll 1
+      for (int i = 0; i < 4; ++i) {
+        float x[32];
+        tmem_ld16(s0_addr + 32 * i, x);
+        tmem_ld16(s0_addr + 32 * i + 16, x + 16);
+        tmem_wait_ld();
+        reg_fence16(x);
+        reg_fence16(x + 16);
+        float a = -INFINITY, b = -INFINITY;
 #pragma unroll
-      for (int a = 0; a < 8; ++a) mx[a] = -INFINITY;
-      if (!full_tile) {
-#pragma unroll
-        for (int j = 0; j < kN; ++j) sv[j] = mask_bit(mw, j) ? sv[j] : -INFINITY;
+        for (int e = 0; e < 32; e += 4) {
+          a = max3(a, sel(w0, e, x[e]), sel(w0, e + 1, x[e + 1]));
+          b = max3(b, sel(w0, e + 2, x[e + 2]), sel(w0, e + 3, x[e + 3]));
+        }
+        m = max3(m, a, b);
+        w0 = w1;
+        w1 = w2;
+        w2 = w3;
       }
+      {
+        float x[16];
+        tmem_ld16(s0_addr + 128, x);
+        tmem_wait_ld();
+        reg_fence16(x);
+        const uint32_t w4 = mw[4];
+        float a = -INFINITY, b = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < kN; j += 2) mx[(j >> 1) & 7] = max3(mx[(j >> 1) & 7], sv[j], sv[j + 1]);
-      float m = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      if (m == -INFINITY) m = 0.f;
+        for (int e = 0; e < 16; e += 4) {
+          a = max3(a, sel(w4, e, x[e]), sel(w4, e + 1, x[e + 1]));
+          b = max3(b, sel(w4, e + 2, x[e + 2]), sel(w4, e + 3, x[e + 3]));
+        }
+        m = max3(m, a, b);
+      }
+      return m == -INFINITY ? 0.f : m;
+    };
+    auto main_row_exp = [&](const uint32_t (&mw)[kMaskWords], float m, int row) -> float {
       const float2 cc = make_float2(c, c), nm = make_float2(-m * c, -m * c);
-      float2 ls[4];
+      float2 l0 = make_float2(0.f, 0.f), l1 = make_float2(0.f, 0.f);
+      uint32_t w0 = mw[0], w1 = mw[1], w2 = mw[2], w3 = mw[3];
+      const uint32_t rsw = row & 7;
+#pragma unroll 1
+      for (int i = 0; i < 4; ++i) {
+        float x[32];
+        tmem_ld16(s0_addr + 32 * i, x);
+        tmem_ld16(s0_addr + 32 * i + 16, x + 16);
+        tmem_wait_ld();
+        reg_fence16(x);
+        reg_fence16(x + 16);
+        uint32_t pk[16];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) ls[a] = make_float2(0.f, 0.f);
+        for (int e = 0; e < 32; e += 4) {
+          const float2 ya = fma2(make_float2(sel(w0, e, x[e]), sel(w0, e + 1, x[e + 1])), cc, nm);
+          const float2 yb = fma2(make_float2(sel(w0, e + 2, x[e + 2]), sel(w0, e + 3, x[e + 3])), cc, nm);
+          const float2 pa = make_float2(ex2(ya.x), ex2(ya.y));
+          const float2 pb = make_float2(ex2(yb.x), ex2(yb.y));
+          l0 = add2(l0, pa);
+          l1 = add2(l1, pb);
+          pk[e / 2] = pack_bf16x2_int(pa.x, pa.y);
+          pk[e / 2 + 1] = pack_bf16x2_int(pb.x, pb.y);
+        }
+        // keys 32i .. 32i+31: 16-byte chunks (i & 1) * 4 + 0..3 of block i / 2
+        const uint32_t blk = sb + (i < 2 ? OFF_P0B0 : OFF_P0B1) + row * 128;
+        const uint32_t cb = (i & 1) * 4;
 #pragma unroll
-      for (int j = 0; j < kN; j += 2) {
-        const float2 x = fma2(make_float2(sv[j], sv[j + 1]), cc, nm);
-        const float2 pr = make_float2(ex2(x.x), ex2(x.y));
-        ls[(j >> 1) & 3] = add2(ls[(j >> 1) & 3], pr);
-        sv[j] = pr.x;
-        sv[j + 1] = pr.y;
+        for (int ch = 0; ch < 4; ++ch)
+          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(blk + (((cb + ch) ^ rsw) << 4)),
+                       "r"(pk[4 * ch]), "r"(pk[4 * ch + 1]), "r"(pk[4 * ch + 2]), "r"(pk[4 * ch + 3])
+                       : "memory");
+        w0 = w1;
+        w1 = w2;
+        w2 = w3;
       }
-      const float2 l2 = add2(add2(ls[0], ls[1]), add2(ls[2], ls[3]));
+      {
+        float x[16];
+        tmem_ld16(s0_addr + 128, x);
+        tmem_wait_ld();
+        reg_fence16(x);
+        const uint32_t w4 = mw[4];
+        uint32_t pk[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+          const float2 ya = fma2(make_float2(sel(w4, e, x[e]), sel(w4, e + 1, x[e + 1])), cc, nm);
+          const float2 yb = fma2(make_float2(sel(w4, e + 2, x[e + 2]), sel(w4, e + 3, x[e + 3])), cc, nm);
+          const float2 pa = make_float2(ex2(ya.x), ex2(ya.y));
+          const float2 pb = make_float2(ex2(yb.x), ex2(yb.y));
+          l0 = add2(l0, pa);
+          l1 = add2(l1, pb);
+          pk[e / 2] = pack_bf16x2_int(pa.x, pa.y);
+          pk[e / 2 + 1] = pack_bf16x2_int(pb.x, pb.y);
+        }
+        // keys 128..143: the 32B-swizzled block
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch)
+          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(sb + OFF_P0B2 + row * 32 +
+                                                                   ((ch ^ ((row >> 2) & 1)) << 4)),
+                       "r"(pk[4 * ch]), "r"(pk[4 * ch + 1]), "r"(pk[4 * ch + 2]), "r"(pk[4 * ch + 3])
+                       : "memory");
+      }
+      const float2 l2 = add2(l0, l1);
       const float l = l2.x + l2.y;
       return l > 0.f ? 1.f / l : 0.f;
     };
-    // Round a probability row to bf16 and store it as row `row` of the P operand (keys
-    // 0..63 and 64..127 in 128B-swizzled blocks, keys 128..143 in a 32B-swizzled block).
-    auto store_p_row = [&](const float (&sv)[kN], int row, uint32_t pb0, uint32_t pb1, uint32_t pb2) {
+
+    // The 16 tail rows (warp 0), spread over the warp with the 16x256b shape: for chunk j
+    // (8 columns) this lane holds columns 8j + 2qd + {0, 1} of rows ra and ra + 8.  Same two
+    // passes as the main rows, six iterations of three chunks; row max and sum finish with
+    // two shuffles among the four lanes (qd = 0..3) sharing a row.
+    auto lane_bits = [&](const uint32_t (&m)[kMaskWords]) -> uint64_t {   // bit 2j+e: column 8j+2qd+e
+      uint64_t r = 0;
 #pragma unroll
-      for (int b = 0; b < 2; ++b) {
-        const uint32_t base = (b == 0 ? pb0 : pb1) + row * 128;
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const int j0 = 64 * b + 8 * ch;
-          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(base + ((ch ^ (row & 7)) << 4)),
-                       "r"(pack_bf16x2_int(sv[j0], sv[j0 + 1])), "r"(pack_bf16x2_int(sv[j0 + 2], sv[j0 + 3])),
-                       "r"(pack_bf16x2_int(sv[j0 + 4], sv[j0 + 5])), "r"(pack_bf16x2_int(sv[j0 + 6], sv[j0 + 7]))
-                       : "memory");
-        }
-      }
-#pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        const int j0 = 128 + 8 * ch;
-        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(pb2 + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4)),
-                     "r"(pack_bf16x2_int(sv[j0], sv[j0 + 1])), "r"(pack_bf16x2_int(sv[j0 + 2], sv[j0 + 3])),
-                     "r"(pack_bf16x2_int(sv[j0 + 4], sv[j0 + 5])), "r"(pack_bf16x2_int(sv[j0 + 6], sv[j0 + 7]))
-                     : "memory");
-      }
+      for (int j = 0; j < kN / 8; ++j)
+        r |= static_cast<uint64_t>((m[j >> 2] >> (8 * (j & 3) + 2 * qd)) & 3u) << (2 * j);
+      return r;
     };
-    // The 16 tail rows, spread over the warp with the 16x256b shape: st[4j + 0..1] holds
-    // columns 8j + 2qd + {0, 1} of row ra, st[4j + 2..3] the same columns of row ra + 8.
-    // Row max / sum finish with two shuffles among the four lanes (qd = 0..3) that share a
-    // row.  Writes both rows' probabilities (bf16) into the tail P blocks and returns the
-    // two 1/rowsum values.
-    auto softmax_tail = [&](float* st, const uint32_t (&ma)[kMaskWords], const uint32_t (&mb)[kMaskWords],
-                            float& inv_a, float& inv_b) {
-      const bool full = __all_sync(0xffffffffu, mask_all(ma) && mask_all(mb));
-      if (!full) {
+    auto selb = [](uint64_t w, int e, float x) { return ((w >> e) & 1ull) ? x : -INFINITY; };
+    auto tail_rows = [&](uint64_t ba, uint64_t bb, float& inv_a, float& inv_b) {
+      float m_a = -INFINITY, m_b = -INFINITY;
+      {
+        uint64_t wa = ba, wb = bb;
+#pragma unroll 1
+        for (int i = 0; i < 6; ++i) {
+          float x[12];
 #pragma unroll
-        for (int j = 0; j < kN / 8; ++j) {
-          const int col = 8 * j + 2 * qd;
-          st[4 * j + 0] = mask_bit(ma, col) ? st[4 * j + 0] : -INFINITY;
-          st[4 * j + 1] = mask_bit(ma, col + 1) ? st[4 * j + 1] : -INFINITY;
-          st[4 * j + 2] = mask_bit(mb, col) ? st[4 * j + 2] : -INFINITY;
-          st[4 * j + 3] = mask_bit(mb, col + 1) ? st[4 * j + 3] : -INFINITY;
+          for (int k = 0; k < 3; ++k) tmem_ld_16x256b(tmem + TM_S1 + 8 * (3 * i + k), x + 4 * k);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 3; ++k) reg_fence4(x + 4 * k);
+#pragma unroll
+          for (int k = 0; k < 3; ++k) {
+            m_a = max3(m_a, selb(wa, 2 * k, x[4 * k]), selb(wa, 2 * k + 1, x[4 * k + 1]));
+            m_b = max3(m_b, selb(wb, 2 * k, x[4 * k + 2]), selb(wb, 2 * k + 1, x[4 * k + 3]));
+          }
+          wa >>= 6;
+          wb >>= 6;
         }
       }
-      float xa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      float xb[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int j = 0; j < kN / 8; ++j) {
-        xa[j & 3] = max3(xa[j & 3], st[4 * j], st[4 * j + 1]);
-        xb[j & 3] = max3(xb[j & 3], st[4 * j + 2], st[4 * j + 3]);
-      }
-      float m_a = fmaxf(fmaxf(xa[0], xa[1]), fmaxf(xa[2], xa[3]));
-      float m_b = fmaxf(fmaxf(xb[0], xb[1]), fmaxf(xb[2], xb[3]));
       m_a = fmaxf(m_a, __shfl_xor_sync(0xffffffffu, m_a, 1));
       m_a = fmaxf(m_a, __shfl_xor_sync(0xffffffffu, m_a, 2));
       m_b = fmaxf(m_b, __shfl_xor_sync(0xffffffffu, m_b, 1));
@@ -597,18 +657,43 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       const float2 cc = make_float2(c, c);
       const float2 na = make_float2(-m_a * c, -m_a * c), nb = make_float2(-m_b * c, -m_b * c);
       float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
+      const int rb = ra + 8;
+      uint64_t wa = ba, wb = bb;
+#pragma unroll 1
+      for (int i = 0; i < 6; ++i) {
+        float x[12];
 #pragma unroll
-      for (int j = 0; j < kN / 8; ++j) {
-        const float2 x = fma2(make_float2(st[4 * j], st[4 * j + 1]), cc, na);
-        const float2 y = fma2(make_float2(st[4 * j + 2], st[4 * j + 3]), cc, nb);
-        const float2 pa = make_float2(ex2(x.x), ex2(x.y));
-        const float2 pb = make_float2(ex2(y.x), ex2(y.y));
-        la = add2(la, pa);
-        lb = add2(lb, pb);
-        st[4 * j] = pa.x;
-        st[4 * j + 1] = pa.y;
-        st[4 * j + 2] = pb.x;
-        st[4 * j + 3] = pb.y;
+        for (int k = 0; k < 3; ++k) tmem_ld_16x256b(tmem + TM_S1 + 8 * (3 * i + k), x + 4 * k);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 3; ++k) reg_fence4(x + 4 * k);
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+          const float2 ya = fma2(make_float2(selb(wa, 2 * k, x[4 * k]), selb(wa, 2 * k + 1, x[4 * k + 1])), cc, na);
+          const float2 yb =
+              fma2(make_float2(selb(wb, 2 * k, x[4 * k + 2]), selb(wb, 2 * k + 1, x[4 * k + 3])), cc, nb);
+          const float2 pa = make_float2(ex2(ya.x), ex2(ya.y));
+          const float2 pb = make_float2(ex2(yb.x), ex2(yb.y));
+          la = add2(la, pa);
+          lb = add2(lb, pb);
+          // chunk j = 3i + k: keys 8j .. 8j+7 -> block j / 8 (the third block is 32B-swizzled)
+          const int j = 3 * i + k;
+          uint32_t addr_a, addr_b;
+          if (j < 16) {
+            const uint32_t blk = sb + (j < 8 ? OFF_P1B0 : OFF_P1B1);
+            const int ch = j & 7;
+            addr_a = blk + ra * 128 + ((ch ^ (ra & 7)) << 4) + 4 * qd;
+            addr_b = blk + rb * 128 + ((ch ^ (rb & 7)) << 4) + 4 * qd;
+          } else {
+            const int ch = j - 16;
+            addr_a = sb + OFF_P1B2 + ra * 32 + ((ch ^ ((ra >> 2) & 1)) << 4) + 4 * qd;
+            addr_b = sb + OFF_P1B2 + rb * 32 + ((ch ^ ((rb >> 2) & 1)) << 4) + 4 * qd;
+          }
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr_a), "r"(pack_bf16x2_int(pa.x, pa.y)) : "memory");
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr_b), "r"(pack_bf16x2_int(pb.x, pb.y)) : "memory");
+        }
+        wa >>= 6;
+        wb >>= 6;
       }
       float sa = la.x + la.y, sbm = lb.x + lb.y;
       sa += __shfl_xor_sync(0xffffffffu, sa, 1);
@@ -617,26 +702,6 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       sbm += __shfl_xor_sync(0xffffffffu, sbm, 2);
       inv_a = sa > 0.f ? 1.f / sa : 0.f;
       inv_b = sbm > 0.f ? 1.f / sbm : 0.f;
-      // bf16 pairs into the tail P blocks (4-byte stores; conflict-free across the warp)
-      const int rb = ra + 8;
-#pragma unroll
-      for (int j = 0; j < kN / 8; ++j) {
-        const uint32_t wa = pack_bf16x2_int(st[4 * j], st[4 * j + 1]);
-        const uint32_t wb = pack_bf16x2_int(st[4 * j + 2], st[4 * j + 3]);
-        uint32_t addr_a, addr_b;
-        if (j < 16) {
-          const uint32_t blk = sb + (j < 8 ? OFF_P1B0 : OFF_P1B1);
-          const int ch = j & 7;
-          addr_a = blk + ra * 128 + ((ch ^ (ra & 7)) << 4) + 4 * qd;
-          addr_b = blk + rb * 128 + ((ch ^ (rb & 7)) << 4) + 4 * qd;
-        } else {
-          const int ch = j - 16;
-          addr_a = sb + OFF_P1B2 + ra * 32 + ((ch ^ ((ra >> 2) & 1)) << 4) + 4 * qd;
-          addr_b = sb + OFF_P1B2 + rb * 32 + ((ch ^ ((rb >> 2) & 1)) << 4) + 4 * qd;
-        }
-        asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr_a), "r"(wa) : "memory");
-        asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr_b), "r"(wb) : "memory");
-      }
     };
 
     for (long long tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
@@ -673,39 +738,18 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         break;
       }
       tc_fence_after();
-      float sv[kN];
-#pragma unroll
-      for (int j = 0; j < kN / 16; ++j) tmem_ld16(tmem + lane_base + TM_S0 + 16 * j, sv + 16 * j);
-      tmem_wait_ld();
-#pragma unroll
-      for (int j = 0; j < kN / 16; ++j) reg_fence16(sv + 16 * j);
-      if (!tail_warp) {
-        tc_fence_before();
-        mbar_arrive(s_empty);   // S(t) is in registers: the next tile's S may be written
-      }
-
-      const bool full_tile = __all_sync(0xffffffffu, mask_all(mw));
-      const float inv = softmax_row(sv, mw, full_tile);
-      float inv_a = 0.f, inv_b = 0.f;
+      const float mrow = main_row_max(mw);
       // P may only be overwritten once the previous tile's PV MMA has consumed it.
       ok = mbar_wait_bounded(p_empty, (it & 1) ^ 1, limit_ns);
       if (!__all_sync(0xffffffffu, ok)) {
         aborted = true;
         break;
       }
-      store_p_row(sv, tid, sb + OFF_P0B0, sb + OFF_P0B1, sb + OFF_P0B2);
-      if (tail_warp) {
-        // the tail rows are loaded only now, so that the main row's registers are free
-        float st[kN / 2];
-#pragma unroll
-        for (int j = 0; j < kN / 8; ++j) tmem_ld_16x256b(tmem + TM_S1 + 8 * j, st + 4 * j);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < kN / 8; ++j) reg_fence4(st + 4 * j);
-        tc_fence_before();
-        mbar_arrive(s_empty);
-        softmax_tail(st, ma, mb, inv_a, inv_b);
-      }
+      const float inv = main_row_exp(mw, mrow, tid);
+      float inv_a = 0.f, inv_b = 0.f;
+      if (tail_warp) tail_rows(lane_bits(ma), lane_bits(mb), inv_a, inv_b);
+      tc_fence_before();
+      mbar_arrive(s_empty);   // every S read of this thread is done: the next tile's S may be written
       fence_proxy_async_smem();
       mbar_arrive(p_full);
       if (have_prev) {
