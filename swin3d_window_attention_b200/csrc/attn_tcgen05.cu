@@ -23,16 +23,14 @@
 //   MMA warp 5         one thread issues S(t+1) as soon as tile t+1 is loaded and S(t) has
 //                      left TMEM, then PV(t) = P V once P(t) is in shared memory (V read as
 //                      an MN-major operand); completion is signalled by tcgen05.commit.
-//   producer warps 6-7 one thread loads the tile's Q, K and V with TMA: one box per
-//                      (t, h) run of window tokens per tensor (two where the run wraps
-//                      around the W seam), straight from grid layout into a 3-stage ring in
-//                      the tensor core's 128-byte swizzled K-major layout; padded
-//                      coordinates are out of bounds and read as zero.  The other threads
-//                      write the slot -> grid-token table, a bitmask of the real slots and
+//   TMA warp 4         one thread loads the tile's Q, K and V with TMA: one box per (t, h)
+//                      run of window tokens per tensor (two where the run wraps around the
+//                      W seam), straight from grid layout into a 3-stage ring in the tensor
+//                      core's 128-byte swizzled K-major layout; padded coordinates are out
+//                      of bounds and read as zero.  It runs ahead as far as the ring allows.
+//   table warps 6-7    write the slot -> grid-token table, a bitmask of the real slots and
 //                      the window's "last along a shifted axis" flags (the mask of a query
-//                      follows from these).  The producers run ahead as far as the ring
-//                      allows.
-//   warp 4             idle after set-up.
+//                      follows from these) for the stage being loaded.
 // Synchronisation is by mbarriers only; every wait is bounded by a time limit and a
 // timeout unwinds the whole CTA (error word set, copies drained, TMEM freed).
 #include <cuda.h>
@@ -87,8 +85,9 @@ struct SlotConst {
 };
 constexpr int OFF_SLOTC = OFF_TABLE + kStages * kTableBytes;
 constexpr int OFF_BARS = OFF_SLOTC + ((static_cast<int>(sizeof(SlotConst)) + 15) & ~15);
-// barriers: full[3], empty[3], s_full, s_empty, p_full, p_empty, o_full, o_empty, drain
-constexpr int kNumBars = 2 * kStages + 7;
+// barriers: load[3] (TMA bytes), empty[3], table[3], s_full, s_empty, p_full, p_empty,
+// o_full, o_empty, drain
+constexpr int kNumBars = 3 * kStages + 7;
 constexpr int OFF_MISC = OFF_BARS + kNumBars * 8;   // tmem address, abort flag, producer stop
 constexpr int kSmemBytes = OFF_MISC + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1024;       // slack for the 1024-byte alignment
@@ -98,9 +97,10 @@ constexpr uint32_t TM_S0 = 0, TM_S1 = 160, TM_O0 = 320, TM_O1 = 384;
 constexpr uint32_t kTmemCols = 512;
 
 constexpr int kThreads = 256;
+constexpr int kTmaWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kFirstProducerWarp = 6;
-constexpr int kProducerThreads = 64;
+constexpr int kProducerThreads = 64;   // table writers (warps 6-7)
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -146,15 +146,16 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
   const uint32_t sb = smem_u32(sm);
   Table* tables = reinterpret_cast<Table*>(sm + OFF_TABLE);
   const uint32_t bar0 = sb + OFF_BARS;
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
-  const uint32_t s_full = bar0 + 8u * (2 * kStages + 0);
-  const uint32_t s_empty = bar0 + 8u * (2 * kStages + 1);
-  const uint32_t p_full = bar0 + 8u * (2 * kStages + 2);
-  const uint32_t p_empty = bar0 + 8u * (2 * kStages + 3);
-  const uint32_t o_full = bar0 + 8u * (2 * kStages + 4);
-  const uint32_t o_empty = bar0 + 8u * (2 * kStages + 5);
-  const uint32_t drain_bar = bar0 + 8u * (2 * kStages + 6);
+  auto load_bar = [&](int s) { return bar0 + 8u * s; };                  // Q/K/V of the stage landed
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };      // stage free again
+  auto table_bar = [&](int s) { return bar0 + 8u * (2 * kStages + s); };  // the stage's table written
+  const uint32_t s_full = bar0 + 8u * (3 * kStages + 0);
+  const uint32_t s_empty = bar0 + 8u * (3 * kStages + 1);
+  const uint32_t p_full = bar0 + 8u * (3 * kStages + 2);
+  const uint32_t p_empty = bar0 + 8u * (3 * kStages + 3);
+  const uint32_t o_full = bar0 + 8u * (3 * kStages + 4);
+  const uint32_t o_empty = bar0 + 8u * (3 * kStages + 5);
+  const uint32_t drain_bar = bar0 + 8u * (3 * kStages + 6);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sm + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
   volatile int* prod_stop = reinterpret_cast<volatile int*>(sm + OFF_MISC + 8);
@@ -166,8 +167,9 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(full_bar(s), kProducerThreads);
-      mbar_init(empty_bar(s), 1 + 128);   // PV commit + every softmax thread (table read)
+      mbar_init(load_bar(s), 1);                        // the TMA thread's expect_tx arrival + bytes
+      mbar_init(empty_bar(s), 1 + 128);                 // PV commit + every softmax thread (table read)
+      mbar_init(table_bar(s), kProducerThreads);
     }
     mbar_init(s_full, 1);
     mbar_init(s_empty, 128);
@@ -226,22 +228,91 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp >= kFirstProducerWarp) {
-    // ------------------------------------------------------------------ producers
-    const int p = tid - kFirstProducerWarp * 32;
-    if (p == 0) {
+  // Window coordinates of a tile (32-bit: the tile count is checked on the host) and the
+  // shifted padded coordinate of its slot offset 0 plus the shift: slot (rt, rh, rw) holds
+  // the original coordinate (base + offset) mod P on each axis.
+  struct TileCoord {
+    int head, bsmp, itw, ih, iw, bt, bh, bw;
+  };
+  auto tile_coord = [&](long long tile) {
+    TileCoord tc;
+    const int t32 = static_cast<int>(tile);
+    const int win = t32 / g.heads;
+    tc.head = t32 - win * g.heads;
+    const int per = g.nwt * g.nwh * g.nww;
+    tc.bsmp = win / per;
+    int rem = win - tc.bsmp * per;
+    tc.iw = rem % g.nww;
+    rem /= g.nww;
+    tc.ih = rem % g.nwh;
+    tc.itw = rem / g.nwh;
+    tc.bt = tc.itw * g.wt + g.st;
+    tc.bh = tc.ih * g.wh + g.sh;
+    tc.bw = tc.iw * g.ww + g.sw;
+    return tc;
+  };
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------------ TMA loads
+    // One thread loads each tile's Q, K and V: one box per (t, h) run of window tokens per
+    // tensor (two where the run wraps around the W seam), straight from grid layout into
+    // the stage; padded coordinates are out of bounds and read as zero.
+    if (lane == 0) {
 #pragma unroll
       for (int a = 0; a < 3; ++a)
 #pragma unroll
         for (int b = 0; b < 3; ++b) prefetch_tmap(&maps.m[a][b]);
+      const uint32_t tile_bytes = static_cast<uint32_t>(3 * g.N * kRowBytes);
+      int it = 0;
+      for (long long tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+        const int s = it % kStages;
+        if (*abort_flag) break;
+        if (!mbar_wait_bounded(empty_bar(s), ((it / kStages) & 1) ^ 1, limit_ns)) {
+          record_error(err, kStatusTimeout);
+          *abort_flag = 1;
+          break;
+        }
+        const TileCoord tc = tile_coord(tile);
+        const uint32_t stage = sb + OFF_STAGE + s * kStageBytes;
+        mbar_arrive_expect_tx(load_bar(s), tile_bytes);
+        const bool wrap = tc.bw + g.ww > g.Pw;
+        const int n1 = g.Pw - tc.bw;
+        const int c0 = tc.head * HD;
+        for (int rt = 0; rt < g.wt; ++rt) {
+          int t = tc.bt + rt;
+          t -= t >= g.Pt ? g.Pt : 0;
+          for (int rh = 0; rh < g.wh; ++rh) {
+            int h = tc.bh + rh;
+            h -= h >= g.Ph ? g.Ph : 0;
+            const uint32_t dst = stage + (rt * g.wh + rh) * g.ww * kRowBytes;
+#pragma unroll
+            for (int tsr = 0; tsr < 3; ++tsr) {
+              const uint32_t d = dst + tsr * kTileBytes;
+              if (!wrap) {
+                tma_load_5d(d, &maps.m[tsr][0], c0, tc.bw, h, t, tc.bsmp, load_bar(s));
+              } else {
+                tma_load_5d(d, &maps.m[tsr][1], c0, tc.bw, h, t, tc.bsmp, load_bar(s));
+                tma_load_5d(d + n1 * kRowBytes, &maps.m[tsr][2], c0, 0, h, t, tc.bsmp, load_bar(s));
+              }
+            }
+          }
+        }
+      }
+      // Before the CTA may exit, every load issued must have landed.  On the normal path
+      // the MMA warp has consumed them all; after an abort, wait (bounded, independently of
+      // the test limit) for the last stages issued.
+      for (int j = it > kStages ? it - kStages : 0; j < it; ++j)
+        if (!mbar_wait_bounded(load_bar(j % kStages), (j / kStages) & 1, 2000000000ull))
+          record_error(err, kStatusTimeout);
     }
-    const uint32_t tile_bytes = static_cast<uint32_t>(3 * g.N * kRowBytes);
+  } else if (warp >= kFirstProducerWarp) {
+    // ------------------------------------------------------------------ tile tables
+    const int p = tid - kFirstProducerWarp * 32;
     int it = 0;
     for (long long tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int s = it % kStages;
-      const uint32_t ph = (it / kStages) & 1;
       if (p == 0) {
-        const bool ok = mbar_wait_bounded(empty_bar(s), ph ^ 1, limit_ns);
+        const bool ok = mbar_wait_bounded(empty_bar(s), ((it / kStages) & 1) ^ 1, limit_ns);
         if (!ok) {
           record_error(err, kStatusTimeout);
           *abort_flag = 1;
@@ -250,85 +321,30 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       }
       named_bar_sync(1, kProducerThreads);
       if (*prod_stop) break;
-      // Window coordinates (32-bit: the tile count is checked on the host).
-      const int t32 = static_cast<int>(tile);
-      const int win = t32 / g.heads;
-      const int head = t32 - win * g.heads;
-      const int per = g.nwt * g.nwh * g.nww;
-      const int bsmp = win / per;
-      int rem = win - bsmp * per;
-      const int iw = rem % g.nww;
-      rem /= g.nww;
-      const int ih = rem % g.nwh;
-      const int itw = rem / g.nwh;
-      // shifted padded coordinate of slot offset 0, plus the shift: slot (rt, rh, rw) of
-      // this window holds the original coordinate (base + offset) mod P on each axis.
-      const int bt = itw * g.wt + g.st, bh = ih * g.wh + g.sh, bw = iw * g.ww + g.sw;
-      const uint32_t stage = sb + OFF_STAGE + s * kStageBytes;
-      if (p == 0) {
-        // One TMA box per (t, h) run of win_w tokens and tensor; a run that wraps around the
-        // W seam is loaded as two boxes.  Padded coordinates (>= T, H or W) read as zero.
-        mbar_arrive_expect_tx(full_bar(s), tile_bytes);
-        const bool wrap = bw + g.ww > g.Pw;
-        const int n1 = g.Pw - bw;
-        const int c0 = head * HD;
-        for (int rt = 0; rt < g.wt; ++rt) {
-          int t = bt + rt;
-          t -= t >= g.Pt ? g.Pt : 0;
-          for (int rh = 0; rh < g.wh; ++rh) {
-            int h = bh + rh;
-            h -= h >= g.Ph ? g.Ph : 0;
-            const uint32_t dst = stage + (rt * g.wh + rh) * g.ww * kRowBytes;
-#pragma unroll
-            for (int tsr = 0; tsr < 3; ++tsr) {
-              const uint32_t d = dst + tsr * kTileBytes;
-              if (!wrap) {
-                tma_load_5d(d, &maps.m[tsr][0], c0, bw, h, t, bsmp, full_bar(s));
-              } else {
-                tma_load_5d(d, &maps.m[tsr][1], c0, bw, h, t, bsmp, full_bar(s));
-                tma_load_5d(d + n1 * kRowBytes, &maps.m[tsr][2], c0, 0, h, t, bsmp, full_bar(s));
-              }
-            }
-          }
-        }
-      }
+      const TileCoord tc = tile_coord(tile);
       auto resolve = [&](int r) -> int {   // grid token of slot r, -1 if padded
         if (r >= g.N) return -1;
         const uint32_t cd = slotc->coord[r];
-        int t = bt + static_cast<int>(cd & 0xffu);
-        int h = bh + static_cast<int>((cd >> 8) & 0xffu);
-        int w = bw + static_cast<int>(cd >> 16);
+        int t = tc.bt + static_cast<int>(cd & 0xffu);
+        int h = tc.bh + static_cast<int>((cd >> 8) & 0xffu);
+        int w = tc.bw + static_cast<int>(cd >> 16);
         t -= t >= g.Pt ? g.Pt : 0;
         h -= h >= g.Ph ? g.Ph : 0;
         w -= w >= g.Pw ? g.Pw : 0;
         if (t >= g.T || h >= g.H || w >= g.W) return -1;
-        return ((bsmp * g.T + t) * g.H + h) * g.W + w;
+        return ((tc.bsmp * g.T + t) * g.H + h) * g.W + w;
       };
-      // Thread 0 only issues the loads (its expect_tx arrival releases nothing else); the
-      // other producer threads write the table and then arrive.
       Table& tb = tables[s];
-      if (p != 0) {
-        for (int r = p - 1; r < kN; r += kProducerThreads - 1) tb.tok[r] = resolve(r);
-        if (p == 1)
-          tb.last = ((itw == g.nwt - 1 && g.st > 0) ? 1u : 0u) | ((ih == g.nwh - 1 && g.sh > 0) ? 2u : 0u) |
-                    ((iw == g.nww - 1 && g.sw > 0) ? 4u : 0u);
+      for (int r = p; r < kN; r += kProducerThreads) tb.tok[r] = resolve(r);
+      if (p == 0)
+        tb.last = ((tc.itw == g.nwt - 1 && g.st > 0) ? 1u : 0u) | ((tc.ih == g.nwh - 1 && g.sh > 0) ? 2u : 0u) |
+                  ((tc.iw == g.nww - 1 && g.sw > 0) ? 4u : 0u);
+      for (int wd = p >> 5; wd < kMaskWords; wd += kProducerThreads / 32) {
+        const int r = 32 * wd + lane;
+        const unsigned m = __ballot_sync(0xffffffffu, r < kN && resolve(r) >= 0);
+        if (lane == 0) tb.real[wd] = m;
       }
-      if (warp == kFirstProducerWarp + 1) {
-#pragma unroll
-        for (int wd = 0; wd < kMaskWords; ++wd) {
-          const int r = 32 * wd + lane;
-          const unsigned m = __ballot_sync(0xffffffffu, r < kN && resolve(r) >= 0);
-          if (lane == 0) tb.real[wd] = m;
-        }
-      }
-      if (p != 0) mbar_arrive(full_bar(s));   // table rows written (release); thread 0 arrived with expect_tx
-    }
-    // Before the CTA may exit, every TMA load issued must have landed.  On the normal path
-    // the MMA warp has consumed them all; after an abort, wait (bounded, independently of
-    // the test limit) for the last stages issued.
-    if (p == 0) {
-      for (int j = it > kStages ? it - kStages : 0; j < it; ++j)
-        if (!mbar_wait_bounded(full_bar(j % kStages), (j / kStages) & 1, 2000000000ull)) record_error(err, kStatusTimeout);
+      mbar_arrive(table_bar(s));   // table written (release)
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
@@ -340,7 +356,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     bool issued = false;
     auto issue_s = [&](int jt) -> bool {   // S(jt) = Q K^T of the tile in stage jt % kStages
       const int s = jt % kStages;
-      if (!mbar_wait_bounded(full_bar(s), (jt / kStages) & 1, limit_ns)) return false;
+      if (!mbar_wait_bounded(load_bar(s), (jt / kStages) & 1, limit_ns)) return false;
       if (!mbar_wait_bounded(s_empty, (jt & 1) ^ 1, limit_ns)) return false;
       fence_proxy_async_smem();
       tc_fence_after();
@@ -711,7 +727,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         aborted = true;
         break;
       }
-      bool ok = mbar_wait_bounded(full_bar(s), ph, limit_ns);
+      bool ok = mbar_wait_bounded(table_bar(s), ph, limit_ns);
       if (!__all_sync(0xffffffffu, ok)) {
         aborted = true;
         break;
