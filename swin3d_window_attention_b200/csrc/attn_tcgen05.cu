@@ -12,14 +12,15 @@
 //    layout, so none of them costs a global-memory pass.
 //
 // Work unit ("tile"): one (sample, window, head).  Roles (warp -> SM sub-partition w % 4):
-//   softmax warps 0-3  thread t owns TMEM lane t = query row t of S0 = Q[0:128] K^T: load
-//                      the row (144 fp32), mask by region label / padding, exact row max,
-//                      exp2, row sum, P rounded to bf16 into shared memory.  Warp 0 also
-//                      owns the 16 tail rows (S1 = Q[128:144] K^T, TMEM lanes 0..15), read
-//                      with the 16x256b shape so all 32 lanes share them.  One tile later
-//                      (the PV MMA overlaps the next softmax) the same thread loads its O
-//                      row, scales by 1/rowsum and stores it to the query's original grid
-//                      position; padded slots are dropped.
+//   softmax warps 0-3  thread t owns TMEM lane t = query row t of S0 = Q[0:128] K^T: two
+//                      passes over the row (masked max; exp2, row sum and P rounded to bf16
+//                      into shared memory).  One tile later (the PV MMA overlaps the next
+//                      softmax) the same thread loads its O row, scales by 1/rowsum and
+//                      stores it to the query's original grid position; padded slots are
+//                      dropped.
+//   tail warp 4        the same for the 16 tail rows (S1 = Q[128:144] K^T in TMEM lanes
+//                      0..15, reachable from warp 4 like from warp 0), read with the 16x256b
+//                      shape so all 32 lanes share them.
 //   MMA warp 5         one thread issues S(t+1) as soon as tile t+1 is loaded and S(t) has
 //                      left TMEM, then PV(t) = P V once P(t) is in shared memory (V read as
 //                      an MN-major operand); completion is signalled by tcgen05.commit.
@@ -97,10 +98,11 @@ constexpr uint32_t TM_S0 = 0, TM_S1 = 160, TM_O0 = 320, TM_O1 = 384;
 constexpr uint32_t kTmemCols = 512;
 
 constexpr int kThreads = 256;
-constexpr int kTmaWarp = 4;
+constexpr int kTailWarp = 4;           // tail rows 128..143 (TMEM lane quarter 0, like warp 0)
 constexpr int kMmaWarp = 5;
-constexpr int kFirstProducerWarp = 6;
-constexpr int kProducerThreads = 64;   // table writers (warps 6-7)
+constexpr int kTmaWarp = 6;
+constexpr int kFirstProducerWarp = 7;
+constexpr int kProducerThreads = 32;   // table writer (warp 7)
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -164,19 +166,20 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
   const int warp = tid >> 5, lane = tid & 31;
   const long long num_tiles = g.windows * g.heads;
   const bool has_tail = g.N > 128;
+  const uint32_t n_soft = has_tail ? 160u : 128u;   // softmax threads: main rows (+ tail warp)
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(load_bar(s), 1);                        // the TMA thread's expect_tx arrival + bytes
-      mbar_init(empty_bar(s), 1 + 128);                 // PV commit + every softmax thread (table read)
+      mbar_init(empty_bar(s), 1 + n_soft);              // PV commit + every softmax thread (table read)
       mbar_init(table_bar(s), kProducerThreads);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_empty, 128);
-    mbar_init(p_full, 128);
+    mbar_init(s_empty, n_soft);
+    mbar_init(p_full, n_soft);
     mbar_init(p_empty, 1);
     mbar_init(o_full, 1);
-    mbar_init(o_empty, 128);
+    mbar_init(o_empty, n_soft);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     *prod_stop = 0;
@@ -424,26 +427,29 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       if (!mbar_wait_bounded(drain_bar, 0, 2000000000ull)) record_error(err, kStatusTimeout);
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 4 || (warp == kTailWarp && has_tail)) {
     // ------------------------------------------------------------------ softmax + epilogue
+    // Warps 0-3: main rows (thread = TMEM lane = query row).  Warp 4: the 16 tail rows,
+    // read through lane quarter 0 with the 16x256b shape (for chunk j of 8 columns, this
+    // lane holds columns 8j + 2qd + {0, 1} of rows ra and ra + 8), so the tail runs beside
+    // warp 0 instead of after it.
+    const bool is_tail = warp == kTailWarp;
     const float c = g.scale_log2;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const bool tail_warp = (warp == 0) && has_tail;
-    // Tail rows seen by this lane through the 16x256b shape: ra and ra + 8, columns
-    // 8j + 2*qd and 8j + 2*qd + 1 of every 8-column chunk j.
-    const int ra = lane >> 2, qd = lane & 3;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int ra = lane >> 2, qd = lane & 3, rb = ra + 8;
     auto hi_bits_of = [&](int r) -> uint32_t {
       uint32_t h = 0;
 #pragma unroll
       for (int a = 0; a < 3; ++a) h |= ((slotc->hi[a][r >> 5] >> (r & 31)) & 1u) << a;
       return h;
     };
-    const uint32_t my_hi = hi_bits_of(tid), hi_a = hi_bits_of(128 + ra), hi_b = hi_bits_of(136 + ra);
+    const uint32_t my_hi = is_tail ? 0u : hi_bits_of(tid);
+    const uint32_t hi_a = hi_bits_of(128 + ra), hi_b = hi_bits_of(128 + rb);
     int it = 0;
     // state of the previous tile, finished one iteration later
     bool have_prev = false;
-    int prev_it = 0, prev_head = 0, prev_tok = -1, prev_tok_a = -1, prev_tok_b = -1;
-    float prev_inv = 0.f, prev_inv_a = 0.f, prev_inv_b = 0.f;
+    int prev_it = 0, prev_head = 0, prev_tok = -1, prev_tok_b = -1;
+    float prev_inv = 0.f, prev_inv_b = 0.f;
     bool aborted = false;
 
     auto store8 = [&](int tk, int head, int col, const float* vals, float scl) {
@@ -481,71 +487,73 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       }
     };
 
-    auto epilogue = [&](int pit, int head, int tok, int tok_a, int tok_b, float inv, float inv_a,
-                        float inv_b) -> bool {
+    // Epilogue of a finished tile: O row(s) from TMEM, scaled by 1/rowsum, stored to the
+    // grid positions of the query slots (padded slots dropped).  For the tail warp `tok`
+    // / `inv` belong to row ra and `tok_b` / `inv_b` to row ra + 8.
+    auto epilogue = [&](int pit, int head, int tok, int tok_b, float inv, float inv_b) -> bool {
       bool ok = mbar_wait_bounded(o_full, pit & 1, limit_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) return false;
       tc_fence_after();
       float ov[HD];
-      float ot[HD / 2];   // tail: (row ra, row ra+8) x 2 columns per 8-column chunk
+      if (!is_tail) {
 #pragma unroll
-      for (int j = 0; j < HD / 16; ++j) tmem_ld16(tmem + lane_base + TM_O0 + 16 * j, ov + 16 * j);
-      if (tail_warp) {
+        for (int j = 0; j < HD / 16; ++j) tmem_ld16(tmem + lane_base + TM_O0 + 16 * j, ov + 16 * j);
+        tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < HD / 8; ++j) tmem_ld_16x256b(tmem + TM_O1 + 8 * j, ot + 4 * j);
-      }
-      tmem_wait_ld();
+        for (int j = 0; j < HD / 16; ++j) reg_fence16(ov + 16 * j);
+      } else {
 #pragma unroll
-      for (int j = 0; j < HD / 16; ++j) reg_fence16(ov + 16 * j);
-      if (tail_warp) {
+        for (int j = 0; j < HD / 8; ++j) tmem_ld_16x256b(tmem + TM_O1 + 8 * j, ov + 4 * j);
+        tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < HD / 8; ++j) reg_fence4(ot + 4 * j);
+        for (int j = 0; j < HD / 8; ++j) reg_fence4(ov + 4 * j);
       }
       tc_fence_before();
       mbar_arrive(o_empty);
-      if (tok >= 0) {
+      if (!is_tail) {
+        if (tok >= 0) {
 #pragma unroll
-        for (int j = 0; j < HD; j += 8) store8(tok, head, j, ov + j, inv);
-      }
-      if (tail_warp) {
+          for (int j = 0; j < HD; j += 8) store8(tok, head, j, ov + j, inv);
+        }
+      } else {
 #pragma unroll
         for (int j = 0; j < HD / 8; ++j) {
-          if (tok_a >= 0) store2(tok_a, head, 8 * j + 2 * qd, ot[4 * j], ot[4 * j + 1], inv_a);
-          if (tok_b >= 0) store2(tok_b, head, 8 * j + 2 * qd, ot[4 * j + 2], ot[4 * j + 3], inv_b);
+          if (tok >= 0) store2(tok, head, 8 * j + 2 * qd, ov[4 * j], ov[4 * j + 1], inv);
+          if (tok_b >= 0) store2(tok_b, head, 8 * j + 2 * qd, ov[4 * j + 2], ov[4 * j + 3], inv_b);
         }
       }
       return true;
     };
 
-    // Softmax of the main rows (thread = TMEM lane = query row), in two passes over TMEM so
-    // that only one 32-column chunk is live in registers and the loop bodies stay small:
-    // pass 1 takes the masked row max, pass 2 reloads the chunk, evaluates exp2, sums the
-    // row and stores P (bf16) into the 128B-swizzled P blocks.  Masked keys become -inf,
-    // hence weight 0, without a branch.
+    // Main rows, two passes over TMEM (64-column chunks, so only 64 logits are live and
+    // the loop bodies stay small): pass 1 takes the masked row max, pass 2 reloads the
+    // chunk, evaluates exp2, sums the row and stores P (bf16) into the 128B-swizzled P
+    // blocks.  Masked keys become -inf, hence weight 0, without a branch.
     const uint32_t s0_addr = tmem + lane_base + TM_S0;
     auto sel = [](uint32_t w, int e, float x) { return ((w >> e) & 1u) ? x : -INFINITY; };
     auto main_row_max = [&](const uint32_t (&mw)[kMaskWords]) -> float {
       float m = -INFINITY;
-      uint32_t w0 = mw[0], w1 = mw[1], w2 = mw[2], w3 = mw[3];
+      uint32_t w0 = mw[0], w1 = mw[1];
 #pragma unroll 1
-      for (int i = 0; i < 4; ++i) {
-        float x[32];
-        tmem_ld16(s0_addr + 32 * i, x);
-        tmem_ld16(s0_addr + 32 * i + 16, x + 16);
+      for (int i = 0; i < 2; ++i) {
+        float x[64];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tmem_ld16(s0_addr + 64 * i + 16 * j, x + 16 * j);
         tmem_wait_ld();
-        reg_fence16(x);
-        reg_fence16(x + 16);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) reg_fence16(x + 16 * j);
         float a = -INFINITY, b = -INFINITY;
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           a = max3(a, sel(w0, e, x[e]), sel(w0, e + 1, x[e + 1]));
           b = max3(b, sel(w0, e + 2, x[e + 2]), sel(w0, e + 3, x[e + 3]));
+          a = max3(a, sel(w1, e, x[32 + e]), sel(w1, e + 1, x[33 + e]));
+          b = max3(b, sel(w1, e + 2, x[34 + e]), sel(w1, e + 3, x[35 + e]));
         }
         m = max3(m, a, b);
-        w0 = w1;
-        w1 = w2;
-        w2 = w3;
+        w0 = mw[2];
+        w1 = mw[3];
       }
       {
         float x[16];
@@ -566,39 +574,38 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     auto main_row_exp = [&](const uint32_t (&mw)[kMaskWords], float m, int row) -> float {
       const float2 cc = make_float2(c, c), nm = make_float2(-m * c, -m * c);
       float2 l0 = make_float2(0.f, 0.f), l1 = make_float2(0.f, 0.f);
-      uint32_t w0 = mw[0], w1 = mw[1], w2 = mw[2], w3 = mw[3];
       const uint32_t rsw = row & 7;
 #pragma unroll 1
-      for (int i = 0; i < 4; ++i) {
-        float x[32];
-        tmem_ld16(s0_addr + 32 * i, x);
-        tmem_ld16(s0_addr + 32 * i + 16, x + 16);
+      for (int i = 0; i < 2; ++i) {
+        float x[64];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tmem_ld16(s0_addr + 64 * i + 16 * j, x + 16 * j);
         tmem_wait_ld();
-        reg_fence16(x);
-        reg_fence16(x + 16);
-        uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float2 ya = fma2(make_float2(sel(w0, e, x[e]), sel(w0, e + 1, x[e + 1])), cc, nm);
-          const float2 yb = fma2(make_float2(sel(w0, e + 2, x[e + 2]), sel(w0, e + 3, x[e + 3])), cc, nm);
-          const float2 pa = make_float2(ex2(ya.x), ex2(ya.y));
-          const float2 pb = make_float2(ex2(yb.x), ex2(yb.y));
-          l0 = add2(l0, pa);
-          l1 = add2(l1, pb);
-          pk[e / 2] = pack_bf16x2_int(pa.x, pa.y);
-          pk[e / 2 + 1] = pack_bf16x2_int(pb.x, pb.y);
+        for (int j = 0; j < 4; ++j) reg_fence16(x + 16 * j);
+        const uint32_t blk = sb + (i == 0 ? OFF_P0B0 : OFF_P0B1) + row * 128;   // keys 64i .. 64i+63
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t w = i == 0 ? mw[h] : mw[2 + h];
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float* xx = x + 32 * h;
+            const float2 ya = fma2(make_float2(sel(w, e, xx[e]), sel(w, e + 1, xx[e + 1])), cc, nm);
+            const float2 yb = fma2(make_float2(sel(w, e + 2, xx[e + 2]), sel(w, e + 3, xx[e + 3])), cc, nm);
+            const float2 pa = make_float2(ex2(ya.x), ex2(ya.y));
+            const float2 pb = make_float2(ex2(yb.x), ex2(yb.y));
+            l0 = add2(l0, pa);
+            l1 = add2(l1, pb);
+            pk[e / 2] = pack_bf16x2_int(pa.x, pa.y);
+            pk[e / 2 + 1] = pack_bf16x2_int(pb.x, pb.y);
+          }
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch)
+            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(blk + (((4 * h + ch) ^ rsw) << 4)),
+                         "r"(pk[4 * ch]), "r"(pk[4 * ch + 1]), "r"(pk[4 * ch + 2]), "r"(pk[4 * ch + 3])
+                         : "memory");
         }
-        // keys 32i .. 32i+31: 16-byte chunks (i & 1) * 4 + 0..3 of block i / 2
-        const uint32_t blk = sb + (i < 2 ? OFF_P0B0 : OFF_P0B1) + row * 128;
-        const uint32_t cb = (i & 1) * 4;
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(blk + (((cb + ch) ^ rsw) << 4)),
-                       "r"(pk[4 * ch]), "r"(pk[4 * ch + 1]), "r"(pk[4 * ch + 2]), "r"(pk[4 * ch + 3])
-                       : "memory");
-        w0 = w1;
-        w1 = w2;
-        w2 = w3;
       }
       {
         float x[16];
@@ -631,10 +638,8 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       return l > 0.f ? 1.f / l : 0.f;
     };
 
-    // The 16 tail rows (warp 0), spread over the warp with the 16x256b shape: for chunk j
-    // (8 columns) this lane holds columns 8j + 2qd + {0, 1} of rows ra and ra + 8.  Same two
-    // passes as the main rows, six iterations of three chunks; row max and sum finish with
-    // two shuffles among the four lanes (qd = 0..3) sharing a row.
+    // Tail rows (warp 4): same two passes, 2 x 9 chunks of 8 columns; row max and sum finish
+    // with two shuffles among the four lanes (qd = 0..3) sharing a row.
     auto lane_bits = [&](const uint32_t (&m)[kMaskWords]) -> uint64_t {   // bit 2j+e: column 8j+2qd+e
       uint64_t r = 0;
 #pragma unroll
@@ -643,26 +648,24 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       return r;
     };
     auto selb = [](uint64_t w, int e, float x) { return ((w >> e) & 1ull) ? x : -INFINITY; };
-    auto tail_rows = [&](uint64_t ba, uint64_t bb, float& inv_a, float& inv_b) {
-      float m_a = -INFINITY, m_b = -INFINITY;
-      {
-        uint64_t wa = ba, wb = bb;
+    auto tail_max = [&](uint64_t ba, uint64_t bb, float& m_a, float& m_b) {
+      m_a = -INFINITY;
+      m_b = -INFINITY;
 #pragma unroll 1
-        for (int i = 0; i < 6; ++i) {
-          float x[12];
+      for (int i = 0; i < 2; ++i) {
+        float x[36];
 #pragma unroll
-          for (int k = 0; k < 3; ++k) tmem_ld_16x256b(tmem + TM_S1 + 8 * (3 * i + k), x + 4 * k);
-          tmem_wait_ld();
+        for (int k = 0; k < 9; ++k) tmem_ld_16x256b(tmem + TM_S1 + 8 * (9 * i + k), x + 4 * k);
+        tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 3; ++k) reg_fence4(x + 4 * k);
+        for (int k = 0; k < 9; ++k) reg_fence4(x + 4 * k);
 #pragma unroll
-          for (int k = 0; k < 3; ++k) {
-            m_a = max3(m_a, selb(wa, 2 * k, x[4 * k]), selb(wa, 2 * k + 1, x[4 * k + 1]));
-            m_b = max3(m_b, selb(wb, 2 * k, x[4 * k + 2]), selb(wb, 2 * k + 1, x[4 * k + 3]));
-          }
-          wa >>= 6;
-          wb >>= 6;
+        for (int k = 0; k < 9; ++k) {
+          m_a = max3(m_a, selb(ba, 2 * k, x[4 * k]), selb(ba, 2 * k + 1, x[4 * k + 1]));
+          m_b = max3(m_b, selb(bb, 2 * k, x[4 * k + 2]), selb(bb, 2 * k + 1, x[4 * k + 3]));
         }
+        ba >>= 18;
+        bb >>= 18;
       }
       m_a = fmaxf(m_a, __shfl_xor_sync(0xffffffffu, m_a, 1));
       m_a = fmaxf(m_a, __shfl_xor_sync(0xffffffffu, m_a, 2));
@@ -670,30 +673,30 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       m_b = fmaxf(m_b, __shfl_xor_sync(0xffffffffu, m_b, 2));
       if (m_a == -INFINITY) m_a = 0.f;
       if (m_b == -INFINITY) m_b = 0.f;
+    };
+    auto tail_exp = [&](uint64_t ba, uint64_t bb, float m_a, float m_b, float& inv_a, float& inv_b) {
       const float2 cc = make_float2(c, c);
       const float2 na = make_float2(-m_a * c, -m_a * c), nb = make_float2(-m_b * c, -m_b * c);
       float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
-      const int rb = ra + 8;
-      uint64_t wa = ba, wb = bb;
 #pragma unroll 1
-      for (int i = 0; i < 6; ++i) {
-        float x[12];
+      for (int i = 0; i < 2; ++i) {
+        float x[36];
 #pragma unroll
-        for (int k = 0; k < 3; ++k) tmem_ld_16x256b(tmem + TM_S1 + 8 * (3 * i + k), x + 4 * k);
+        for (int k = 0; k < 9; ++k) tmem_ld_16x256b(tmem + TM_S1 + 8 * (9 * i + k), x + 4 * k);
         tmem_wait_ld();
 #pragma unroll
-        for (int k = 0; k < 3; ++k) reg_fence4(x + 4 * k);
+        for (int k = 0; k < 9; ++k) reg_fence4(x + 4 * k);
 #pragma unroll
-        for (int k = 0; k < 3; ++k) {
-          const float2 ya = fma2(make_float2(selb(wa, 2 * k, x[4 * k]), selb(wa, 2 * k + 1, x[4 * k + 1])), cc, na);
+        for (int k = 0; k < 9; ++k) {
+          const float2 ya = fma2(make_float2(selb(ba, 2 * k, x[4 * k]), selb(ba, 2 * k + 1, x[4 * k + 1])), cc, na);
           const float2 yb =
-              fma2(make_float2(selb(wb, 2 * k, x[4 * k + 2]), selb(wb, 2 * k + 1, x[4 * k + 3])), cc, nb);
+              fma2(make_float2(selb(bb, 2 * k, x[4 * k + 2]), selb(bb, 2 * k + 1, x[4 * k + 3])), cc, nb);
           const float2 pa = make_float2(ex2(ya.x), ex2(ya.y));
           const float2 pb = make_float2(ex2(yb.x), ex2(yb.y));
           la = add2(la, pa);
           lb = add2(lb, pb);
-          // chunk j = 3i + k: keys 8j .. 8j+7 -> block j / 8 (the third block is 32B-swizzled)
-          const int j = 3 * i + k;
+          // chunk j = 9i + k: keys 8j .. 8j+7 -> block j / 8 (the third block is 32B-swizzled)
+          const int j = 9 * i + k;
           uint32_t addr_a, addr_b;
           if (j < 16) {
             const uint32_t blk = sb + (j < 8 ? OFF_P1B0 : OFF_P1B1);
@@ -708,8 +711,8 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
           asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr_a), "r"(pack_bf16x2_int(pa.x, pa.y)) : "memory");
           asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr_b), "r"(pack_bf16x2_int(pb.x, pb.y)) : "memory");
         }
-        wa >>= 6;
-        wb >>= 6;
+        ba >>= 18;
+        bb >>= 18;
       }
       float sa = la.x + la.y, sbm = lb.x + lb.y;
       sa += __shfl_xor_sync(0xffffffffu, sa, 1);
@@ -735,15 +738,16 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       const long long win = tile / g.heads;
       const int head = static_cast<int>(tile - win * g.heads);
       const Table& tb = tables[s];
-      const int tok = tb.tok[tid];
       const uint32_t last = tb.last;
-      uint32_t mw[kMaskWords], ma[kMaskWords], mb[kMaskWords];
-      build_mask(tb, *slotc, last, my_hi, mw);
-      int tok_a = -1, tok_b = -1;
-      if (tail_warp) {
-        tok_a = tb.tok[128 + ra];
-        tok_b = tb.tok[136 + ra];
-        build_mask(tb, *slotc, last, hi_a, ma);
+      uint32_t mw[kMaskWords], mb[kMaskWords];
+      int tok, tok_b = -1;
+      if (!is_tail) {
+        tok = tb.tok[tid];
+        build_mask(tb, *slotc, last, my_hi, mw);
+      } else {
+        tok = tb.tok[128 + ra];   // row ra, mask in mw
+        tok_b = tb.tok[128 + rb];
+        build_mask(tb, *slotc, last, hi_a, mw);
         build_mask(tb, *slotc, last, hi_b, mb);
       }
       mbar_arrive(empty_bar(s));
@@ -754,22 +758,32 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         break;
       }
       tc_fence_after();
-      const float mrow = main_row_max(mw);
+      float mrow = 0.f, mrow_b = 0.f;
+      uint64_t ba = 0, bb = 0;
+      if (!is_tail) {
+        mrow = main_row_max(mw);
+      } else {
+        ba = lane_bits(mw);
+        bb = lane_bits(mb);
+        tail_max(ba, bb, mrow, mrow_b);
+      }
       // P may only be overwritten once the previous tile's PV MMA has consumed it.
       ok = mbar_wait_bounded(p_empty, (it & 1) ^ 1, limit_ns);
       if (!__all_sync(0xffffffffu, ok)) {
         aborted = true;
         break;
       }
-      const float inv = main_row_exp(mw, mrow, tid);
-      float inv_a = 0.f, inv_b = 0.f;
-      if (tail_warp) tail_rows(lane_bits(ma), lane_bits(mb), inv_a, inv_b);
+      float inv = 0.f, inv_b = 0.f;
+      if (!is_tail)
+        inv = main_row_exp(mw, mrow, tid);
+      else
+        tail_exp(ba, bb, mrow, mrow_b, inv, inv_b);
       tc_fence_before();
       mbar_arrive(s_empty);   // every S read of this thread is done: the next tile's S may be written
       fence_proxy_async_smem();
       mbar_arrive(p_full);
       if (have_prev) {
-        if (!epilogue(prev_it, prev_head, prev_tok, prev_tok_a, prev_tok_b, prev_inv, prev_inv_a, prev_inv_b)) {
+        if (!epilogue(prev_it, prev_head, prev_tok, prev_tok_b, prev_inv, prev_inv_b)) {
           aborted = true;
           have_prev = false;
           break;
@@ -779,15 +793,12 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       prev_it = it;
       prev_head = head;
       prev_tok = tok;
-      prev_tok_a = tok_a;
       prev_tok_b = tok_b;
       prev_inv = inv;
-      prev_inv_a = inv_a;
       prev_inv_b = inv_b;
     }
     if (have_prev && !aborted) {
-      if (!epilogue(prev_it, prev_head, prev_tok, prev_tok_a, prev_tok_b, prev_inv, prev_inv_a, prev_inv_b))
-        aborted = true;
+      if (!epilogue(prev_it, prev_head, prev_tok, prev_tok_b, prev_inv, prev_inv_b)) aborted = true;
     }
     if (aborted) {
       if (lane == 0) record_error(err, kStatusTimeout);
