@@ -281,23 +281,40 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         const bool wrap = tc.bw + g.ww > g.Pw;
         const int n1 = g.Pw - tc.bw;
         const int c0 = tc.head * HD;
-        for (int rt = 0; rt < g.wt; ++rt) {
-          int t = tc.bt + rt;
-          t -= t >= g.Pt ? g.Pt : 0;
-          for (int rh = 0; rh < g.wh; ++rh) {
-            int h = tc.bh + rh;
-            h -= h >= g.Ph ? g.Ph : 0;
-            const uint32_t dst = stage + (rt * g.wh + rh) * g.ww * kRowBytes;
+        // One flat loop over the window's (t, h) runs, unrolled 12 ways (a whole (2,6,12)
+        // window per pass): a TMA instruction reads its operand registers late, so issuing
+        // from a rolled loop that rewrites them every iteration stalls each issue.
+        int rt = 0, rh = 0;
+        int t = tc.bt;
+        t -= t >= g.Pt ? g.Pt : 0;
+        int h = tc.bh;
+        h -= h >= g.Ph ? g.Ph : 0;
+        const int nruns = g.wt * g.wh;
+        const uint32_t run_bytes = static_cast<uint32_t>(g.ww) * kRowBytes;
+#pragma unroll 12
+        for (int run = 0; run < nruns; ++run) {
+          const uint32_t dst = stage + run * run_bytes;
 #pragma unroll
-            for (int tsr = 0; tsr < 3; ++tsr) {
-              const uint32_t d = dst + tsr * kTileBytes;
-              if (!wrap) {
-                tma_load_5d(d, &maps.m[tsr][0], c0, tc.bw, h, t, tc.bsmp, load_bar(s));
-              } else {
-                tma_load_5d(d, &maps.m[tsr][1], c0, tc.bw, h, t, tc.bsmp, load_bar(s));
-                tma_load_5d(d + n1 * kRowBytes, &maps.m[tsr][2], c0, 0, h, t, tc.bsmp, load_bar(s));
-              }
+          for (int tsr = 0; tsr < 3; ++tsr) {
+            const uint32_t d = dst + tsr * kTileBytes;
+            if (!wrap) {
+              tma_load_5d(d, &maps.m[tsr][0], c0, tc.bw, h, t, tc.bsmp, load_bar(s));
+            } else {
+              tma_load_5d(d, &maps.m[tsr][1], c0, tc.bw, h, t, tc.bsmp, load_bar(s));
+              tma_load_5d(d + n1 * kRowBytes, &maps.m[tsr][2], c0, 0, h, t, tc.bsmp, load_bar(s));
             }
+          }
+          // next run: h advances, and at the end of a row of runs t advances (mod P)
+          if (++rh == g.wh) {
+            rh = 0;
+            ++rt;
+            h = tc.bh;
+            h -= h >= g.Ph ? g.Ph : 0;
+            t = tc.bt + rt;
+            t -= t >= g.Pt ? g.Pt : 0;
+          } else {
+            ++h;
+            h -= h >= g.Ph ? g.Ph : 0;
           }
         }
       }
