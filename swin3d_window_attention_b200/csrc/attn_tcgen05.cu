@@ -281,9 +281,9 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         const bool wrap = tc.bw + g.ww > g.Pw;
         const int n1 = g.Pw - tc.bw;
         const int c0 = tc.head * HD;
-        // One flat loop over the window's (t, h) runs, unrolled 12 ways (a whole (2,6,12)
-        // window per pass): a TMA instruction reads its operand registers late, so issuing
-        // from a rolled loop that rewrites them every iteration stalls each issue.
+        // One flat loop over the window's (t, h) runs.  A TMA instruction reads its operand
+        // registers late, so rewriting them right after an issue stalls; two runs per
+        // iteration halve those stalls while keeping the code small.
         int rt = 0, rh = 0;
         int t = tc.bt;
         t -= t >= g.Pt ? g.Pt : 0;
@@ -291,7 +291,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         h -= h >= g.Ph ? g.Ph : 0;
         const int nruns = g.wt * g.wh;
         const uint32_t run_bytes = static_cast<uint32_t>(g.ww) * kRowBytes;
-#pragma unroll 12
+#pragma unroll 2
         for (int run = 0; run < nruns; ++run) {
           const uint32_t dst = stage + run * run_bytes;
 #pragma unroll
@@ -421,15 +421,16 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       umma_commit(empty_bar(s));
       return true;
     };
+    // Step j issues S(j) (if tile j exists) and then PV(j-1): S(0); S(1), PV(0); S(2), PV(1); ...
+    // Lane 0 issues; every lane follows the same control flow (decisions are broadcast).
     int ok = 1;
-    if (lane == 0 && static_cast<long long>(blockIdx.x) < num_tiles) ok = issue_s(0);
-    ok = __shfl_sync(0xffffffffu, ok, 0);   // every lane takes the same path from here on
-    int it = 0;
-    for (long long tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
+    const long long my_tiles =
+        static_cast<long long>(blockIdx.x) < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    for (long long j = 0; ok && j <= my_tiles; ++j) {
       if (lane == 0) {
         ok = !*abort_flag;
-        if (ok && tile + gridDim.x < num_tiles) ok = issue_s(it + 1);
-        if (ok) ok = issue_pv(it);
+        if (ok && j < my_tiles) ok = issue_s(static_cast<int>(j));
+        if (ok && j > 0) ok = issue_pv(static_cast<int>(j - 1));
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
     }
@@ -543,73 +544,67 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       return true;
     };
 
-    // Main rows, two passes over TMEM (64-column chunks, so only 64 logits are live and
-    // the loop bodies stay small): pass 1 takes the masked row max, pass 2 reloads the
-    // chunk, evaluates exp2, sums the row and stores P (bf16) into the 128B-swizzled P
-    // blocks.  Masked keys become -inf, hence weight 0, without a branch.
+    // Main rows, two passes over TMEM in three rolled chunks of 48 columns (144 = 3 x 48),
+    // so only 48 logits are live and the loop bodies stay small (the code of every role
+    // has to stay resident in the instruction caches): pass 1 takes the masked row max,
+    // pass 2 reloads the chunk, evaluates exp2, sums the row and stores P (bf16) into the
+    // P blocks.  Masked keys become -inf, hence weight 0, without a branch.  The 144-bit
+    // mask is consumed 48 bits per chunk from a 64-bit shift register.
     const uint32_t s0_addr = tmem + lane_base + TM_S0;
-    auto sel = [](uint32_t w, int e, float x) { return ((w >> e) & 1u) ? x : -INFINITY; };
+    auto selb = [](uint64_t w, int e, float x) { return ((w >> e) & 1ull) ? x : -INFINITY; };
+    auto chunk_masks = [](const uint32_t (&mw)[kMaskWords], uint64_t& c0, uint64_t& c1, uint64_t& c2) {
+      // bits [0,48), [48,96), [96,144) of the row mask
+      c0 = (static_cast<uint64_t>(mw[0]) | (static_cast<uint64_t>(mw[1]) << 32)) & 0xffffffffffffull;
+      c1 = ((static_cast<uint64_t>(mw[1]) >> 16) | (static_cast<uint64_t>(mw[2]) << 16)) & 0xffffffffffffull;
+      c2 = (static_cast<uint64_t>(mw[3]) | (static_cast<uint64_t>(mw[4]) << 32)) & 0xffffffffffffull;
+    };
     auto main_row_max = [&](const uint32_t (&mw)[kMaskWords]) -> float {
-      float m = -INFINITY;
-      uint32_t w0 = mw[0], w1 = mw[1];
+      uint64_t c0, c1, c2;
+      chunk_masks(mw, c0, c1, c2);
+      float a = -INFINITY, b = -INFINITY;
 #pragma unroll 1
-      for (int i = 0; i < 2; ++i) {
-        float x[64];
+      for (int i = 0; i < 3; ++i) {
+        float x[48];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) tmem_ld16(s0_addr + 64 * i + 16 * j, x + 16 * j);
+        for (int j = 0; j < 3; ++j) tmem_ld16(s0_addr + 48 * i + 16 * j, x + 16 * j);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 4; ++j) reg_fence16(x + 16 * j);
-        float a = -INFINITY, b = -INFINITY;
+        for (int j = 0; j < 3; ++j) reg_fence16(x + 16 * j);
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          a = max3(a, sel(w0, e, x[e]), sel(w0, e + 1, x[e + 1]));
-          b = max3(b, sel(w0, e + 2, x[e + 2]), sel(w0, e + 3, x[e + 3]));
-          a = max3(a, sel(w1, e, x[32 + e]), sel(w1, e + 1, x[33 + e]));
-          b = max3(b, sel(w1, e + 2, x[34 + e]), sel(w1, e + 3, x[35 + e]));
+        for (int e = 0; e < 48; e += 4) {
+          a = max3(a, selb(c0, e, x[e]), selb(c0, e + 1, x[e + 1]));
+          b = max3(b, selb(c0, e + 2, x[e + 2]), selb(c0, e + 3, x[e + 3]));
         }
-        m = max3(m, a, b);
-        w0 = mw[2];
-        w1 = mw[3];
+        c0 = c1;
+        c1 = c2;
       }
-      {
-        float x[16];
-        tmem_ld16(s0_addr + 128, x);
-        tmem_wait_ld();
-        reg_fence16(x);
-        const uint32_t w4 = mw[4];
-        float a = -INFINITY, b = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < 16; e += 4) {
-          a = max3(a, sel(w4, e, x[e]), sel(w4, e + 1, x[e + 1]));
-          b = max3(b, sel(w4, e + 2, x[e + 2]), sel(w4, e + 3, x[e + 3]));
-        }
-        m = max3(m, a, b);
-      }
+      const float m = fmaxf(a, b);
       return m == -INFINITY ? 0.f : m;
     };
     auto main_row_exp = [&](const uint32_t (&mw)[kMaskWords], float m, int row) -> float {
       const float2 cc = make_float2(c, c), nm = make_float2(-m * c, -m * c);
       float2 l0 = make_float2(0.f, 0.f), l1 = make_float2(0.f, 0.f);
+      uint64_t c0, c1, c2;
+      chunk_masks(mw, c0, c1, c2);
       const uint32_t rsw = row & 7;
+      const uint32_t row128 = static_cast<uint32_t>(row) * 128, row32 = static_cast<uint32_t>(row) * 32;
+      const uint32_t sw32 = (row >> 2) & 1;
 #pragma unroll 1
-      for (int i = 0; i < 2; ++i) {
-        float x[64];
+      for (int i = 0; i < 3; ++i) {
+        float x[48];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) tmem_ld16(s0_addr + 64 * i + 16 * j, x + 16 * j);
+        for (int j = 0; j < 3; ++j) tmem_ld16(s0_addr + 48 * i + 16 * j, x + 16 * j);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 4; ++j) reg_fence16(x + 16 * j);
-        const uint32_t blk = sb + (i == 0 ? OFF_P0B0 : OFF_P0B1) + row * 128;   // keys 64i .. 64i+63
+        for (int j = 0; j < 3; ++j) reg_fence16(x + 16 * j);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t w = i == 0 ? mw[h] : mw[2 + h];
-          uint32_t pk[16];
+        for (int k = 0; k < 6; ++k) {   // 8 keys: 8g .. 8g+7, g = 6i + k
+          uint32_t pk[4];
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const float* xx = x + 32 * h;
-            const float2 ya = fma2(make_float2(sel(w, e, xx[e]), sel(w, e + 1, xx[e + 1])), cc, nm);
-            const float2 yb = fma2(make_float2(sel(w, e + 2, xx[e + 2]), sel(w, e + 3, xx[e + 3])), cc, nm);
+          for (int e = 0; e < 8; e += 4) {
+            const int q = 8 * k + e;
+            const float2 ya = fma2(make_float2(selb(c0, q, x[q]), selb(c0, q + 1, x[q + 1])), cc, nm);
+            const float2 yb = fma2(make_float2(selb(c0, q + 2, x[q + 2]), selb(c0, q + 3, x[q + 3])), cc, nm);
             const float2 pa = make_float2(ex2(ya.x), ex2(ya.y));
             const float2 pb = make_float2(ex2(yb.x), ex2(yb.y));
             l0 = add2(l0, pa);
@@ -617,38 +612,18 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
             pk[e / 2] = pack_bf16x2_int(pa.x, pa.y);
             pk[e / 2 + 1] = pack_bf16x2_int(pb.x, pb.y);
           }
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch)
-            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(blk + (((4 * h + ch) ^ rsw) << 4)),
-                         "r"(pk[4 * ch]), "r"(pk[4 * ch + 1]), "r"(pk[4 * ch + 2]), "r"(pk[4 * ch + 3])
-                         : "memory");
-        }
-      }
-      {
-        float x[16];
-        tmem_ld16(s0_addr + 128, x);
-        tmem_wait_ld();
-        reg_fence16(x);
-        const uint32_t w4 = mw[4];
-        uint32_t pk[8];
-#pragma unroll
-        for (int e = 0; e < 16; e += 4) {
-          const float2 ya = fma2(make_float2(sel(w4, e, x[e]), sel(w4, e + 1, x[e + 1])), cc, nm);
-          const float2 yb = fma2(make_float2(sel(w4, e + 2, x[e + 2]), sel(w4, e + 3, x[e + 3])), cc, nm);
-          const float2 pa = make_float2(ex2(ya.x), ex2(ya.y));
-          const float2 pb = make_float2(ex2(yb.x), ex2(yb.y));
-          l0 = add2(l0, pa);
-          l1 = add2(l1, pb);
-          pk[e / 2] = pack_bf16x2_int(pa.x, pa.y);
-          pk[e / 2 + 1] = pack_bf16x2_int(pb.x, pb.y);
-        }
-        // keys 128..143: the 32B-swizzled block
-#pragma unroll
-        for (int ch = 0; ch < 2; ++ch)
-          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(sb + OFF_P0B2 + row * 32 +
-                                                                   ((ch ^ ((row >> 2) & 1)) << 4)),
-                       "r"(pk[4 * ch]), "r"(pk[4 * ch + 1]), "r"(pk[4 * ch + 2]), "r"(pk[4 * ch + 3])
+          const int g8 = 6 * i + k;   // 16-byte chunk of P along the keys
+          uint32_t addr;
+          if (g8 < 16)
+            addr = sb + (g8 < 8 ? OFF_P0B0 : OFF_P0B1) + row128 + ((((g8 & 7) ^ rsw)) << 4);
+          else
+            addr = sb + OFF_P0B2 + row32 + (((g8 - 16) ^ sw32) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(pk[0]), "r"(pk[1]), "r"(pk[2]),
+                       "r"(pk[3])
                        : "memory");
+        }
+        c0 = c1;
+        c1 = c2;
       }
       const float2 l2 = add2(l0, l1);
       const float l = l2.x + l2.y;
@@ -664,7 +639,6 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         r |= static_cast<uint64_t>((m[j >> 2] >> (8 * (j & 3) + 2 * qd)) & 3u) << (2 * j);
       return r;
     };
-    auto selb = [](uint64_t w, int e, float x) { return ((w >> e) & 1ull) ? x : -INFINITY; };
     auto tail_max = [&](uint64_t ba, uint64_t bb, float& m_a, float& m_b) {
       m_a = -INFINITY;
       m_b = -INFINITY;
@@ -740,72 +714,77 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       inv_b = sbm > 0.f ? 1.f / sbm : 0.f;
     };
 
-    for (long long tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
-      const int s = it % kStages;
-      const uint32_t ph = (it / kStages) & 1;
-      if (__any_sync(0xffffffffu, *abort_flag != 0)) {
-        aborted = true;
-        break;
-      }
-      bool ok = mbar_wait_bounded(table_bar(s), ph, limit_ns);
-      if (!__all_sync(0xffffffffu, ok)) {
-        aborted = true;
-        break;
-      }
-      const long long win = tile / g.heads;
-      const int head = static_cast<int>(tile - win * g.heads);
-      const Table& tb = tables[s];
-      const uint32_t last = tb.last;
-      uint32_t mw[kMaskWords], mb[kMaskWords];
-      int tok, tok_b = -1;
-      if (!is_tail) {
-        tok = tb.tok[tid];
-        build_mask(tb, *slotc, last, my_hi, mw);
-      } else {
-        tok = tb.tok[128 + ra];   // row ra, mask in mw
-        tok_b = tb.tok[128 + rb];
-        build_mask(tb, *slotc, last, hi_a, mw);
-        build_mask(tb, *slotc, last, hi_b, mb);
-      }
-      mbar_arrive(empty_bar(s));
-
-      ok = mbar_wait_bounded(s_full, it & 1, limit_ns);
-      if (!__all_sync(0xffffffffu, ok)) {
-        aborted = true;
-        break;
-      }
-      tc_fence_after();
-      float mrow = 0.f, mrow_b = 0.f;
-      uint64_t ba = 0, bb = 0;
-      if (!is_tail) {
-        mrow = main_row_max(mw);
-      } else {
-        ba = lane_bits(mw);
-        bb = lane_bits(mb);
-        tail_max(ba, bb, mrow, mrow_b);
-      }
-      // P may only be overwritten once the previous tile's PV MMA has consumed it.
-      ok = mbar_wait_bounded(p_empty, (it & 1) ^ 1, limit_ns);
-      if (!__all_sync(0xffffffffu, ok)) {
-        aborted = true;
-        break;
-      }
+    // Iteration `it` does the softmax of tile `it` (if any) and then the epilogue of tile
+    // it-1, so the PV MMA of a tile overlaps the next tile's softmax.  One call site each.
+    for (long long tile = blockIdx.x;; tile += gridDim.x, ++it) {
+      const bool have_cur = tile < num_tiles;
+      int head = 0, tok = -1, tok_b = -1;
       float inv = 0.f, inv_b = 0.f;
-      if (!is_tail)
-        inv = main_row_exp(mw, mrow, tid);
-      else
-        tail_exp(ba, bb, mrow, mrow_b, inv, inv_b);
-      tc_fence_before();
-      mbar_arrive(s_empty);   // every S read of this thread is done: the next tile's S may be written
-      fence_proxy_async_smem();
-      mbar_arrive(p_full);
+      if (have_cur) {
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        if (__any_sync(0xffffffffu, *abort_flag != 0)) {
+          aborted = true;
+          break;
+        }
+        bool ok = mbar_wait_bounded(table_bar(s), ph, limit_ns);
+        if (!__all_sync(0xffffffffu, ok)) {
+          aborted = true;
+          break;
+        }
+        const long long win = tile / g.heads;
+        head = static_cast<int>(tile - win * g.heads);
+        const Table& tb = tables[s];
+        const uint32_t last = tb.last;
+        uint32_t mw[kMaskWords], mb[kMaskWords];
+        if (!is_tail) {
+          tok = tb.tok[tid];
+          build_mask(tb, *slotc, last, my_hi, mw);
+        } else {
+          tok = tb.tok[128 + ra];   // row ra, mask in mw
+          tok_b = tb.tok[128 + rb];
+          build_mask(tb, *slotc, last, hi_a, mw);
+          build_mask(tb, *slotc, last, hi_b, mb);
+        }
+        mbar_arrive(empty_bar(s));
+
+        ok = mbar_wait_bounded(s_full, it & 1, limit_ns);
+        if (!__all_sync(0xffffffffu, ok)) {
+          aborted = true;
+          break;
+        }
+        tc_fence_after();
+        float mrow = 0.f, mrow_b = 0.f;
+        uint64_t ba = 0, bb = 0;
+        if (!is_tail) {
+          mrow = main_row_max(mw);
+        } else {
+          ba = lane_bits(mw);
+          bb = lane_bits(mb);
+          tail_max(ba, bb, mrow, mrow_b);
+        }
+        // P may only be overwritten once the previous tile's PV MMA has consumed it.
+        ok = mbar_wait_bounded(p_empty, (it & 1) ^ 1, limit_ns);
+        if (!__all_sync(0xffffffffu, ok)) {
+          aborted = true;
+          break;
+        }
+        if (!is_tail)
+          inv = main_row_exp(mw, mrow, tid);
+        else
+          tail_exp(ba, bb, mrow, mrow_b, inv, inv_b);
+        tc_fence_before();
+        mbar_arrive(s_empty);   // every S read of this thread is done: the next tile's S may be written
+        fence_proxy_async_smem();
+        mbar_arrive(p_full);
+      }
       if (have_prev) {
         if (!epilogue(prev_it, prev_head, prev_tok, prev_tok_b, prev_inv, prev_inv_b)) {
           aborted = true;
-          have_prev = false;
           break;
         }
       }
+      if (!have_cur) break;
       have_prev = true;
       prev_it = it;
       prev_head = head;
@@ -813,9 +792,6 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       prev_tok_b = tok_b;
       prev_inv = inv;
       prev_inv_b = inv_b;
-    }
-    if (have_prev && !aborted) {
-      if (!epilogue(prev_it, prev_head, prev_tok, prev_tok_b, prev_inv, prev_inv_b)) aborted = true;
     }
     if (aborted) {
       if (lane == 0) record_error(err, kStatusTimeout);
