@@ -132,6 +132,10 @@ int make_geometry(const void* q, const void* k, const void* v, void* o, int B, i
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
   g.scale_log2 = sc * 1.4426950408889634f;  // log2(e): the softmax is evaluated with exp2
   g.o_rows_32b = ((reinterpret_cast<uintptr_t>(o) & 31u) == 0 && (o_token_stride * ob) % 32 == 0) ? 1 : 0;
+  g.div_heads = s3w::make_fastdiv(static_cast<uint32_t>(heads));
+  g.div_per_sample = s3w::make_fastdiv(static_cast<uint32_t>(per_sample));
+  g.div_nww = s3w::make_fastdiv(static_cast<uint32_t>(g.nww));
+  g.div_nwh = s3w::make_fastdiv(static_cast<uint32_t>(g.nwh));
   return S3W_OK;
 }
 

@@ -130,13 +130,18 @@ __device__ __forceinline__ void build_mask(const Table& tb, const SlotConst& sc,
   }
 }
 
-// Tensor maps of Q, K and V over the grid as a 5-D tensor (channel, W, H, T, sample), one
-// per box height along W: a whole window run (win_w tokens), and the two pieces of a run
-// that wraps around the W seam (win_w - shift_w, then shift_w tokens).  Box width is 64
-// channels (one head of 64; for head_dim 32 the head plus its neighbour, 128 bytes either
-// way), 128-byte swizzle, out-of-bounds elements (padding) read as zero.
+// Tensor maps of Q, K and V over the grid as a 5-D tensor (channel, W, H, T, sample),
+// one per box shape.  A window is loaded one T-slab (win_h x win_w tokens) at a time:
+// a whole slab in one box where the window does not wrap around a seam; a slab cut at
+// the H seam in two boxes (win_h - shift_h rows, then shift_h rows); and where the window
+// wraps around the W seam, one box per (t, h) run cut in two (win_w - shift_w, then
+// shift_w tokens), since a box narrower than the window would pack its rows too densely.
+// Box width is 64 channels (one head of 64; for head_dim 32 the head plus its
+// neighbour, 128 bytes either way), 128-byte swizzle, out-of-bounds elements (padding)
+// read as zero.
+enum : int { kBoxSlab = 0, kBoxSeamH1 = 1, kBoxSeamH2 = 2, kBoxSeamW1 = 3, kBoxSeamW2 = 4, kBoxShapes = 5 };
 struct TmaMaps {
-  CUtensorMap m[3][3];   // [tensor q/k/v][box: full run, wrap part 1, wrap part 2]
+  CUtensorMap m[3][kBoxShapes];   // [tensor q/k/v][box shape]
 };
 
 template <int HD, bool OUT_F32>
@@ -240,15 +245,14 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
   auto tile_coord = [&](long long tile) {
     TileCoord tc;
     const int t32 = static_cast<int>(tile);
-    const int win = t32 / g.heads;
+    const int win = fdiv(t32, g.div_heads);
     tc.head = t32 - win * g.heads;
-    const int per = g.nwt * g.nwh * g.nww;
-    tc.bsmp = win / per;
-    int rem = win - tc.bsmp * per;
-    tc.iw = rem % g.nww;
-    rem /= g.nww;
-    tc.ih = rem % g.nwh;
-    tc.itw = rem / g.nwh;
+    tc.bsmp = fdiv(win, g.div_per_sample);
+    const int rem = win - tc.bsmp * (g.nwt * g.nwh * g.nww);
+    const int q1 = fdiv(rem, g.div_nww);
+    tc.iw = rem - q1 * g.nww;
+    tc.itw = fdiv(q1, g.div_nwh);
+    tc.ih = q1 - tc.itw * g.nwh;
     tc.bt = tc.itw * g.wt + g.st;
     tc.bh = tc.ih * g.wh + g.sh;
     tc.bw = tc.iw * g.ww + g.sw;
@@ -264,8 +268,9 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
 #pragma unroll
       for (int a = 0; a < 3; ++a)
 #pragma unroll
-        for (int b = 0; b < 3; ++b) prefetch_tmap(&maps.m[a][b]);
+        for (int b = 0; b < kBoxShapes; ++b) prefetch_tmap(&maps.m[a][b]);
       const uint32_t tile_bytes = static_cast<uint32_t>(3 * g.N * kRowBytes);
+      const uint32_t run_bytes = static_cast<uint32_t>(g.ww) * kRowBytes;
       int it = 0;
       for (long long tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
         const int s = it % kStages;
@@ -277,44 +282,45 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         }
         const TileCoord tc = tile_coord(tile);
         const uint32_t stage = sb + OFF_STAGE + s * kStageBytes;
-        mbar_arrive_expect_tx(load_bar(s), tile_bytes);
-        const bool wrap = tc.bw + g.ww > g.Pw;
-        const int n1 = g.Pw - tc.bw;
+        const uint32_t bar = load_bar(s);
+        mbar_arrive_expect_tx(bar, tile_bytes);
+        // The window's first slot sits at (bt, bh, bw), inside the padded grid on every
+        // axis; a window wraps around an axis's seam only if it is the last one along a
+        // shifted axis.
+        const bool wrap_w = tc.bw + g.ww > g.Pw;
+        const bool wrap_h = tc.bh + g.wh > g.Ph;
+        const int n1w = g.Pw - tc.bw, n1h = g.Ph - tc.bh;
         const int c0 = tc.head * HD;
-        // One flat loop over the window's (t, h) runs.  A TMA instruction reads its operand
-        // registers late, so rewriting them right after an issue stalls; two runs per
-        // iteration halve those stalls while keeping the code small.
-        int rt = 0, rh = 0;
-        int t = tc.bt;
-        t -= t >= g.Pt ? g.Pt : 0;
-        int h = tc.bh;
-        h -= h >= g.Ph ? g.Ph : 0;
-        const int nruns = g.wt * g.wh;
-        const uint32_t run_bytes = static_cast<uint32_t>(g.ww) * kRowBytes;
-#pragma unroll 2
-        for (int run = 0; run < nruns; ++run) {
-          const uint32_t dst = stage + run * run_bytes;
+#pragma unroll 1
+        for (int rt = 0; rt < g.wt; ++rt) {
+          int t = tc.bt + rt;
+          t -= t >= g.Pt ? g.Pt : 0;
+          const uint32_t slab = stage + rt * g.wh * run_bytes;
+          if (!wrap_w) {
 #pragma unroll
-          for (int tsr = 0; tsr < 3; ++tsr) {
-            const uint32_t d = dst + tsr * kTileBytes;
-            if (!wrap) {
-              tma_load_5d(d, &maps.m[tsr][0], c0, tc.bw, h, t, tc.bsmp, load_bar(s));
-            } else {
-              tma_load_5d(d, &maps.m[tsr][1], c0, tc.bw, h, t, tc.bsmp, load_bar(s));
-              tma_load_5d(d + n1 * kRowBytes, &maps.m[tsr][2], c0, 0, h, t, tc.bsmp, load_bar(s));
+            for (int tsr = 0; tsr < 3; ++tsr) {
+              const uint32_t d = slab + tsr * kTileBytes;
+              if (!wrap_h) {
+                tma_load_5d(d, &maps.m[tsr][kBoxSlab], c0, tc.bw, tc.bh, t, tc.bsmp, bar);
+              } else {
+                tma_load_5d(d, &maps.m[tsr][kBoxSeamH1], c0, tc.bw, tc.bh, t, tc.bsmp, bar);
+                tma_load_5d(d + n1h * run_bytes, &maps.m[tsr][kBoxSeamH2], c0, tc.bw, 0, t, tc.bsmp, bar);
+              }
             }
-          }
-          // next run: h advances, and at the end of a row of runs t advances (mod P)
-          if (++rh == g.wh) {
-            rh = 0;
-            ++rt;
-            h = tc.bh;
-            h -= h >= g.Ph ? g.Ph : 0;
-            t = tc.bt + rt;
-            t -= t >= g.Pt ? g.Pt : 0;
           } else {
-            ++h;
-            h -= h >= g.Ph ? g.Ph : 0;
+            int h = tc.bh;
+#pragma unroll 1
+            for (int rh = 0; rh < g.wh; ++rh) {
+              const uint32_t dst = slab + rh * run_bytes;
+#pragma unroll
+              for (int tsr = 0; tsr < 3; ++tsr) {
+                const uint32_t d = dst + tsr * kTileBytes;
+                tma_load_5d(d, &maps.m[tsr][kBoxSeamW1], c0, tc.bw, h, t, tc.bsmp, bar);
+                tma_load_5d(d + n1w * kRowBytes, &maps.m[tsr][kBoxSeamW2], c0, 0, h, t, tc.bsmp, bar);
+              }
+              ++h;
+              h -= h >= g.Ph ? g.Ph : 0;
+            }
           }
         }
       }
@@ -548,8 +554,10 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     // so only 48 logits are live and the loop bodies stay small (the code of every role
     // has to stay resident in the instruction caches): pass 1 takes the masked row max,
     // pass 2 reloads the chunk, evaluates exp2, sums the row and stores P (bf16) into the
-    // P blocks.  Masked keys become -inf, hence weight 0, without a branch.  The 144-bit
-    // mask is consumed 48 bits per chunk from a 64-bit shift register.
+    // P blocks.  For a tile whose rows of this warp all keep every key (the usual case
+    // away from the shift seams and the padding) the chunks go straight to max / exp2;
+    // otherwise masked keys become -inf first, hence weight 0.  The 144-bit mask is
+    // consumed 48 bits per chunk from a 64-bit shift register.
     const uint32_t s0_addr = tmem + lane_base + TM_S0;
     auto selb = [](uint64_t w, int e, float x) { return ((w >> e) & 1ull) ? x : -INFINITY; };
     auto chunk_masks = [](const uint32_t (&mw)[kMaskWords], uint64_t& c0, uint64_t& c1, uint64_t& c2) {
@@ -558,22 +566,31 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       c1 = ((static_cast<uint64_t>(mw[1]) >> 16) | (static_cast<uint64_t>(mw[2]) << 16)) & 0xffffffffffffull;
       c2 = (static_cast<uint64_t>(mw[3]) | (static_cast<uint64_t>(mw[4]) << 32)) & 0xffffffffffffull;
     };
-    auto main_row_max = [&](const uint32_t (&mw)[kMaskWords]) -> float {
+    // Masked keys of a chunk become -inf in place (only called for tiles with a mask).
+    auto mask_chunk = [&](float* x, uint64_t cm) {
+#pragma unroll
+      for (int e = 0; e < 48; ++e) x[e] = selb(cm, e, x[e]);
+    };
+    auto load_chunk = [&](int i, float* x) {
+#pragma unroll
+      for (int j = 0; j < 3; ++j) tmem_ld16(s0_addr + 48 * i + 16 * j, x + 16 * j);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 3; ++j) reg_fence16(x + 16 * j);
+    };
+    auto main_row_max = [&](const uint32_t (&mw)[kMaskWords], bool masked) -> float {
       uint64_t c0, c1, c2;
       chunk_masks(mw, c0, c1, c2);
       float a = -INFINITY, b = -INFINITY;
 #pragma unroll 1
       for (int i = 0; i < 3; ++i) {
         float x[48];
-#pragma unroll
-        for (int j = 0; j < 3; ++j) tmem_ld16(s0_addr + 48 * i + 16 * j, x + 16 * j);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 3; ++j) reg_fence16(x + 16 * j);
+        load_chunk(i, x);
+        if (masked) mask_chunk(x, c0);
 #pragma unroll
         for (int e = 0; e < 48; e += 4) {
-          a = max3(a, selb(c0, e, x[e]), selb(c0, e + 1, x[e + 1]));
-          b = max3(b, selb(c0, e + 2, x[e + 2]), selb(c0, e + 3, x[e + 3]));
+          a = max3(a, x[e], x[e + 1]);
+          b = max3(b, x[e + 2], x[e + 3]);
         }
         c0 = c1;
         c1 = c2;
@@ -581,7 +598,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       const float m = fmaxf(a, b);
       return m == -INFINITY ? 0.f : m;
     };
-    auto main_row_exp = [&](const uint32_t (&mw)[kMaskWords], float m, int row) -> float {
+    auto main_row_exp = [&](const uint32_t (&mw)[kMaskWords], bool masked, float m, int row) -> float {
       const float2 cc = make_float2(c, c), nm = make_float2(-m * c, -m * c);
       float2 l0 = make_float2(0.f, 0.f), l1 = make_float2(0.f, 0.f);
       uint64_t c0, c1, c2;
@@ -592,19 +609,16 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
 #pragma unroll 1
       for (int i = 0; i < 3; ++i) {
         float x[48];
-#pragma unroll
-        for (int j = 0; j < 3; ++j) tmem_ld16(s0_addr + 48 * i + 16 * j, x + 16 * j);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 3; ++j) reg_fence16(x + 16 * j);
+        load_chunk(i, x);
+        if (masked) mask_chunk(x, c0);
 #pragma unroll
         for (int k = 0; k < 6; ++k) {   // 8 keys: 8g .. 8g+7, g = 6i + k
           uint32_t pk[4];
 #pragma unroll
           for (int e = 0; e < 8; e += 4) {
             const int q = 8 * k + e;
-            const float2 ya = fma2(make_float2(selb(c0, q, x[q]), selb(c0, q + 1, x[q + 1])), cc, nm);
-            const float2 yb = fma2(make_float2(selb(c0, q + 2, x[q + 2]), selb(c0, q + 3, x[q + 3])), cc, nm);
+            const float2 ya = fma2(make_float2(x[q], x[q + 1]), cc, nm);
+            const float2 yb = fma2(make_float2(x[q + 2], x[q + 3]), cc, nm);
             const float2 pa = make_float2(ex2(ya.x), ex2(ya.y));
             const float2 pb = make_float2(ex2(yb.x), ex2(yb.y));
             l0 = add2(l0, pa);
@@ -732,8 +746,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
           aborted = true;
           break;
         }
-        const long long win = tile / g.heads;
-        head = static_cast<int>(tile - win * g.heads);
+        head = static_cast<int>(tile) - fdiv(static_cast<int>(tile), g.div_heads) * g.heads;
         const Table& tb = tables[s];
         const uint32_t last = tb.last;
         uint32_t mw[kMaskWords], mb[kMaskWords];
@@ -756,8 +769,11 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         tc_fence_after();
         float mrow = 0.f, mrow_b = 0.f;
         uint64_t ba = 0, bb = 0;
+        bool masked = false;
         if (!is_tail) {
-          mrow = main_row_max(mw);
+          masked = !__all_sync(0xffffffffu, ((mw[0] & mw[1] & mw[2] & mw[3]) == 0xffffffffu) &&
+                                                ((mw[4] & 0xffffu) == 0xffffu));
+          mrow = main_row_max(mw, masked);
         } else {
           ba = lane_bits(mw);
           bb = lane_bits(mb);
@@ -770,7 +786,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
           break;
         }
         if (!is_tail)
-          inv = main_row_exp(mw, mrow, tid);
+          inv = main_row_exp(mw, masked, mrow, tid);
         else
           tail_exp(ba, bb, mrow, mrow_b, inv, inv_b);
         tc_fence_before();
@@ -827,12 +843,19 @@ cudaError_t make_maps(const WinGeom& g, const void* const ptrs[3], TmaMaps* maps
                               static_cast<cuuint64_t>(g.T), static_cast<cuuint64_t>(g.B)};
   const cuuint64_t row = static_cast<cuuint64_t>(g.qkv_stride) * es;
   const cuuint64_t strides[4] = {row, row * g.W, row * g.W * g.H, row * g.W * g.H * g.T};
-  const cuuint32_t boxw[3] = {static_cast<cuuint32_t>(g.ww), static_cast<cuuint32_t>(g.ww - g.sw),
-                              static_cast<cuuint32_t>(g.sw > 0 ? g.sw : g.ww)};
+  // box (W, H) extents per shape; a seam shape of an unshifted axis is never used and
+  // gets the whole window instead
+  const cuuint32_t ww = static_cast<cuuint32_t>(g.ww), wh = static_cast<cuuint32_t>(g.wh);
+  const cuuint32_t sw = static_cast<cuuint32_t>(g.sw), sh = static_cast<cuuint32_t>(g.sh);
+  const cuuint32_t boxwh[kBoxShapes][2] = {{ww, wh},
+                                           {ww, wh - sh},
+                                           {ww, sh > 0 ? sh : wh},
+                                           {ww - sw, 1},
+                                           {sw > 0 ? sw : ww, 1}};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   for (int t = 0; t < 3; ++t)
-    for (int b = 0; b < 3; ++b) {
-      const cuuint32_t box[5] = {64, boxw[b], 1, 1, 1};
+    for (int b = 0; b < kBoxShapes; ++b) {
+      const cuuint32_t box[5] = {64, boxwh[b][0], boxwh[b][1], 1, 1};
       CUresult r = enc(&maps->m[t][b], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptrs[t]), dims, strides,
                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

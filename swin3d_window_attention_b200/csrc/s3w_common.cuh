@@ -19,6 +19,27 @@ namespace s3w {
 
 enum : int { kStatusTimeout = 5 };
 
+// Division by a runtime-invariant divisor d >= 1 for 0 <= n < 2^31 by one 64-bit multiply
+// and a shift (Granlund and Montgomery, "Division by invariant integers using
+// multiplication", 1994): with l = ceil(log2 d) and m = ceil(2^(31+l) / d),
+// n / d = (n * m) >> (31 + l).  The host computes (m, l).
+struct FastDiv {
+  uint32_t m;
+  int shift;   // 31 + l
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  int l = 0;
+  while ((1ull << l) < d) ++l;
+  const unsigned long long num = 1ull << (31 + l);
+  FastDiv f;
+  f.m = static_cast<uint32_t>((num + d - 1) / d);
+  f.shift = 31 + l;
+  return f;
+}
+__device__ __forceinline__ int fdiv(int n, const FastDiv& f) {
+  return static_cast<int>((static_cast<unsigned long long>(static_cast<uint32_t>(n)) * f.m) >> f.shift);
+}
+
 // Everything a kernel needs to map (window id, slot) to a grid token.  Passed by value.
 struct WinGeom {
   int B, T, H, W;          // unpadded grid
@@ -33,6 +54,7 @@ struct WinGeom {
   long long o_stride;      // elements between tokens in o
   float scale_log2;        // scale * log2(e)
   int o_rows_32b;          // 1 if every output row start is 32-byte aligned
+  FastDiv div_heads, div_per_sample, div_nww, div_nwh;   // tile -> (sample, window, head)
 };
 
 // Per-axis region label on the shifted, padded grid.

@@ -44,15 +44,21 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity
   return ok != 0;
 }
 
-// Wait for phase `parity` of an mbarrier, giving up after `limit_ns` nanoseconds.
-// Returns false on timeout (the caller records the error and unwinds).
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Slow path of mbar_wait_bounded, kept out of line so that the many wait sites of the
+// kernels stay small in the instruction cache.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
+}
+
+// Wait for phase `parity` of an mbarrier, giving up after `limit_ns` nanoseconds.
+// Returns false on timeout (the caller records the error and unwinds).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, limit_ns);
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
