@@ -12,24 +12,28 @@
 //    layout, so none of them costs a global-memory pass.
 //
 // Work unit ("tile"): one (sample, window, head).  Roles (warp -> SM sub-partition w % 4):
-//   softmax warps 0-3  thread t owns TMEM lane t = query row t of S0 = Q[0:128] K^T: two
-//                      passes over the row (masked max; exp2, row sum and P rounded to bf16
-//                      into shared memory).  One tile later (the PV MMA overlaps the next
-//                      softmax) the same thread loads its O row, scales by 1/rowsum and
-//                      stores it to the query's original grid position; padded slots are
-//                      dropped.
-//   tail warp 4        the same for the 16 tail rows (S1 = Q[128:144] K^T in TMEM lanes
-//                      0..15, reachable from warp 4 like from warp 0), read with the 16x256b
+//   softmax warps 0-7  warp w owns TMEM lanes 32 (w % 4) .. +31 = query rows of
+//                      S0 = Q[0:128] K^T, and of each row the keys of half w / 4 (72 keys).
+//                      It reads its 72 logits out of TMEM once (releasing S for the next
+//                      tile), takes the masked max, swaps it with the warp holding the other
+//                      half, then exp2, the partial row sum and P rounded to bf16 into shared
+//                      memory.  One tile later (the PV MMA overlaps the next softmax) it adds
+//                      the partner's row sum, loads half of the row's O columns, scales by
+//                      1/rowsum and stores them to the query's original grid position;
+//                      padded slots are dropped.
+//   tail warp 8        the same for the 16 tail rows (S1 = Q[128:144] K^T in TMEM lanes
+//                      0..15, reachable from warp 8 like from warp 0), read with the 16x256b
 //                      shape so all 32 lanes share them.
-//   MMA warp 5         one thread issues S(t+1) as soon as tile t+1 is loaded and S(t) has
+//   MMA warp 9         one thread issues S(t+1) as soon as tile t+1 is loaded and S(t) has
 //                      left TMEM, then PV(t) = P V once P(t) is in shared memory (V read as
 //                      an MN-major operand); completion is signalled by tcgen05.commit.
-//   TMA warp 4         one thread loads the tile's Q, K and V with TMA: one box per (t, h)
-//                      run of window tokens per tensor (two where the run wraps around the
-//                      W seam), straight from grid layout into a 3-stage ring in the tensor
-//                      core's 128-byte swizzled K-major layout; padded coordinates are out
-//                      of bounds and read as zero.  It runs ahead as far as the ring allows.
-//   table warps 6-7    write the slot -> grid-token table, a bitmask of the real slots and
+//   TMA warp 10        one thread loads the tile's Q, K and V with TMA: one box per T-slab
+//                      of the window (win_h x win_w tokens) per tensor, cut where the window
+//                      wraps around a seam of the shifted grid, straight from grid layout into
+//                      a 3-stage ring in the tensor core's 128-byte swizzled K-major layout;
+//                      padded coordinates are out of bounds and read as zero.  It runs ahead
+//                      as far as the ring allows.
+//   table warp 11      writes the slot -> grid-token table, a bitmask of the real slots and
 //                      the window's "last along a shifted axis" flags (the mask of a query
 //                      follows from these) for the stage being loaded.
 // Synchronisation is by mbarriers only; every wait is bounded by a time limit and a
@@ -87,21 +91,27 @@ struct SlotConst {
 constexpr int OFF_SLOTC = OFF_TABLE + kStages * kTableBytes;
 constexpr int OFF_BARS = OFF_SLOTC + ((static_cast<int>(sizeof(SlotConst)) + 15) & ~15);
 // barriers: load[3] (TMA bytes), empty[3], table[3], s_full, s_empty, p_full, p_empty,
-// o_full, o_empty, drain
-constexpr int kNumBars = 3 * kStages + 7;
-constexpr int OFF_MISC = OFF_BARS + kNumBars * 8;   // tmem address, abort flag, producer stop
+// o_full, o_empty, drain, row max written[2], row sum written[2] (one per key half)
+constexpr int kNumBars = 3 * kStages + 11;
+// Row max / row sum of each key half of the main rows, exchanged between the two warps
+// that share a row: [tile parity][key half][row].
+constexpr int OFF_XCHG = OFF_BARS + kNumBars * 8;
+constexpr int kXchgFloats = 2 * 2 * 128;
+constexpr int OFF_MISC = OFF_XCHG + 2 * kXchgFloats * 4;   // tmem address, abort flag, producer stop
 constexpr int kSmemBytes = OFF_MISC + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1024;       // slack for the 1024-byte alignment
+static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
 
 // TMEM columns (fp32 accumulators, lane = row).  Every MMA destination is 32-aligned.
 constexpr uint32_t TM_S0 = 0, TM_S1 = 160, TM_O0 = 320, TM_O1 = 384;
 constexpr uint32_t kTmemCols = 512;
 
-constexpr int kThreads = 256;
-constexpr int kTailWarp = 4;           // tail rows 128..143 (TMEM lane quarter 0, like warp 0)
-constexpr int kMmaWarp = 5;
-constexpr int kTmaWarp = 6;
-constexpr int kFirstProducerWarp = 7;
+constexpr int kThreads = 384;
+constexpr int kMainWarps = 8;          // rows 0..127: warp w holds lanes 32 (w % 4) .., keys 72 (w / 4) ..
+constexpr int kTailWarp = 8;           // tail rows 128..143 (TMEM lane quarter 0, like warp 0)
+constexpr int kMmaWarp = 9;
+constexpr int kTmaWarp = 10;
+constexpr int kFirstProducerWarp = 11;
 constexpr int kProducerThreads = 32;   // table writer (warp 7)
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
@@ -163,6 +173,10 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
   const uint32_t o_full = bar0 + 8u * (3 * kStages + 4);
   const uint32_t o_empty = bar0 + 8u * (3 * kStages + 5);
   const uint32_t drain_bar = bar0 + 8u * (3 * kStages + 6);
+  auto xmax_bar = [&](int h) { return bar0 + 8u * (3 * kStages + 7 + h); };   // key half h wrote its row maxima
+  auto xsum_bar = [&](int h) { return bar0 + 8u * (3 * kStages + 9 + h); };   // key half h wrote its row sums
+  float* xmax = reinterpret_cast<float*>(sm + OFF_XCHG);
+  float* xsum = xmax + kXchgFloats;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sm + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
   volatile int* prod_stop = reinterpret_cast<volatile int*>(sm + OFF_MISC + 8);
@@ -171,7 +185,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
   const int warp = tid >> 5, lane = tid & 31;
   const long long num_tiles = g.windows * g.heads;
   const bool has_tail = g.N > 128;
-  const uint32_t n_soft = has_tail ? 160u : 128u;   // softmax threads: main rows (+ tail warp)
+  const uint32_t n_soft = has_tail ? 288u : 256u;   // softmax threads: main rows (+ tail warp)
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -186,6 +200,10 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     mbar_init(o_full, 1);
     mbar_init(o_empty, n_soft);
     mbar_init(drain_bar, 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(xmax_bar(h), 128);
+      mbar_init(xsum_bar(h), 128);
+    }
     *abort_flag = 0;
     *prod_stop = 0;
     fence_barrier_init();
@@ -451,15 +469,19 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       if (!mbar_wait_bounded(drain_bar, 0, 2000000000ull)) record_error(err, kStatusTimeout);
     }
     __syncwarp();
-  } else if (warp < 4 || (warp == kTailWarp && has_tail)) {
+  } else if (warp < kMainWarps || (warp == kTailWarp && has_tail)) {
     // ------------------------------------------------------------------ softmax + epilogue
-    // Warps 0-3: main rows (thread = TMEM lane = query row).  Warp 4: the 16 tail rows,
+    // Warps 0-7: main rows (thread = TMEM lane = query row); warp w takes the keys of half
+    // w / 4 (72 each) of the rows of lane quarter w % 4, and the two warps of a row swap
+    // their partial row max and row sum through shared memory.  Warp 8: the 16 tail rows,
     // read through lane quarter 0 with the 16x256b shape (for chunk j of 8 columns, this
     // lane holds columns 8j + 2qd + {0, 1} of rows ra and ra + 8), so the tail runs beside
-    // warp 0 instead of after it.
+    // the main rows instead of after them.
     const bool is_tail = warp == kTailWarp;
     const float c = g.scale_log2;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int half = (warp >> 2) & 1;                 // key half of a main-row warp
+    const int row = (warp & 3) * 32 + lane;           // its query row
     const int ra = lane >> 2, qd = lane & 3, rb = ra + 8;
     auto hi_bits_of = [&](int r) -> uint32_t {
       uint32_t h = 0;
@@ -467,7 +489,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       for (int a = 0; a < 3; ++a) h |= ((slotc->hi[a][r >> 5] >> (r & 31)) & 1u) << a;
       return h;
     };
-    const uint32_t my_hi = is_tail ? 0u : hi_bits_of(tid);
+    const uint32_t my_hi = is_tail ? 0u : hi_bits_of(row);
     const uint32_t hi_a = hi_bits_of(128 + ra), hi_b = hi_bits_of(128 + rb);
     int it = 0;
     // state of the previous tile, finished one iteration later
@@ -512,8 +534,10 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     };
 
     // Epilogue of a finished tile: O row(s) from TMEM, scaled by 1/rowsum, stored to the
-    // grid positions of the query slots (padded slots dropped).  For the tail warp `tok`
-    // / `inv` belong to row ra and `tok_b` / `inv_b` to row ra + 8.
+    // grid positions of the query slots (padded slots dropped).  A main-row warp stores
+    // the columns of its key half's number (O has head_dim columns: half h takes
+    // [h * head_dim / 2, (h + 1) * head_dim / 2)).  For the tail warp `tok` / `inv` belong
+    // to row ra and `tok_b` / `inv_b` to row ra + 8.
     auto epilogue = [&](int pit, int head, int tok, int tok_b, float inv, float inv_b) -> bool {
       bool ok = mbar_wait_bounded(o_full, pit & 1, limit_ns);
       ok = __all_sync(0xffffffffu, ok);
@@ -522,10 +546,10 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       float ov[HD];
       if (!is_tail) {
 #pragma unroll
-        for (int j = 0; j < HD / 16; ++j) tmem_ld16(tmem + lane_base + TM_O0 + 16 * j, ov + 16 * j);
+        for (int j = 0; j < HD / 32; ++j) tmem_ld16(tmem + lane_base + TM_O0 + half * (HD / 2) + 16 * j, ov + 16 * j);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < HD / 16; ++j) reg_fence16(ov + 16 * j);
+        for (int j = 0; j < HD / 32; ++j) reg_fence16(ov + 16 * j);
       } else {
 #pragma unroll
         for (int j = 0; j < HD / 8; ++j) tmem_ld_16x256b(tmem + TM_O1 + 8 * j, ov + 4 * j);
@@ -538,7 +562,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       if (!is_tail) {
         if (tok >= 0) {
 #pragma unroll
-          for (int j = 0; j < HD; j += 8) store8(tok, head, j, ov + j, inv);
+          for (int j = 0; j < HD / 2; j += 8) store8(tok, head, half * (HD / 2) + j, ov + j, inv);
         }
       } else {
 #pragma unroll
@@ -550,102 +574,79 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       return true;
     };
 
-    // Main rows, two passes over TMEM in three rolled chunks of 48 columns (144 = 3 x 48),
-    // so only 48 logits are live and the loop bodies stay small (the code of every role
-    // has to stay resident in the instruction caches): pass 1 takes the masked row max,
-    // pass 2 reloads the chunk, evaluates exp2, sums the row and stores P (bf16) into the
-    // P blocks.  For a tile whose rows of this warp all keep every key (the usual case
-    // away from the shift seams and the padding) the chunks go straight to max / exp2;
-    // otherwise masked keys become -inf first, hence weight 0.  The 144-bit mask is
-    // consumed 48 bits per chunk from a 64-bit shift register.
-    const uint32_t s0_addr = tmem + lane_base + TM_S0;
+    // Main rows: the warp's 72 logits of a row are read from TMEM once (nine 8-column
+    // loads) and stay in registers.  If any row of the warp has a masked key in this half
+    // (near the shift seams and the padding), masked keys become -inf first, hence weight
+    // 0.  The row max of the half goes to the partner warp; with the full row max, exp2,
+    // the partial row sum, and P (bf16) into the P blocks.
+    const uint32_t s_half = tmem + lane_base + TM_S0 + 72 * half;
     auto selb = [](uint64_t w, int e, float x) { return ((w >> e) & 1ull) ? x : -INFINITY; };
-    auto chunk_masks = [](const uint32_t (&mw)[kMaskWords], uint64_t& c0, uint64_t& c1, uint64_t& c2) {
-      // bits [0,48), [48,96), [96,144) of the row mask
-      c0 = (static_cast<uint64_t>(mw[0]) | (static_cast<uint64_t>(mw[1]) << 32)) & 0xffffffffffffull;
-      c1 = ((static_cast<uint64_t>(mw[1]) >> 16) | (static_cast<uint64_t>(mw[2]) << 16)) & 0xffffffffffffull;
-      c2 = (static_cast<uint64_t>(mw[3]) | (static_cast<uint64_t>(mw[4]) << 32)) & 0xffffffffffffull;
+    // bits [72 h, 72 h + 72) of a row mask: 64 in lo, 8 in hi
+    auto half_mask = [&](const uint32_t (&mw)[kMaskWords], uint64_t& lo, uint32_t& hi) {
+      const uint64_t lo0 = static_cast<uint64_t>(mw[0]) | (static_cast<uint64_t>(mw[1]) << 32);
+      const uint64_t lo1 = static_cast<uint64_t>(mw[2] >> 8) | (static_cast<uint64_t>(mw[3]) << 24) |
+                           (static_cast<uint64_t>(mw[4]) << 56);
+      lo = half ? lo1 : lo0;
+      hi = (half ? (mw[4] >> 8) : mw[2]) & 0xffu;
     };
-    // Masked keys of a chunk become -inf in place (only called for tiles with a mask).
-    auto mask_chunk = [&](float* x, uint64_t cm) {
+    auto main_row_max = [&](float (&x)[72], uint64_t mlo, uint32_t mhi, bool masked) -> float {
 #pragma unroll
-      for (int e = 0; e < 48; ++e) x[e] = selb(cm, e, x[e]);
-    };
-    auto load_chunk = [&](int i, float* x) {
-#pragma unroll
-      for (int j = 0; j < 3; ++j) tmem_ld16(s0_addr + 48 * i + 16 * j, x + 16 * j);
+      for (int j = 0; j < 9; ++j) tmem_ld8(s_half + 8 * j, x + 8 * j);
       tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 3; ++j) reg_fence16(x + 16 * j);
-    };
-    auto main_row_max = [&](const uint32_t (&mw)[kMaskWords], bool masked) -> float {
-      uint64_t c0, c1, c2;
-      chunk_masks(mw, c0, c1, c2);
-      float a = -INFINITY, b = -INFINITY;
-#pragma unroll 1
-      for (int i = 0; i < 3; ++i) {
-        float x[48];
-        load_chunk(i, x);
-        if (masked) mask_chunk(x, c0);
+      for (int j = 0; j < 9; ++j) reg_fence8(x + 8 * j);
+      if (masked) {
 #pragma unroll
-        for (int e = 0; e < 48; e += 4) {
-          a = max3(a, x[e], x[e + 1]);
-          b = max3(b, x[e + 2], x[e + 3]);
-        }
-        c0 = c1;
-        c1 = c2;
+        for (int e = 0; e < 64; ++e) x[e] = selb(mlo, e, x[e]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[64 + e] = selb(mhi, e, x[64 + e]);
       }
-      const float m = fmaxf(a, b);
-      return m == -INFINITY ? 0.f : m;
+      float a = -INFINITY, b = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 72; e += 4) {
+        a = max3(a, x[e], x[e + 1]);
+        b = max3(b, x[e + 2], x[e + 3]);
+      }
+      return fmaxf(a, b);
     };
-    auto main_row_exp = [&](const uint32_t (&mw)[kMaskWords], bool masked, float m, int row) -> float {
+    auto main_row_exp = [&](const float (&x)[72], float m) -> float {
       const float2 cc = make_float2(c, c), nm = make_float2(-m * c, -m * c);
       float2 l0 = make_float2(0.f, 0.f), l1 = make_float2(0.f, 0.f);
-      uint64_t c0, c1, c2;
-      chunk_masks(mw, c0, c1, c2);
       const uint32_t rsw = row & 7;
       const uint32_t row128 = static_cast<uint32_t>(row) * 128, row32 = static_cast<uint32_t>(row) * 32;
       const uint32_t sw32 = (row >> 2) & 1;
-#pragma unroll 1
-      for (int i = 0; i < 3; ++i) {
-        float x[48];
-        load_chunk(i, x);
-        if (masked) mask_chunk(x, c0);
 #pragma unroll
-        for (int k = 0; k < 6; ++k) {   // 8 keys: 8g .. 8g+7, g = 6i + k
-          uint32_t pk[4];
+      for (int k = 0; k < 9; ++k) {   // 8 keys: 8 g8 .. 8 g8 + 7, g8 = 9 half + k
+        uint32_t pk[4];
 #pragma unroll
-          for (int e = 0; e < 8; e += 4) {
-            const int q = 8 * k + e;
-            const float2 ya = fma2(make_float2(x[q], x[q + 1]), cc, nm);
-            const float2 yb = fma2(make_float2(x[q + 2], x[q + 3]), cc, nm);
-            const float2 pa = make_float2(ex2(ya.x), ex2(ya.y));
-            const float2 pb = make_float2(ex2(yb.x), ex2(yb.y));
-            l0 = add2(l0, pa);
-            l1 = add2(l1, pb);
-            pk[e / 2] = pack_bf16x2_int(pa.x, pa.y);
-            pk[e / 2 + 1] = pack_bf16x2_int(pb.x, pb.y);
-          }
-          const int g8 = 6 * i + k;   // 16-byte chunk of P along the keys
-          uint32_t addr;
-          if (g8 < 16)
-            addr = sb + (g8 < 8 ? OFF_P0B0 : OFF_P0B1) + row128 + ((((g8 & 7) ^ rsw)) << 4);
-          else
-            addr = sb + OFF_P0B2 + row32 + (((g8 - 16) ^ sw32) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(pk[0]), "r"(pk[1]), "r"(pk[2]),
-                       "r"(pk[3])
-                       : "memory");
+        for (int e = 0; e < 8; e += 4) {
+          const int q = 8 * k + e;
+          const float2 ya = fma2(make_float2(x[q], x[q + 1]), cc, nm);
+          const float2 yb = fma2(make_float2(x[q + 2], x[q + 3]), cc, nm);
+          const float2 pa = make_float2(ex2(ya.x), ex2(ya.y));
+          const float2 pb = make_float2(ex2(yb.x), ex2(yb.y));
+          l0 = add2(l0, pa);
+          l1 = add2(l1, pb);
+          pk[e / 2] = pack_bf16x2_int(pa.x, pa.y);
+          pk[e / 2 + 1] = pack_bf16x2_int(pb.x, pb.y);
         }
-        c0 = c1;
-        c1 = c2;
+        const int g8 = 9 * half + k;   // 16-byte chunk of P along the keys
+        uint32_t addr;
+        if (g8 < 16)
+          addr = sb + (g8 < 8 ? OFF_P0B0 : OFF_P0B1) + row128 + ((((g8 & 7) ^ rsw)) << 4);
+        else
+          addr = sb + OFF_P0B2 + row32 + (((g8 - 16) ^ sw32) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(pk[0]), "r"(pk[1]), "r"(pk[2]),
+                     "r"(pk[3])
+                     : "memory");
       }
       const float2 l2 = add2(l0, l1);
-      const float l = l2.x + l2.y;
-      return l > 0.f ? 1.f / l : 0.f;
+      return l2.x + l2.y;
     };
 
-    // Tail rows (warp 4): same two passes, 2 x 9 chunks of 8 columns; row max and sum finish
-    // with two shuffles among the four lanes (qd = 0..3) sharing a row.
+    // Tail rows (warp 8): the same steps on 18 chunks of 8 columns, all held in registers;
+    // row max and sum finish with two shuffles among the four lanes (qd = 0..3) sharing a
+    // row.
     auto lane_bits = [&](const uint32_t (&m)[kMaskWords]) -> uint64_t {   // bit 2j+e: column 8j+2qd+e
       uint64_t r = 0;
 #pragma unroll
@@ -653,24 +654,28 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         r |= static_cast<uint64_t>((m[j >> 2] >> (8 * (j & 3) + 2 * qd)) & 3u) << (2 * j);
       return r;
     };
-    auto tail_max = [&](uint64_t ba, uint64_t bb, float& m_a, float& m_b) {
+    auto tail_max = [&](float (&x)[72], uint64_t ba, uint64_t bb, float& m_a, float& m_b) {
+#pragma unroll
+      for (int j = 0; j < 18; ++j) tmem_ld_16x256b(tmem + TM_S1 + 8 * j, x + 4 * j);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 18; ++j) reg_fence4(x + 4 * j);
+      constexpr uint64_t kAll = (1ull << 36) - 1;
+      if (!__all_sync(0xffffffffu, ba == kAll && bb == kAll)) {
+#pragma unroll
+        for (int j = 0; j < 18; ++j) {
+          x[4 * j] = selb(ba, 2 * j, x[4 * j]);
+          x[4 * j + 1] = selb(ba, 2 * j + 1, x[4 * j + 1]);
+          x[4 * j + 2] = selb(bb, 2 * j, x[4 * j + 2]);
+          x[4 * j + 3] = selb(bb, 2 * j + 1, x[4 * j + 3]);
+        }
+      }
       m_a = -INFINITY;
       m_b = -INFINITY;
-#pragma unroll 1
-      for (int i = 0; i < 2; ++i) {
-        float x[36];
 #pragma unroll
-        for (int k = 0; k < 9; ++k) tmem_ld_16x256b(tmem + TM_S1 + 8 * (9 * i + k), x + 4 * k);
-        tmem_wait_ld();
-#pragma unroll
-        for (int k = 0; k < 9; ++k) reg_fence4(x + 4 * k);
-#pragma unroll
-        for (int k = 0; k < 9; ++k) {
-          m_a = max3(m_a, selb(ba, 2 * k, x[4 * k]), selb(ba, 2 * k + 1, x[4 * k + 1]));
-          m_b = max3(m_b, selb(bb, 2 * k, x[4 * k + 2]), selb(bb, 2 * k + 1, x[4 * k + 3]));
-        }
-        ba >>= 18;
-        bb >>= 18;
+      for (int j = 0; j < 18; ++j) {
+        m_a = max3(m_a, x[4 * j], x[4 * j + 1]);
+        m_b = max3(m_b, x[4 * j + 2], x[4 * j + 3]);
       }
       m_a = fmaxf(m_a, __shfl_xor_sync(0xffffffffu, m_a, 1));
       m_a = fmaxf(m_a, __shfl_xor_sync(0xffffffffu, m_a, 2));
@@ -679,45 +684,32 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       if (m_a == -INFINITY) m_a = 0.f;
       if (m_b == -INFINITY) m_b = 0.f;
     };
-    auto tail_exp = [&](uint64_t ba, uint64_t bb, float m_a, float m_b, float& inv_a, float& inv_b) {
+    auto tail_exp = [&](const float (&x)[72], float m_a, float m_b, float& inv_a, float& inv_b) {
       const float2 cc = make_float2(c, c);
       const float2 na = make_float2(-m_a * c, -m_a * c), nb = make_float2(-m_b * c, -m_b * c);
       float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
-#pragma unroll 1
-      for (int i = 0; i < 2; ++i) {
-        float x[36];
 #pragma unroll
-        for (int k = 0; k < 9; ++k) tmem_ld_16x256b(tmem + TM_S1 + 8 * (9 * i + k), x + 4 * k);
-        tmem_wait_ld();
-#pragma unroll
-        for (int k = 0; k < 9; ++k) reg_fence4(x + 4 * k);
-#pragma unroll
-        for (int k = 0; k < 9; ++k) {
-          const float2 ya = fma2(make_float2(selb(ba, 2 * k, x[4 * k]), selb(ba, 2 * k + 1, x[4 * k + 1])), cc, na);
-          const float2 yb =
-              fma2(make_float2(selb(bb, 2 * k, x[4 * k + 2]), selb(bb, 2 * k + 1, x[4 * k + 3])), cc, nb);
-          const float2 pa = make_float2(ex2(ya.x), ex2(ya.y));
-          const float2 pb = make_float2(ex2(yb.x), ex2(yb.y));
-          la = add2(la, pa);
-          lb = add2(lb, pb);
-          // chunk j = 9i + k: keys 8j .. 8j+7 -> block j / 8 (the third block is 32B-swizzled)
-          const int j = 9 * i + k;
-          uint32_t addr_a, addr_b;
-          if (j < 16) {
-            const uint32_t blk = sb + (j < 8 ? OFF_P1B0 : OFF_P1B1);
-            const int ch = j & 7;
-            addr_a = blk + ra * 128 + ((ch ^ (ra & 7)) << 4) + 4 * qd;
-            addr_b = blk + rb * 128 + ((ch ^ (rb & 7)) << 4) + 4 * qd;
-          } else {
-            const int ch = j - 16;
-            addr_a = sb + OFF_P1B2 + ra * 32 + ((ch ^ ((ra >> 2) & 1)) << 4) + 4 * qd;
-            addr_b = sb + OFF_P1B2 + rb * 32 + ((ch ^ ((rb >> 2) & 1)) << 4) + 4 * qd;
-          }
-          asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr_a), "r"(pack_bf16x2_int(pa.x, pa.y)) : "memory");
-          asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr_b), "r"(pack_bf16x2_int(pb.x, pb.y)) : "memory");
+      for (int j = 0; j < 18; ++j) {
+        const float2 ya = fma2(make_float2(x[4 * j], x[4 * j + 1]), cc, na);
+        const float2 yb = fma2(make_float2(x[4 * j + 2], x[4 * j + 3]), cc, nb);
+        const float2 pa = make_float2(ex2(ya.x), ex2(ya.y));
+        const float2 pb = make_float2(ex2(yb.x), ex2(yb.y));
+        la = add2(la, pa);
+        lb = add2(lb, pb);
+        // chunk j: keys 8j .. 8j+7 -> block j / 8 (the third block is 32B-swizzled)
+        uint32_t addr_a, addr_b;
+        if (j < 16) {
+          const uint32_t blk = sb + (j < 8 ? OFF_P1B0 : OFF_P1B1);
+          const int ch = j & 7;
+          addr_a = blk + ra * 128 + ((ch ^ (ra & 7)) << 4) + 4 * qd;
+          addr_b = blk + rb * 128 + ((ch ^ (rb & 7)) << 4) + 4 * qd;
+        } else {
+          const int ch = j - 16;
+          addr_a = sb + OFF_P1B2 + ra * 32 + ((ch ^ ((ra >> 2) & 1)) << 4) + 4 * qd;
+          addr_b = sb + OFF_P1B2 + rb * 32 + ((ch ^ ((rb >> 2) & 1)) << 4) + 4 * qd;
         }
-        ba >>= 18;
-        bb >>= 18;
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr_a), "r"(pack_bf16x2_int(pa.x, pa.y)) : "memory");
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr_b), "r"(pack_bf16x2_int(pb.x, pb.y)) : "memory");
       }
       float sa = la.x + la.y, sbm = lb.x + lb.y;
       sa += __shfl_xor_sync(0xffffffffu, sa, 1);
@@ -730,8 +722,21 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
 
     // Iteration `it` does the softmax of tile `it` (if any) and then the epilogue of tile
     // it-1, so the PV MMA of a tile overlaps the next tile's softmax.  One call site each.
+    // S is read out of TMEM into registers in one go, so it is released (s_empty) before
+    // the exponentials, and the MMA warp can compute the next tile's S underneath them.
     for (long long tile = blockIdx.x;; tile += gridDim.x, ++it) {
       const bool have_cur = tile < num_tiles;
+      if (have_prev && !is_tail) {
+        // The partner warp's row sum of the previous tile.  Taken here, before this warp's
+        // next arrival on an exchange barrier, so the partner can never be two phases ahead.
+        const bool ok = mbar_wait_bounded(xsum_bar(half ^ 1), prev_it & 1, limit_ns);
+        if (!__all_sync(0xffffffffu, ok)) {
+          aborted = true;
+          break;
+        }
+        const float l = prev_inv + xsum[((prev_it & 1) * 2 + (half ^ 1)) * 128 + row];
+        prev_inv = l > 0.f ? 1.f / l : 0.f;
+      }
       int head = 0, tok = -1, tok_b = -1;
       float inv = 0.f, inv_b = 0.f;
       if (have_cur) {
@@ -751,7 +756,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         const uint32_t last = tb.last;
         uint32_t mw[kMaskWords], mb[kMaskWords];
         if (!is_tail) {
-          tok = tb.tok[tid];
+          tok = tb.tok[row];
           build_mask(tb, *slotc, last, my_hi, mw);
         } else {
           tok = tb.tok[128 + ra];   // row ra, mask in mw
@@ -767,30 +772,44 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
           break;
         }
         tc_fence_after();
+        float x[72];
         float mrow = 0.f, mrow_b = 0.f;
-        uint64_t ba = 0, bb = 0;
-        bool masked = false;
+        const int par = it & 1;
         if (!is_tail) {
-          masked = !__all_sync(0xffffffffu, ((mw[0] & mw[1] & mw[2] & mw[3]) == 0xffffffffu) &&
-                                                ((mw[4] & 0xffffu) == 0xffffu));
-          mrow = main_row_max(mw, masked);
+          uint64_t mlo;
+          uint32_t mhi;
+          half_mask(mw, mlo, mhi);
+          const bool masked = !__all_sync(0xffffffffu, mlo == ~0ull && mhi == 0xffu);
+          const float mh = main_row_max(x, mlo, mhi, masked);
+          tc_fence_before();
+          mbar_arrive(s_empty);   // S of this thread is in registers: the next S may be written
+          xmax[(par * 2 + half) * 128 + row] = mh;
+          mbar_arrive(xmax_bar(half));
+          ok = mbar_wait_bounded(xmax_bar(half ^ 1), par, limit_ns);
+          if (!__all_sync(0xffffffffu, ok)) {
+            aborted = true;
+            break;
+          }
+          mrow = fmaxf(mh, xmax[(par * 2 + (half ^ 1)) * 128 + row]);
+          if (mrow == -INFINITY) mrow = 0.f;
         } else {
-          ba = lane_bits(mw);
-          bb = lane_bits(mb);
-          tail_max(ba, bb, mrow, mrow_b);
+          tail_max(x, lane_bits(mw), lane_bits(mb), mrow, mrow_b);
+          tc_fence_before();
+          mbar_arrive(s_empty);
         }
         // P may only be overwritten once the previous tile's PV MMA has consumed it.
-        ok = mbar_wait_bounded(p_empty, (it & 1) ^ 1, limit_ns);
+        ok = mbar_wait_bounded(p_empty, par ^ 1, limit_ns);
         if (!__all_sync(0xffffffffu, ok)) {
           aborted = true;
           break;
         }
-        if (!is_tail)
-          inv = main_row_exp(mw, masked, mrow, tid);
-        else
-          tail_exp(ba, bb, mrow, mrow_b, inv, inv_b);
-        tc_fence_before();
-        mbar_arrive(s_empty);   // every S read of this thread is done: the next tile's S may be written
+        if (!is_tail) {
+          inv = main_row_exp(x, mrow);   // the half's row sum; 1 / (full sum) next iteration
+          xsum[(par * 2 + half) * 128 + row] = inv;
+          mbar_arrive(xsum_bar(half));
+        } else {
+          tail_exp(x, mrow, mrow_b, inv, inv_b);
+        }
         fence_proxy_async_smem();
         mbar_arrive(p_full);
       }

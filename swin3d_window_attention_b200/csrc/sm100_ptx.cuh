@@ -123,6 +123,16 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
         "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
       : "r"(taddr));
 }
+// 32 lanes x 32 bits, 8 consecutive columns (start column a multiple of 8).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void reg_fence8(float* v) {
+  asm volatile("" : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]),
+               "+f"(v[7]));
+}
 // 16 lanes x 256 bits (8 columns): thread t gets lanes base + t/4 and base + 8 + t/4,
 // columns 2*(t%4) and 2*(t%4)+1: v = {(r, c), (r, c+1), (r+8, c), (r+8, c+1)}.
 __device__ __forceinline__ void tmem_ld_16x256b(uint32_t taddr, float* v) {
