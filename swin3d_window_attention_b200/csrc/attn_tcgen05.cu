@@ -315,7 +315,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
           t -= t >= g.Pt ? g.Pt : 0;
           const uint32_t slab = stage + rt * g.wh * run_bytes;
           if (!wrap_w) {
-#pragma unroll
+#pragma unroll 1
             for (int tsr = 0; tsr < 3; ++tsr) {
               const uint32_t d = slab + tsr * kTileBytes;
               if (!wrap_h) {
@@ -330,7 +330,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
 #pragma unroll 1
             for (int rh = 0; rh < g.wh; ++rh) {
               const uint32_t dst = slab + rh * run_bytes;
-#pragma unroll
+#pragma unroll 1
               for (int tsr = 0; tsr < 3; ++tsr) {
                 const uint32_t d = dst + tsr * kTileBytes;
                 tma_load_5d(d, &maps.m[tsr][kBoxSeamW1], c0, tc.bw, h, t, tc.bsmp, bar);
@@ -379,10 +379,12 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         return ((tc.bsmp * g.T + t) * g.H + h) * g.W + w;
       };
       Table& tb = tables[s];
+#pragma unroll 1
       for (int r = p; r < kN; r += kProducerThreads) tb.tok[r] = resolve(r);
       if (p == 0)
         tb.last = ((tc.itw == g.nwt - 1 && g.st > 0) ? 1u : 0u) | ((tc.ih == g.nwh - 1 && g.sh > 0) ? 2u : 0u) |
                   ((tc.iw == g.nww - 1 && g.sw > 0) ? 4u : 0u);
+#pragma unroll 1
       for (int wd = p >> 5; wd < kMaskWords; wd += kProducerThreads / 32) {
         const int r = 32 * wd + lane;
         const unsigned m = __ballot_sync(0xffffffffu, r < kN && resolve(r) >= 0);
@@ -405,14 +407,12 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       fence_proxy_async_smem();
       tc_fence_after();
       const uint32_t qa = sb + OFF_STAGE + s * kStageBytes, ka = qa + kTileBytes;
-#pragma unroll
-      for (int kk = 0; kk < HD / 16; ++kk)
-        umma_bf16_ss(tmem + TM_S0, desc_kmajor_sw128(qa + kk * 32), desc_kmajor_sw128(ka + kk * 32), idesc_s, kk > 0);
-      if (has_tail) {
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk)
-          umma_bf16_ss(tmem + TM_S1, desc_kmajor_sw128(qa + 128 * kRowBytes + kk * 32),
-                       desc_kmajor_sw128(ka + kk * 32), idesc_s, kk > 0);
+#pragma unroll 1
+      for (int kk = 0; kk < HD / 16; ++kk) {
+        const uint64_t kd = desc_kmajor_sw128(ka + kk * 32);
+        umma_bf16_ss(tmem + TM_S0, desc_kmajor_sw128(qa + kk * 32), kd, idesc_s, kk > 0);
+        if (has_tail)
+          umma_bf16_ss(tmem + TM_S1, desc_kmajor_sw128(qa + 128 * kRowBytes + kk * 32), kd, idesc_s, kk > 0);
       }
       umma_commit(s_full);
       issued = true;
@@ -424,18 +424,17 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       if (!mbar_wait_bounded(o_empty, (jt & 1) ^ 1, limit_ns)) return false;
       tc_fence_after();
       const uint32_t va = sb + OFF_STAGE + s * kStageBytes + 2 * kTileBytes;
-#pragma unroll
+#pragma unroll 1
       for (int kk = 0; kk < kN / 16; ++kk) {
         const uint64_t vd = desc_mnmajor_sw128(va + kk * 2048);
-        const uint64_t pd0 = kk < 8 ? desc_kmajor_sw128(sb + (kk < 4 ? OFF_P0B0 : OFF_P0B1) + (kk & 3) * 32)
+        // keys 16kk .. 16kk + 15 of P: blocks of 64 keys (128B swizzle), the last 16 keys
+        // in the 32B-swizzled block
+        const uint32_t koff = static_cast<uint32_t>((kk & 3) * 32);
+        const uint64_t pd0 = kk < 8 ? desc_kmajor_sw128(sb + OFF_P0B0 + (kk >> 2) * (OFF_P0B1 - OFF_P0B0) + koff)
                                     : desc_kmajor_sw32(sb + OFF_P0B2);
         umma_bf16_ss(tmem + TM_O0, pd0, vd, idesc_o, kk > 0);
-      }
-      if (has_tail) {
-#pragma unroll
-        for (int kk = 0; kk < kN / 16; ++kk) {
-          const uint64_t vd = desc_mnmajor_sw128(va + kk * 2048);
-          const uint64_t pd1 = kk < 8 ? desc_kmajor_sw128(sb + (kk < 4 ? OFF_P1B0 : OFF_P1B1) + (kk & 3) * 32)
+        if (has_tail) {
+          const uint64_t pd1 = kk < 8 ? desc_kmajor_sw128(sb + OFF_P1B0 + (kk >> 2) * (OFF_P1B1 - OFF_P1B0) + koff)
                                       : desc_kmajor_sw32(sb + OFF_P1B2);
           umma_bf16_ss(tmem + TM_O1, pd1, vd, idesc_o, kk > 0);
         }
@@ -471,31 +470,38 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     __syncwarp();
   } else if (warp < kMainWarps || (warp == kTailWarp && has_tail)) {
     // ------------------------------------------------------------------ softmax + epilogue
-    // Warps 0-7: main rows (thread = TMEM lane = query row); warp w takes the keys of half
-    // w / 4 (72 each) of the rows of lane quarter w % 4, and the two warps of a row swap
-    // their partial row max and row sum through shared memory.  Warp 8: the 16 tail rows,
-    // read through lane quarter 0 with the 16x256b shape (for chunk j of 8 columns, this
-    // lane holds columns 8j + 2qd + {0, 1} of rows ra and ra + 8), so the tail runs beside
-    // the main rows instead of after them.
+    // Every softmax thread owns one (query row, key half) and runs the same code.  Half h
+    // holds the key groups 2k + h (k = 0..8) of 8 keys each, 72 keys.  Main warp w: row
+    // 32 (w % 4) + lane (its TMEM lane in S0 = Q[0:128] K^T), half w / 4, read with the
+    // 32x32b shape at column 16k + 8h; its partner (same row, other half) is warp w ^ 4,
+    // and the two swap row max and row sum through shared memory.  Tail warp 8: row
+    // 128 + lane % 16 (TMEM lane lane % 16 of S1 = Q[128:144] K^T), half lane / 16, read
+    // with the 16x32bx2 shape (threads 16..31 see the columns 8 further on); its partner is
+    // lane ^ 16 of the same warp (a shuffle).
     const bool is_tail = warp == kTailWarp;
     const float c = g.scale_log2;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const int half = (warp >> 2) & 1;                 // key half of a main-row warp
-    const int row = (warp & 3) * 32 + lane;           // its query row
-    const int ra = lane >> 2, qd = lane & 3, rb = ra + 8;
-    auto hi_bits_of = [&](int r) -> uint32_t {
+    const int half = is_tail ? (lane >> 4) : ((warp >> 2) & 1);
+    const int row = is_tail ? 128 + (lane & 15) : (warp & 3) * 32 + lane;
+    const int lrow = is_tail ? (lane & 15) : row;   // row inside its P blocks
+    const uint32_t pb0 = sb + (is_tail ? OFF_P1B0 : OFF_P0B0);
+    const uint32_t pb1 = sb + (is_tail ? OFF_P1B1 : OFF_P0B1);
+    const uint32_t pb2 = sb + (is_tail ? OFF_P1B2 : OFF_P0B2);
+    const uint32_t s_base = is_tail ? tmem + TM_S1 : tmem + lane_base + TM_S0 + 8 * half;
+    // O columns of a thread: groups of 16, 32m + 16h .. +15 (m < head_dim / 32); the main
+    // rows take them with 32x32b at that column, the tail with 16x32bx2 at column 32m.
+    const uint32_t o_base = is_tail ? tmem + TM_O1 : tmem + lane_base + TM_O0 + 16 * half;
+    const uint32_t my_hi = [&] {
       uint32_t h = 0;
 #pragma unroll
-      for (int a = 0; a < 3; ++a) h |= ((slotc->hi[a][r >> 5] >> (r & 31)) & 1u) << a;
+      for (int a = 0; a < 3; ++a) h |= ((slotc->hi[a][row >> 5] >> (row & 31)) & 1u) << a;
       return h;
-    };
-    const uint32_t my_hi = is_tail ? 0u : hi_bits_of(row);
-    const uint32_t hi_a = hi_bits_of(128 + ra), hi_b = hi_bits_of(128 + rb);
+    }();
     int it = 0;
     // state of the previous tile, finished one iteration later
     bool have_prev = false;
-    int prev_it = 0, prev_head = 0, prev_tok = -1, prev_tok_b = -1;
-    float prev_inv = 0.f, prev_inv_b = 0.f;
+    int prev_it = 0, prev_head = 0, prev_tok = -1;
+    float prev_inv = 0.f;
     bool aborted = false;
 
     auto store8 = [&](int tk, int head, int col, const float* vals, float scl) {
@@ -522,84 +528,62 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         *reinterpret_cast<uint4*>(dst) = u;
       }
     };
-    auto store2 = [&](int tk, int head, int col, float a, float b, float scl) {
-      if constexpr (OUT_F32) {
-        float* dst = static_cast<float*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD + col;
-        *reinterpret_cast<float2*>(dst) = make_float2(a * scl, b * scl);
-      } else {
-        __nv_bfloat16* dst =
-            static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD + col;
-        *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(a * scl, b * scl);
-      }
-    };
 
-    // Epilogue of a finished tile: O row(s) from TMEM, scaled by 1/rowsum, stored to the
-    // grid positions of the query slots (padded slots dropped).  A main-row warp stores
-    // the columns of its key half's number (O has head_dim columns: half h takes
-    // [h * head_dim / 2, (h + 1) * head_dim / 2)).  For the tail warp `tok` / `inv` belong
-    // to row ra and `tok_b` / `inv_b` to row ra + 8.
-    auto epilogue = [&](int pit, int head, int tok, int tok_b, float inv, float inv_b) -> bool {
+    // Epilogue of a finished tile: this thread's O columns from TMEM, scaled by 1/rowsum,
+    // stored to the grid position of the query slot (padded slots dropped).
+    auto epilogue = [&](int pit, int head, int tok, float inv) -> bool {
       bool ok = mbar_wait_bounded(o_full, pit & 1, limit_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) return false;
       tc_fence_after();
-      float ov[HD];
+      float ov[HD / 2];
       if (!is_tail) {
 #pragma unroll
-        for (int j = 0; j < HD / 32; ++j) tmem_ld16(tmem + lane_base + TM_O0 + half * (HD / 2) + 16 * j, ov + 16 * j);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < HD / 32; ++j) reg_fence16(ov + 16 * j);
+        for (int m = 0; m < HD / 32; ++m) tmem_ld16(o_base + 32 * m, ov + 16 * m);
       } else {
 #pragma unroll
-        for (int j = 0; j < HD / 8; ++j) tmem_ld_16x256b(tmem + TM_O1 + 8 * j, ov + 4 * j);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < HD / 8; ++j) reg_fence4(ov + 4 * j);
+        for (int m = 0; m < HD / 32; ++m) tmem_ld_16x32bx2_x16(o_base + 32 * m, ov + 16 * m);
       }
+      tmem_wait_ld();
+#pragma unroll
+      for (int m = 0; m < HD / 32; ++m) reg_fence16(ov + 16 * m);
       tc_fence_before();
       mbar_arrive(o_empty);
-      if (!is_tail) {
-        if (tok >= 0) {
+      if (tok >= 0) {
 #pragma unroll
-          for (int j = 0; j < HD / 2; j += 8) store8(tok, head, half * (HD / 2) + j, ov + j, inv);
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < HD / 8; ++j) {
-          if (tok >= 0) store2(tok, head, 8 * j + 2 * qd, ov[4 * j], ov[4 * j + 1], inv);
-          if (tok_b >= 0) store2(tok_b, head, 8 * j + 2 * qd, ov[4 * j + 2], ov[4 * j + 3], inv_b);
+        for (int m = 0; m < HD / 32; ++m) {
+          store8(tok, head, 32 * m + 16 * half, ov + 16 * m, inv);
+          store8(tok, head, 32 * m + 16 * half + 8, ov + 16 * m + 8, inv);
         }
       }
       return true;
     };
 
-    // Main rows: the warp's 72 logits of a row are read from TMEM once (nine 8-column
-    // loads) and stay in registers.  If any row of the warp has a masked key in this half
-    // (near the shift seams and the padding), masked keys become -inf first, hence weight
-    // 0.  The row max of the half goes to the partner warp; with the full row max, exp2,
-    // the partial row sum, and P (bf16) into the P blocks.
-    const uint32_t s_half = tmem + lane_base + TM_S0 + 72 * half;
-    auto selb = [](uint64_t w, int e, float x) { return ((w >> e) & 1ull) ? x : -INFINITY; };
-    // bits [72 h, 72 h + 72) of a row mask: 64 in lo, 8 in hi
-    auto half_mask = [&](const uint32_t (&mw)[kMaskWords], uint64_t& lo, uint32_t& hi) {
-      const uint64_t lo0 = static_cast<uint64_t>(mw[0]) | (static_cast<uint64_t>(mw[1]) << 32);
-      const uint64_t lo1 = static_cast<uint64_t>(mw[2] >> 8) | (static_cast<uint64_t>(mw[3]) << 24) |
-                           (static_cast<uint64_t>(mw[4]) << 56);
-      lo = half ? lo1 : lo0;
-      hi = (half ? (mw[4] >> 8) : mw[2]) & 0xffu;
-    };
-    auto main_row_max = [&](float (&x)[72], uint64_t mlo, uint32_t mhi, bool masked) -> float {
+    // The thread's 72 logits are read from TMEM once (nine 8-column loads) and stay in
+    // registers.  If any thread of the warp has a masked key (near the shift seams and the
+    // padding), masked keys become -inf first, hence weight 0.
+    auto selb = [](uint32_t w, int e, float x) { return ((w >> e) & 1u) ? x : -INFINITY; };
+    auto row_max = [&](float (&x)[72], const uint32_t (&mw)[kMaskWords]) -> float {
+      if (!is_tail) {
 #pragma unroll
-      for (int j = 0; j < 9; ++j) tmem_ld8(s_half + 8 * j, x + 8 * j);
+        for (int k = 0; k < 9; ++k) tmem_ld8(s_base + 16 * k, x + 8 * k);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 9; ++k) tmem_ld_16x32bx2_x8(s_base + 16 * k, x + 8 * k);
+      }
       tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 9; ++j) reg_fence8(x + 8 * j);
-      if (masked) {
+      for (int k = 0; k < 9; ++k) reg_fence8(x + 8 * k);
+      // key group 2k + h = row-mask bits [16k + 8h, +8)
+      uint32_t kb[9];
 #pragma unroll
-        for (int e = 0; e < 64; ++e) x[e] = selb(mlo, e, x[e]);
+      for (int k = 0; k < 9; ++k) kb[k] = (mw[k >> 1] >> (16 * (k & 1) + 8 * half)) & 0xffu;
+      const uint32_t all = kb[0] & kb[1] & kb[2] & kb[3] & kb[4] & kb[5] & kb[6] & kb[7] & kb[8];
+      if (!__all_sync(0xffffffffu, all == 0xffu)) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[64 + e] = selb(mhi, e, x[64 + e]);
+        for (int k = 0; k < 9; ++k)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[8 * k + e] = selb(kb[k], e, x[8 * k + e]);
       }
       float a = -INFINITY, b = -INFINITY;
 #pragma unroll
@@ -609,14 +593,15 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       }
       return fmaxf(a, b);
     };
-    auto main_row_exp = [&](const float (&x)[72], float m) -> float {
+    // exp2, the half's row sum, and P (bf16) into the P blocks.
+    auto row_exp = [&](const float (&x)[72], float m) -> float {
       const float2 cc = make_float2(c, c), nm = make_float2(-m * c, -m * c);
       float2 l0 = make_float2(0.f, 0.f), l1 = make_float2(0.f, 0.f);
-      const uint32_t rsw = row & 7;
-      const uint32_t row128 = static_cast<uint32_t>(row) * 128, row32 = static_cast<uint32_t>(row) * 32;
-      const uint32_t sw32 = (row >> 2) & 1;
+      const uint32_t rsw = lrow & 7;
+      const uint32_t row128 = static_cast<uint32_t>(lrow) * 128, row32 = static_cast<uint32_t>(lrow) * 32;
+      const uint32_t sw32 = (lrow >> 2) & 1;
 #pragma unroll
-      for (int k = 0; k < 9; ++k) {   // 8 keys: 8 g8 .. 8 g8 + 7, g8 = 9 half + k
+      for (int k = 0; k < 9; ++k) {
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 8; e += 4) {
@@ -630,94 +615,18 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
           pk[e / 2] = pack_bf16x2_int(pa.x, pa.y);
           pk[e / 2 + 1] = pack_bf16x2_int(pb.x, pb.y);
         }
-        const int g8 = 9 * half + k;   // 16-byte chunk of P along the keys
+        const int g8 = 2 * k + half;   // 16-byte chunk of P along the keys
         uint32_t addr;
-        if (g8 < 16)
-          addr = sb + (g8 < 8 ? OFF_P0B0 : OFF_P0B1) + row128 + ((((g8 & 7) ^ rsw)) << 4);
+        if (k < 8)
+          addr = (k < 4 ? pb0 : pb1) + row128 + ((((g8 & 7) ^ rsw)) << 4);
         else
-          addr = sb + OFF_P0B2 + row32 + (((g8 - 16) ^ sw32) << 4);
+          addr = pb2 + row32 + (((g8 - 16) ^ sw32) << 4);
         asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(pk[0]), "r"(pk[1]), "r"(pk[2]),
                      "r"(pk[3])
                      : "memory");
       }
       const float2 l2 = add2(l0, l1);
       return l2.x + l2.y;
-    };
-
-    // Tail rows (warp 8): the same steps on 18 chunks of 8 columns, all held in registers;
-    // row max and sum finish with two shuffles among the four lanes (qd = 0..3) sharing a
-    // row.
-    auto lane_bits = [&](const uint32_t (&m)[kMaskWords]) -> uint64_t {   // bit 2j+e: column 8j+2qd+e
-      uint64_t r = 0;
-#pragma unroll
-      for (int j = 0; j < kN / 8; ++j)
-        r |= static_cast<uint64_t>((m[j >> 2] >> (8 * (j & 3) + 2 * qd)) & 3u) << (2 * j);
-      return r;
-    };
-    auto tail_max = [&](float (&x)[72], uint64_t ba, uint64_t bb, float& m_a, float& m_b) {
-#pragma unroll
-      for (int j = 0; j < 18; ++j) tmem_ld_16x256b(tmem + TM_S1 + 8 * j, x + 4 * j);
-      tmem_wait_ld();
-#pragma unroll
-      for (int j = 0; j < 18; ++j) reg_fence4(x + 4 * j);
-      constexpr uint64_t kAll = (1ull << 36) - 1;
-      if (!__all_sync(0xffffffffu, ba == kAll && bb == kAll)) {
-#pragma unroll
-        for (int j = 0; j < 18; ++j) {
-          x[4 * j] = selb(ba, 2 * j, x[4 * j]);
-          x[4 * j + 1] = selb(ba, 2 * j + 1, x[4 * j + 1]);
-          x[4 * j + 2] = selb(bb, 2 * j, x[4 * j + 2]);
-          x[4 * j + 3] = selb(bb, 2 * j + 1, x[4 * j + 3]);
-        }
-      }
-      m_a = -INFINITY;
-      m_b = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < 18; ++j) {
-        m_a = max3(m_a, x[4 * j], x[4 * j + 1]);
-        m_b = max3(m_b, x[4 * j + 2], x[4 * j + 3]);
-      }
-      m_a = fmaxf(m_a, __shfl_xor_sync(0xffffffffu, m_a, 1));
-      m_a = fmaxf(m_a, __shfl_xor_sync(0xffffffffu, m_a, 2));
-      m_b = fmaxf(m_b, __shfl_xor_sync(0xffffffffu, m_b, 1));
-      m_b = fmaxf(m_b, __shfl_xor_sync(0xffffffffu, m_b, 2));
-      if (m_a == -INFINITY) m_a = 0.f;
-      if (m_b == -INFINITY) m_b = 0.f;
-    };
-    auto tail_exp = [&](const float (&x)[72], float m_a, float m_b, float& inv_a, float& inv_b) {
-      const float2 cc = make_float2(c, c);
-      const float2 na = make_float2(-m_a * c, -m_a * c), nb = make_float2(-m_b * c, -m_b * c);
-      float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int j = 0; j < 18; ++j) {
-        const float2 ya = fma2(make_float2(x[4 * j], x[4 * j + 1]), cc, na);
-        const float2 yb = fma2(make_float2(x[4 * j + 2], x[4 * j + 3]), cc, nb);
-        const float2 pa = make_float2(ex2(ya.x), ex2(ya.y));
-        const float2 pb = make_float2(ex2(yb.x), ex2(yb.y));
-        la = add2(la, pa);
-        lb = add2(lb, pb);
-        // chunk j: keys 8j .. 8j+7 -> block j / 8 (the third block is 32B-swizzled)
-        uint32_t addr_a, addr_b;
-        if (j < 16) {
-          const uint32_t blk = sb + (j < 8 ? OFF_P1B0 : OFF_P1B1);
-          const int ch = j & 7;
-          addr_a = blk + ra * 128 + ((ch ^ (ra & 7)) << 4) + 4 * qd;
-          addr_b = blk + rb * 128 + ((ch ^ (rb & 7)) << 4) + 4 * qd;
-        } else {
-          const int ch = j - 16;
-          addr_a = sb + OFF_P1B2 + ra * 32 + ((ch ^ ((ra >> 2) & 1)) << 4) + 4 * qd;
-          addr_b = sb + OFF_P1B2 + rb * 32 + ((ch ^ ((rb >> 2) & 1)) << 4) + 4 * qd;
-        }
-        asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr_a), "r"(pack_bf16x2_int(pa.x, pa.y)) : "memory");
-        asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr_b), "r"(pack_bf16x2_int(pb.x, pb.y)) : "memory");
-      }
-      float sa = la.x + la.y, sbm = lb.x + lb.y;
-      sa += __shfl_xor_sync(0xffffffffu, sa, 1);
-      sa += __shfl_xor_sync(0xffffffffu, sa, 2);
-      sbm += __shfl_xor_sync(0xffffffffu, sbm, 1);
-      sbm += __shfl_xor_sync(0xffffffffu, sbm, 2);
-      inv_a = sa > 0.f ? 1.f / sa : 0.f;
-      inv_b = sbm > 0.f ? 1.f / sbm : 0.f;
     };
 
     // Iteration `it` does the softmax of tile `it` (if any) and then the epilogue of tile
@@ -737,8 +646,8 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         const float l = prev_inv + xsum[((prev_it & 1) * 2 + (half ^ 1)) * 128 + row];
         prev_inv = l > 0.f ? 1.f / l : 0.f;
       }
-      int head = 0, tok = -1, tok_b = -1;
-      float inv = 0.f, inv_b = 0.f;
+      int head = 0, tok = -1;
+      float inv = 0.f;
       if (have_cur) {
         const int s = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
@@ -753,17 +662,9 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         }
         head = static_cast<int>(tile) - fdiv(static_cast<int>(tile), g.div_heads) * g.heads;
         const Table& tb = tables[s];
-        const uint32_t last = tb.last;
-        uint32_t mw[kMaskWords], mb[kMaskWords];
-        if (!is_tail) {
-          tok = tb.tok[row];
-          build_mask(tb, *slotc, last, my_hi, mw);
-        } else {
-          tok = tb.tok[128 + ra];   // row ra, mask in mw
-          tok_b = tb.tok[128 + rb];
-          build_mask(tb, *slotc, last, hi_a, mw);
-          build_mask(tb, *slotc, last, hi_b, mb);
-        }
+        uint32_t mw[kMaskWords];
+        tok = tb.tok[row];
+        build_mask(tb, *slotc, tb.last, my_hi, mw);
         mbar_arrive(empty_bar(s));
 
         ok = mbar_wait_bounded(s_full, it & 1, limit_ns);
@@ -773,16 +674,12 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         }
         tc_fence_after();
         float x[72];
-        float mrow = 0.f, mrow_b = 0.f;
+        const float mh = row_max(x, mw);
+        tc_fence_before();
+        mbar_arrive(s_empty);   // S of this thread is in registers: the next S may be written
         const int par = it & 1;
+        float mrow;
         if (!is_tail) {
-          uint64_t mlo;
-          uint32_t mhi;
-          half_mask(mw, mlo, mhi);
-          const bool masked = !__all_sync(0xffffffffu, mlo == ~0ull && mhi == 0xffu);
-          const float mh = main_row_max(x, mlo, mhi, masked);
-          tc_fence_before();
-          mbar_arrive(s_empty);   // S of this thread is in registers: the next S may be written
           xmax[(par * 2 + half) * 128 + row] = mh;
           mbar_arrive(xmax_bar(half));
           ok = mbar_wait_bounded(xmax_bar(half ^ 1), par, limit_ns);
@@ -791,30 +688,30 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
             break;
           }
           mrow = fmaxf(mh, xmax[(par * 2 + (half ^ 1)) * 128 + row]);
-          if (mrow == -INFINITY) mrow = 0.f;
         } else {
-          tail_max(x, lane_bits(mw), lane_bits(mb), mrow, mrow_b);
-          tc_fence_before();
-          mbar_arrive(s_empty);
+          mrow = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 16));
         }
+        if (mrow == -INFINITY) mrow = 0.f;
         // P may only be overwritten once the previous tile's PV MMA has consumed it.
         ok = mbar_wait_bounded(p_empty, par ^ 1, limit_ns);
         if (!__all_sync(0xffffffffu, ok)) {
           aborted = true;
           break;
         }
+        const float lh = row_exp(x, mrow);
         if (!is_tail) {
-          inv = main_row_exp(x, mrow);   // the half's row sum; 1 / (full sum) next iteration
-          xsum[(par * 2 + half) * 128 + row] = inv;
+          inv = lh;   // the half's row sum; 1 / (full sum) once the partner's is in
+          xsum[(par * 2 + half) * 128 + row] = lh;
           mbar_arrive(xsum_bar(half));
         } else {
-          tail_exp(x, mrow, mrow_b, inv, inv_b);
+          const float l = lh + __shfl_xor_sync(0xffffffffu, lh, 16);
+          inv = l > 0.f ? 1.f / l : 0.f;
         }
         fence_proxy_async_smem();
         mbar_arrive(p_full);
       }
       if (have_prev) {
-        if (!epilogue(prev_it, prev_head, prev_tok, prev_tok_b, prev_inv, prev_inv_b)) {
+        if (!epilogue(prev_it, prev_head, prev_tok, prev_inv)) {
           aborted = true;
           break;
         }
@@ -824,9 +721,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       prev_it = it;
       prev_head = head;
       prev_tok = tok;
-      prev_tok_b = tok_b;
       prev_inv = inv;
-      prev_inv_b = inv_b;
     }
     if (aborted) {
       if (lane == 0) record_error(err, kStatusTimeout);

@@ -133,6 +133,21 @@ __device__ __forceinline__ void reg_fence8(float* v) {
   asm volatile("" : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]),
                "+f"(v[7]));
 }
+// 16 lanes x 32 bits, twice: threads 0..15 get lanes base + t, columns [c, c + 8); threads
+// 16..31 get lanes base + t - 16, columns [c + 8, c + 16).
+__device__ __forceinline__ void tmem_ld_16x32bx2_x8(uint32_t taddr, float* v) {
+  asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], 8;"
+               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+               : "r"(taddr));
+}
+// The same with 16 columns per half: threads 16..31 get columns [c + 16, c + 32).
+__device__ __forceinline__ void tmem_ld_16x32bx2_x16(uint32_t taddr, float* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], 16;"
+      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]),
+        "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
+      : "r"(taddr));
+}
 // 16 lanes x 256 bits (8 columns): thread t gets lanes base + t/4 and base + 8 + t/4,
 // columns 2*(t%4) and 2*(t%4)+1: v = {(r, c), (r, c+1), (r+8, c), (r+8, c+1)}.
 __device__ __forceinline__ void tmem_ld_16x256b(uint32_t taddr, float* v) {
