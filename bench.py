@@ -59,7 +59,7 @@ def load_peaks():
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples taken while the timed region runs."""
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -74,11 +74,13 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
 
-    def stop(self):
+    def stop(self, window=None):
+        """Median SM clock and the throttle reasons seen; with window = (t0, t1) in epoch
+        seconds only the samples taken inside it count (all of them if none is)."""
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -88,19 +90,29 @@ class ClockSampler:
             self.proc.kill()
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        import datetime
+
+        rows = []
         for line in open(self.path):
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                ts = None
+            try:
+                rows.append((ts, float(f[2]), float(f[3]), f[6:10]))
             except ValueError:
                 continue
-            for nm, val in zip(names, f[5:9]):
+        os.unlink(self.path)
+        inside = [r for r in rows if window and (r[0] is None or window[0] <= r[0] <= window[1])]
+        for _, s_mhz, m_mhz, flags in (inside or rows):
+            sm.append(s_mhz)
+            mx.append(m_mhz)
+            for nm, val in zip(names, flags):
                 if val.lower() == "active":
                     reasons.add(nm)
-        os.unlink(self.path)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
                 "samples": len(sm), "reasons": sorted(reasons)}
 
@@ -122,6 +134,25 @@ def make_device_inputs(torch, dev):
         devt[kname] = t.to(dev)
     return host, devt
 
+
+
+def recorded_traffic():
+    """DRAM bytes per attention launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
+    committed ncu summary, or None if the kernel source changed since that capture."""
+    import hashlib
+    import re
+    summ = os.path.join(ROOT, "profiles", "window_attn_tc_stage1_full.md")
+    src = os.path.join(ROOT, "swin3d_window_attention_b200", "csrc", "attn_tcgen05.cu")
+    if not (os.path.exists(summ) and os.path.exists(src)):
+        return None
+    text = open(summ).read()
+    sha = re.search(r"sha256 `([0-9a-f]{64})`", text)
+    nbytes = re.search(r"dram_bytes_per_launch: (\d+)", text)
+    if not sha or not nbytes:
+        return None
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != sha.group(1):
+        return None
+    return int(nbytes.group(1))
 
 def bench_cuda(args):
     import torch
@@ -174,13 +205,15 @@ def bench_cuda(args):
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
+    wall0 = time.time()
     t0.record(stream)
     for _ in range(args.steps):
         step(record=True)
     t1.record(stream)
     torch.cuda.synchronize()
+    wall1 = time.time()
     ms = t0.elapsed_time(t1)
-    clk = clocks.stop()
+    clk = clocks.stop((wall0, wall1))
     if s3w.poll_device_error() != 0:
         raise SystemExit("device error word set during the timed region")
     if dist:
@@ -262,7 +295,7 @@ def bench_cuda(args):
                  "hbm_frac": attn_gbs / hbm_peak, "tensor_frac": attn_tflops / tc_peak,
                  "legacy_mma_baseline_ms": legacy_ms},
         "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": attn_gbs / hbm_peak, "traffic": None, "peak_source": peak_src,
+                     "frac": attn_gbs / hbm_peak, "traffic": recorded_traffic(), "peak_source": peak_src,
                      "kernel": "window attention", "algorithmic_bytes_per_launch": ATTN_BYTES},
         "e2e": {"value": windows_per_step * world / (e2e_ms * 1e-3), "unit": "windows/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -351,8 +384,8 @@ def bench_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
