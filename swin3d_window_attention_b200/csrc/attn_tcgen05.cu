@@ -78,6 +78,9 @@ struct Table {
   int tok[kN];
   uint32_t real[kMaskWords];
   uint32_t last;
+  // The key mask a softmax thread applies, per (region combination of the query, key half):
+  // bytes 0..8 = key groups 2k + half (k = 0..8), one bit per key; w = 1 if any key is masked.
+  uint4 maskq[16];
 };
 constexpr int kTableBytes = (static_cast<int>(sizeof(Table)) + 15) & ~15;
 // Per CTA, the same for every tile: the (t, h, w) offset of each slot inside the window
@@ -390,6 +393,19 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         const unsigned m = __ballot_sync(0xffffffffu, r < kN && resolve(r) >= 0);
         if (lane == 0) tb.real[wd] = m;
       }
+      __syncwarp();
+      if (lane < 16) {
+        // combination c of the query's wrapped-around sides (bit a: axis a), key half h
+        const uint32_t c = static_cast<uint32_t>(lane) >> 1, h = static_cast<uint32_t>(lane) & 1u;
+        uint32_t mw[kMaskWords];
+        build_mask(tb, *slotc, tb.last, c, mw);
+        uint32_t kb[9];
+#pragma unroll
+        for (int k = 0; k < 9; ++k) kb[k] = (mw[k >> 1] >> (16 * (k & 1) + 8 * h)) & 0xffu;
+        const uint32_t all = kb[0] & kb[1] & kb[2] & kb[3] & kb[4] & kb[5] & kb[6] & kb[7] & kb[8];
+        tb.maskq[lane] = make_uint4(kb[0] | kb[1] << 8 | kb[2] << 16 | kb[3] << 24,
+                                    kb[4] | kb[5] << 8 | kb[6] << 16 | kb[7] << 24, kb[8], all == 0xffu ? 0u : 1u);
+      }
       mbar_arrive(table_bar(s));   // table written (release)
     }
   } else if (warp == kMmaWarp) {
@@ -399,6 +415,14 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     // tile t, and PV(t) runs underneath the softmax of tile t+1.
     constexpr uint32_t idesc_s = idesc_bf16_f32(128, kN, false, false);
     constexpr uint32_t idesc_o = idesc_bf16_f32(128, HD, false, true);
+    // Operand descriptors are linear in the address field (bits 0..13 = address / 16, every
+    // operand below 256 KB), so each MMA's descriptor is a base plus a constant: the stage
+    // moves it by kStageBytes / 16, a K step by 32 B (K-major) or 16 keys = 2048 B (V).
+    const uint64_t dq0 = desc_kmajor_sw128(sb + OFF_STAGE);                    // Q of stage 0
+    const uint64_t dv0 = desc_mnmajor_sw128(sb + OFF_STAGE + 2 * kTileBytes);  // V of stage 0
+    const uint64_t dp0 = desc_kmajor_sw128(sb + OFF_P0B0), dp0b = desc_kmajor_sw32(sb + OFF_P0B2);
+    const uint64_t dp1 = desc_kmajor_sw128(sb + OFF_P1B0), dp1b = desc_kmajor_sw32(sb + OFF_P1B2);
+    constexpr uint64_t kStageStep = kStageBytes >> 4;
     bool issued = false;
     auto issue_s = [&](int jt) -> bool {   // S(jt) = Q K^T of the tile in stage jt % kStages
       const int s = jt % kStages;
@@ -406,38 +430,36 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       if (!mbar_wait_bounded(s_empty, (jt & 1) ^ 1, limit_ns)) return false;
       fence_proxy_async_smem();
       tc_fence_after();
-      const uint32_t qa = sb + OFF_STAGE + s * kStageBytes, ka = qa + kTileBytes;
-#pragma unroll 1
-      for (int kk = 0; kk < HD / 16; ++kk) {
-        const uint64_t kd = desc_kmajor_sw128(ka + kk * 32);
-        umma_bf16_ss(tmem + TM_S0, desc_kmajor_sw128(qa + kk * 32), kd, idesc_s, kk > 0);
-        if (has_tail)
-          umma_bf16_ss(tmem + TM_S1, desc_kmajor_sw128(qa + 128 * kRowBytes + kk * 32), kd, idesc_s, kk > 0);
+      const uint64_t qd = dq0 + s * kStageStep, kd = qd + (kTileBytes >> 4);
+#pragma unroll
+      for (int kk = 0; kk < HD / 16; ++kk) umma_bf16_ss(tmem + TM_S0, qd + 2 * kk, kd + 2 * kk, idesc_s, kk > 0);
+      if (has_tail) {
+        const uint64_t qtd = qd + ((128 * kRowBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) umma_bf16_ss(tmem + TM_S1, qtd + 2 * kk, kd + 2 * kk, idesc_s, kk > 0);
       }
       umma_commit(s_full);
       issued = true;
       return true;
+    };
+    // keys 16kk .. 16kk + 15 of P: blocks of 64 keys (128B swizzle), the last 16 keys in the
+    // 32B-swizzled block
+    auto p_desc = [](uint64_t d128, uint64_t d32, int kk, int block_bytes) {
+      return kk < 8 ? d128 + static_cast<uint64_t>(((kk >> 2) * block_bytes + (kk & 3) * 32) >> 4) : d32;
     };
     auto issue_pv = [&](int jt) -> bool {  // O(jt) = P V of the tile in stage jt % kStages
       const int s = jt % kStages;
       if (!mbar_wait_bounded(p_full, jt & 1, limit_ns)) return false;
       if (!mbar_wait_bounded(o_empty, (jt & 1) ^ 1, limit_ns)) return false;
       tc_fence_after();
-      const uint32_t va = sb + OFF_STAGE + s * kStageBytes + 2 * kTileBytes;
-#pragma unroll 1
-      for (int kk = 0; kk < kN / 16; ++kk) {
-        const uint64_t vd = desc_mnmajor_sw128(va + kk * 2048);
-        // keys 16kk .. 16kk + 15 of P: blocks of 64 keys (128B swizzle), the last 16 keys
-        // in the 32B-swizzled block
-        const uint32_t koff = static_cast<uint32_t>((kk & 3) * 32);
-        const uint64_t pd0 = kk < 8 ? desc_kmajor_sw128(sb + OFF_P0B0 + (kk >> 2) * (OFF_P0B1 - OFF_P0B0) + koff)
-                                    : desc_kmajor_sw32(sb + OFF_P0B2);
-        umma_bf16_ss(tmem + TM_O0, pd0, vd, idesc_o, kk > 0);
-        if (has_tail) {
-          const uint64_t pd1 = kk < 8 ? desc_kmajor_sw128(sb + OFF_P1B0 + (kk >> 2) * (OFF_P1B1 - OFF_P1B0) + koff)
-                                      : desc_kmajor_sw32(sb + OFF_P1B2);
-          umma_bf16_ss(tmem + TM_O1, pd1, vd, idesc_o, kk > 0);
-        }
+      const uint64_t vd = dv0 + s * kStageStep;
+#pragma unroll
+      for (int kk = 0; kk < kN / 16; ++kk)
+        umma_bf16_ss(tmem + TM_O0, p_desc(dp0, dp0b, kk, OFF_P0B1 - OFF_P0B0), vd + 128 * kk, idesc_o, kk > 0);
+      if (has_tail) {
+#pragma unroll
+        for (int kk = 0; kk < kN / 16; ++kk)
+          umma_bf16_ss(tmem + TM_O1, p_desc(dp1, dp1b, kk, OFF_P1B1 - OFF_P1B0), vd + 128 * kk, idesc_o, kk > 0);
       }
       umma_commit(o_full);
       umma_commit(p_empty);
@@ -563,7 +585,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     // registers.  If any thread of the warp has a masked key (near the shift seams and the
     // padding), masked keys become -inf first, hence weight 0.
     auto selb = [](uint32_t w, int e, float x) { return ((w >> e) & 1u) ? x : -INFINITY; };
-    auto row_max = [&](float (&x)[72], const uint32_t (&mw)[kMaskWords]) -> float {
+    auto row_max = [&](float (&x)[72], const uint4 mq) -> float {
       if (!is_tail) {
 #pragma unroll
         for (int k = 0; k < 9; ++k) tmem_ld8(s_base + 16 * k, x + 8 * k);
@@ -574,16 +596,13 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       tmem_wait_ld();
 #pragma unroll
       for (int k = 0; k < 9; ++k) reg_fence8(x + 8 * k);
-      // key group 2k + h = row-mask bits [16k + 8h, +8)
-      uint32_t kb[9];
+      if (__any_sync(0xffffffffu, mq.w != 0u)) {
 #pragma unroll
-      for (int k = 0; k < 9; ++k) kb[k] = (mw[k >> 1] >> (16 * (k & 1) + 8 * half)) & 0xffu;
-      const uint32_t all = kb[0] & kb[1] & kb[2] & kb[3] & kb[4] & kb[5] & kb[6] & kb[7] & kb[8];
-      if (!__all_sync(0xffffffffu, all == 0xffu)) {
+        for (int k = 0; k < 9; ++k) {
+          const uint32_t kb = k < 4 ? mq.x >> (8 * k) : (k < 8 ? mq.y >> (8 * (k - 4)) : mq.z);
 #pragma unroll
-        for (int k = 0; k < 9; ++k)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) x[8 * k + e] = selb(kb[k], e, x[8 * k + e]);
+          for (int e = 0; e < 8; ++e) x[8 * k + e] = selb(kb, e, x[8 * k + e]);
+        }
       }
       float a = -INFINITY, b = -INFINITY;
 #pragma unroll
@@ -662,9 +681,8 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         }
         head = static_cast<int>(tile) - fdiv(static_cast<int>(tile), g.div_heads) * g.heads;
         const Table& tb = tables[s];
-        uint32_t mw[kMaskWords];
         tok = tb.tok[row];
-        build_mask(tb, *slotc, tb.last, my_hi, mw);
+        const uint4 mq = tb.maskq[my_hi * 2 + half];
         mbar_arrive(empty_bar(s));
 
         ok = mbar_wait_bounded(s_full, it & 1, limit_ns);
@@ -674,7 +692,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         }
         tc_fence_after();
         float x[72];
-        const float mh = row_max(x, mw);
+        const float mh = row_max(x, mq);
         tc_fence_before();
         mbar_arrive(s_empty);   // S of this thread is in registers: the next S may be written
         const int par = it & 1;
