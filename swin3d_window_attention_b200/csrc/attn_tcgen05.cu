@@ -70,7 +70,12 @@ constexpr int OFF_P0B0 = 5120;     // P rows 0..127, keys 0..63
 constexpr int OFF_P0B1 = OFF_P0B0 + 16384;
 constexpr int OFF_P0B2 = OFF_P0B1 + 16384;   // keys 128..143, 32B swizzle, 4 KB
 constexpr int OFF_STAGE = OFF_P0B2 + 4096;   // 41984 (1024-aligned)
-constexpr int OFF_TABLE = OFF_STAGE + kStages * kStageBytes;
+// 16 key rows of bf16 ones in the V operand's layout: the PV MMA reads them as 16 more
+// output columns (through the descriptor's leading byte offset), so every such column of O
+// is the row sum of P as rounded to bf16, the exact normaliser of the P the MMA used.
+constexpr int OFF_ONES = OFF_STAGE + kStages * kStageBytes;
+constexpr int kOnesBytes = 16 * kRowBytes;
+constexpr int OFF_TABLE = OFF_ONES + kOnesBytes;
 
 // Per tile: grid token of every slot (-1 = padded), which slots are real, and along which
 // shifted axes the window is the last one (where Swin's mask splits it in two regions).
@@ -94,19 +99,22 @@ struct SlotConst {
 constexpr int OFF_SLOTC = OFF_TABLE + kStages * kTableBytes;
 constexpr int OFF_BARS = OFF_SLOTC + ((static_cast<int>(sizeof(SlotConst)) + 15) & ~15);
 // barriers: load[3] (TMA bytes), empty[3], table[3], s_full, s_empty, p_full, p_empty,
-// o_full, o_empty, drain, row max written[2], row sum written[2] (one per key half)
-constexpr int kNumBars = 3 * kStages + 11;
-// Row max / row sum of each key half of the main rows, exchanged between the two warps
-// that share a row: [tile parity][key half][row].
+// o_full, o_empty, drain, row max written[2] (one per key half)
+constexpr int kNumBars = 3 * kStages + 9;
+// Row max of each key half of the main rows, exchanged between the two warps that share a
+// row: [tile parity][key half][row].
 constexpr int OFF_XCHG = OFF_BARS + kNumBars * 8;
 constexpr int kXchgFloats = 2 * 2 * 128;
-constexpr int OFF_MISC = OFF_XCHG + 2 * kXchgFloats * 4;   // tmem address, abort flag, producer stop
+constexpr int OFF_MISC = OFF_XCHG + kXchgFloats * 4;   // tmem address, abort flag, producer stop
 constexpr int kSmemBytes = OFF_MISC + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1024;       // slack for the 1024-byte alignment
 static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
 
-// TMEM columns (fp32 accumulators, lane = row).  Every MMA destination is 32-aligned.
-constexpr uint32_t TM_S0 = 0, TM_S1 = 160, TM_O0 = 320, TM_O1 = 384;
+// TMEM columns (fp32 accumulators, lane = row).  Every MMA destination is 32-aligned.  O
+// has 80 columns: the head's outputs (the first head_dim of 64), then from column 64 on 16
+// copies of the row sum.
+constexpr uint32_t TM_S0 = 0, TM_S1 = 160, TM_O0 = 320, TM_O1 = 416;
+constexpr uint32_t kOnesCol = 64;
 constexpr uint32_t kTmemCols = 512;
 
 constexpr int kThreads = 384;
@@ -123,10 +131,10 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
 
 // Operand descriptors.  K-major 128B swizzle: 8-row x 128-byte atoms, 1024 bytes apart.
 // K-major 32B swizzle: 8-row x 32-byte atoms, 256 bytes apart.  MN-major 128B swizzle (V,
-// whose rows are keys = the K dimension): 8-key x 64-element atoms, 1024 bytes apart.
+// whose rows are keys = the K dimension): 8-key x 64-element atoms, 1024 bytes apart along
+// K; the leading byte offset is the distance to the next 64 elements along N.
 __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t addr) { return smem_desc(addr, 16, 1024, kSwizzle128B); }
 __device__ __forceinline__ uint64_t desc_kmajor_sw32(uint32_t addr) { return smem_desc(addr, 16, 256, kSwizzle32B); }
-__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t addr) { return smem_desc(addr, 16, 1024, kSwizzle128B); }
 
 // Keys visible to a query in slot r: real slots, restricted on every axis where the window
 // is the last one of a shifted axis to the query's side of the wrap-around split.
@@ -177,9 +185,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
   const uint32_t o_empty = bar0 + 8u * (3 * kStages + 5);
   const uint32_t drain_bar = bar0 + 8u * (3 * kStages + 6);
   auto xmax_bar = [&](int h) { return bar0 + 8u * (3 * kStages + 7 + h); };   // key half h wrote its row maxima
-  auto xsum_bar = [&](int h) { return bar0 + 8u * (3 * kStages + 9 + h); };   // key half h wrote its row sums
   float* xmax = reinterpret_cast<float*>(sm + OFF_XCHG);
-  float* xsum = xmax + kXchgFloats;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sm + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
   volatile int* prod_stop = reinterpret_cast<volatile int*>(sm + OFF_MISC + 8);
@@ -203,10 +209,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     mbar_init(o_full, 1);
     mbar_init(o_empty, n_soft);
     mbar_init(drain_bar, 1);
-    for (int h = 0; h < 2; ++h) {
-      mbar_init(xmax_bar(h), 128);
-      mbar_init(xsum_bar(h), 128);
-    }
+    for (int h = 0; h < 2; ++h) mbar_init(xmax_bar(h), 128);
     *abort_flag = 0;
     *prod_stop = 0;
     fence_barrier_init();
@@ -236,6 +239,9 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       slotc->all[w] = bits;
     }
   }
+  for (int i = tid; i < kOnesBytes / 16; i += kThreads)   // bf16 1.0 = 0x3f80
+    *reinterpret_cast<uint4*>(sm + OFF_ONES + 16 * i) = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);
+  fence_proxy_async_smem();
   // Slots N..143 are never loaded: keep them zero (finite) for the whole kernel.
   if (g.N < kN) {
     for (int i = tid; i < kStages * 3 * (kN - g.N) * (kRowBytes / 16); i += kThreads) {
@@ -414,31 +420,35 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     // out of TMEM, before PV(t); the softmax warps then find S(t+1) ready when they finish
     // tile t, and PV(t) runs underneath the softmax of tile t+1.
     constexpr uint32_t idesc_s = idesc_bf16_f32(128, kN, false, false);
-    constexpr uint32_t idesc_o = idesc_bf16_f32(128, HD, false, true);
+    // N = 64 V columns (the box is 64 channels wide for head_dim 32 too) + 16 ones columns
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, kOnesCol + 16, false, true);
     // Operand descriptors are linear in the address field (bits 0..13 = address / 16, every
     // operand below 256 KB), so each MMA's descriptor is a base plus a constant: the stage
     // moves it by kStageBytes / 16, a K step by 32 B (K-major) or 16 keys = 2048 B (V).
     const uint64_t dq0 = desc_kmajor_sw128(sb + OFF_STAGE);                    // Q of stage 0
-    const uint64_t dv0 = desc_mnmajor_sw128(sb + OFF_STAGE + 2 * kTileBytes);  // V of stage 0
+    // V of stage 0; its second 64-column atom along N (leading byte offset) is the ones block
+    const uint64_t dv0 = smem_desc(sb + OFF_STAGE + 2 * kTileBytes, OFF_ONES - (OFF_STAGE + 2 * kTileBytes), 1024,
+                                   kSwizzle128B);
     const uint64_t dp0 = desc_kmajor_sw128(sb + OFF_P0B0), dp0b = desc_kmajor_sw32(sb + OFF_P0B2);
     const uint64_t dp1 = desc_kmajor_sw128(sb + OFF_P1B0), dp1b = desc_kmajor_sw32(sb + OFF_P1B2);
     constexpr uint64_t kStageStep = kStageBytes >> 4;
+    const uint32_t leader = lane == 0 ? 1u : 0u;
     bool issued = false;
     auto issue_s = [&](int jt) -> bool {   // S(jt) = Q K^T of the tile in stage jt % kStages
       const int s = jt % kStages;
-      if (!mbar_wait_bounded(load_bar(s), (jt / kStages) & 1, limit_ns)) return false;
-      if (!mbar_wait_bounded(s_empty, (jt & 1) ^ 1, limit_ns)) return false;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(load_bar(s), (jt / kStages) & 1, limit_ns))) return false;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(s_empty, (jt & 1) ^ 1, limit_ns))) return false;
       fence_proxy_async_smem();
       tc_fence_after();
       const uint64_t qd = dq0 + s * kStageStep, kd = qd + (kTileBytes >> 4);
 #pragma unroll
-      for (int kk = 0; kk < HD / 16; ++kk) umma_bf16_ss(tmem + TM_S0, qd + 2 * kk, kd + 2 * kk, idesc_s, kk > 0);
+      for (int kk = 0; kk < HD / 16; ++kk) umma_bf16_ss_leader(tmem + TM_S0, qd + 2 * kk, kd + 2 * kk, idesc_s, kk > 0, leader);
       if (has_tail) {
         const uint64_t qtd = qd + ((128 * kRowBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) umma_bf16_ss(tmem + TM_S1, qtd + 2 * kk, kd + 2 * kk, idesc_s, kk > 0);
+        for (int kk = 0; kk < HD / 16; ++kk) umma_bf16_ss_leader(tmem + TM_S1, qtd + 2 * kk, kd + 2 * kk, idesc_s, kk > 0, leader);
       }
-      umma_commit(s_full);
+      umma_commit_leader(s_full, leader);
       issued = true;
       return true;
     };
@@ -449,35 +459,37 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     };
     auto issue_pv = [&](int jt) -> bool {  // O(jt) = P V of the tile in stage jt % kStages
       const int s = jt % kStages;
-      if (!mbar_wait_bounded(p_full, jt & 1, limit_ns)) return false;
-      if (!mbar_wait_bounded(o_empty, (jt & 1) ^ 1, limit_ns)) return false;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(p_full, jt & 1, limit_ns))) return false;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(o_empty, (jt & 1) ^ 1, limit_ns))) return false;
       tc_fence_after();
-      const uint64_t vd = dv0 + s * kStageStep;
+      // Moving V by d (bytes / 16) moves the ones block's leading offset by -d.
+      auto v_desc = [&](int kk) {
+        const uint64_t d = s * kStageStep + 128 * kk;
+        return dv0 + d - (d << 16);
+      };
 #pragma unroll
       for (int kk = 0; kk < kN / 16; ++kk)
-        umma_bf16_ss(tmem + TM_O0, p_desc(dp0, dp0b, kk, OFF_P0B1 - OFF_P0B0), vd + 128 * kk, idesc_o, kk > 0);
+        umma_bf16_ss_leader(tmem + TM_O0, p_desc(dp0, dp0b, kk, OFF_P0B1 - OFF_P0B0), v_desc(kk), idesc_o, kk > 0, leader);
       if (has_tail) {
 #pragma unroll
         for (int kk = 0; kk < kN / 16; ++kk)
-          umma_bf16_ss(tmem + TM_O1, p_desc(dp1, dp1b, kk, OFF_P1B1 - OFF_P1B0), vd + 128 * kk, idesc_o, kk > 0);
+          umma_bf16_ss_leader(tmem + TM_O1, p_desc(dp1, dp1b, kk, OFF_P1B1 - OFF_P1B0), v_desc(kk), idesc_o, kk > 0, leader);
       }
-      umma_commit(o_full);
-      umma_commit(p_empty);
-      umma_commit(empty_bar(s));
+      umma_commit_leader(o_full, leader);
+      umma_commit_leader(p_empty, leader);
+      umma_commit_leader(empty_bar(s), leader);
       return true;
     };
     // Step j issues S(j) (if tile j exists) and then PV(j-1): S(0); S(1), PV(0); S(2), PV(1); ...
-    // Lane 0 issues; every lane follows the same control flow (decisions are broadcast).
-    int ok = 1;
+    // The whole warp runs this (every wait's outcome is agreed by a vote); lane 0 alone
+    // issues the MMAs and commits.
+    bool ok = true;
     const long long my_tiles =
         static_cast<long long>(blockIdx.x) < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     for (long long j = 0; ok && j <= my_tiles; ++j) {
-      if (lane == 0) {
-        ok = !*abort_flag;
-        if (ok && j < my_tiles) ok = issue_s(static_cast<int>(j));
-        if (ok && j > 0) ok = issue_pv(static_cast<int>(j - 1));
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ok = !__any_sync(0xffffffffu, *abort_flag != 0);
+      if (ok && j < my_tiles) ok = issue_s(static_cast<int>(j));
+      if (ok && j > 0) ok = issue_pv(static_cast<int>(j - 1));
     }
     if (!ok && lane == 0) {
       record_error(err, kStatusTimeout);
@@ -523,7 +535,6 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     // state of the previous tile, finished one iteration later
     bool have_prev = false;
     int prev_it = 0, prev_head = 0, prev_tok = -1;
-    float prev_inv = 0.f;
     bool aborted = false;
 
     auto store8 = [&](int tk, int head, int col, const float* vals, float scl) {
@@ -551,31 +562,47 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       }
     };
 
-    // Epilogue of a finished tile: this thread's O columns from TMEM, scaled by 1/rowsum,
-    // stored to the grid position of the query slot (padded slots dropped).
-    auto epilogue = [&](int pit, int head, int tok, float inv) -> bool {
+    // Epilogue of a finished tile: this thread's O columns and the row sum (column 64 of O)
+    // from TMEM, scaled by 1/rowsum, stored to the grid position of the query slot
+    // (padded slots dropped).
+    auto epilogue = [&](int pit, int head, int tok) -> bool {
       bool ok = mbar_wait_bounded(o_full, pit & 1, limit_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) return false;
       tc_fence_after();
       float ov[HD / 2];
+      float l;
       if (!is_tail) {
 #pragma unroll
         for (int m = 0; m < HD / 32; ++m) tmem_ld16(o_base + 32 * m, ov + 16 * m);
+        tmem_ld1(o_base - 16 * half + kOnesCol, &l);
       } else {
 #pragma unroll
         for (int m = 0; m < HD / 32; ++m) tmem_ld_16x32bx2_x16(o_base + 32 * m, ov + 16 * m);
+        tmem_ld_16x32bx2_x1(o_base + kOnesCol, &l);
       }
       tmem_wait_ld();
 #pragma unroll
       for (int m = 0; m < HD / 32; ++m) reg_fence16(ov + 16 * m);
+      reg_fence1(&l);
       tc_fence_before();
       mbar_arrive(o_empty);
+      const float inv = l > 0.f ? 1.f / l : 0.f;
       if (tok >= 0) {
 #pragma unroll
         for (int m = 0; m < HD / 32; ++m) {
-          store8(tok, head, 32 * m + 16 * half, ov + 16 * m, inv);
-          store8(tok, head, 32 * m + 16 * half + 8, ov + 16 * m + 8, inv);
+          const int col = 32 * m + 16 * half;
+          if constexpr (!OUT_F32) {
+            if (g.o_rows_32b) {   // 16 bf16 = one 32-byte store
+              uint32_t u[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) u[e] = pack_bf16x2(ov[16 * m + 2 * e] * inv, ov[16 * m + 2 * e + 1] * inv);
+              st_global_v8(static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tok) * g.o_stride + head * HD + col, u);
+              continue;
+            }
+          }
+          store8(tok, head, col, ov + 16 * m, inv);
+          store8(tok, head, col + 8, ov + 16 * m + 8, inv);
         }
       }
       return true;
@@ -612,10 +639,9 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       }
       return fmaxf(a, b);
     };
-    // exp2, the half's row sum, and P (bf16) into the P blocks.
-    auto row_exp = [&](const float (&x)[72], float m) -> float {
+    // exp2 and P (bf16) into the P blocks.  The row sum comes out of the PV MMA.
+    auto row_exp = [&](const float (&x)[72], float m) {
       const float2 cc = make_float2(c, c), nm = make_float2(-m * c, -m * c);
-      float2 l0 = make_float2(0.f, 0.f), l1 = make_float2(0.f, 0.f);
       const uint32_t rsw = lrow & 7;
       const uint32_t row128 = static_cast<uint32_t>(lrow) * 128, row32 = static_cast<uint32_t>(lrow) * 32;
       const uint32_t sw32 = (lrow >> 2) & 1;
@@ -629,8 +655,6 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
           const float2 yb = fma2(make_float2(x[q + 2], x[q + 3]), cc, nm);
           const float2 pa = make_float2(ex2(ya.x), ex2(ya.y));
           const float2 pb = make_float2(ex2(yb.x), ex2(yb.y));
-          l0 = add2(l0, pa);
-          l1 = add2(l1, pb);
           pk[e / 2] = pack_bf16x2_int(pa.x, pa.y);
           pk[e / 2 + 1] = pack_bf16x2_int(pb.x, pb.y);
         }
@@ -644,8 +668,6 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
                      "r"(pk[3])
                      : "memory");
       }
-      const float2 l2 = add2(l0, l1);
-      return l2.x + l2.y;
     };
 
     // Iteration `it` does the softmax of tile `it` (if any) and then the epilogue of tile
@@ -654,19 +676,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     // the exponentials, and the MMA warp can compute the next tile's S underneath them.
     for (long long tile = blockIdx.x;; tile += gridDim.x, ++it) {
       const bool have_cur = tile < num_tiles;
-      if (have_prev && !is_tail) {
-        // The partner warp's row sum of the previous tile.  Taken here, before this warp's
-        // next arrival on an exchange barrier, so the partner can never be two phases ahead.
-        const bool ok = mbar_wait_bounded(xsum_bar(half ^ 1), prev_it & 1, limit_ns);
-        if (!__all_sync(0xffffffffu, ok)) {
-          aborted = true;
-          break;
-        }
-        const float l = prev_inv + xsum[((prev_it & 1) * 2 + (half ^ 1)) * 128 + row];
-        prev_inv = l > 0.f ? 1.f / l : 0.f;
-      }
       int head = 0, tok = -1;
-      float inv = 0.f;
       if (have_cur) {
         const int s = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
@@ -716,20 +726,12 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
           aborted = true;
           break;
         }
-        const float lh = row_exp(x, mrow);
-        if (!is_tail) {
-          inv = lh;   // the half's row sum; 1 / (full sum) once the partner's is in
-          xsum[(par * 2 + half) * 128 + row] = lh;
-          mbar_arrive(xsum_bar(half));
-        } else {
-          const float l = lh + __shfl_xor_sync(0xffffffffu, lh, 16);
-          inv = l > 0.f ? 1.f / l : 0.f;
-        }
+        row_exp(x, mrow);
         fence_proxy_async_smem();
         mbar_arrive(p_full);
       }
       if (have_prev) {
-        if (!epilogue(prev_it, prev_head, prev_tok, prev_inv)) {
+        if (!epilogue(prev_it, prev_head, prev_tok)) {
           aborted = true;
           break;
         }
@@ -739,7 +741,6 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       prev_it = it;
       prev_head = head;
       prev_tok = tok;
-      prev_inv = inv;
     }
     if (aborted) {
       if (lane == 0) record_error(err, kStatusTimeout);

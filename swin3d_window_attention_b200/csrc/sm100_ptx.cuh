@@ -133,6 +133,16 @@ __device__ __forceinline__ void reg_fence8(float* v) {
   asm volatile("" : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]),
                "+f"(v[7]));
 }
+// 32 lanes x 32 bits, one column: thread t gets lane base + t.
+__device__ __forceinline__ void tmem_ld1(uint32_t taddr, float* v) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=f"(v[0]) : "r"(taddr));
+}
+__device__ __forceinline__ void reg_fence1(float* v) { asm volatile("" : "+f"(v[0])); }
+// 16 lanes x 32 bits, twice, one column each: threads 0..15 get lanes base + t, column c;
+// threads 16..31 get lanes base + t - 16, column c + 1.
+__device__ __forceinline__ void tmem_ld_16x32bx2_x1(uint32_t taddr, float* v) {
+  asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x1.b32 {%0}, [%1], 1;" : "=f"(v[0]) : "r"(taddr));
+}
 // 16 lanes x 32 bits, twice: threads 0..15 get lanes base + t, columns [c, c + 8); threads
 // 16..31 get lanes base + t - 16, columns [c + 8, c + 16).
 __device__ __forceinline__ void tmem_ld_16x32bx2_x8(uint32_t taddr, float* v) {
@@ -174,6 +184,24 @@ __device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, u
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The same, executed by a whole warp with only the `leader` lane issuing: the warp stays
+// converged, so the descriptor arithmetic around it can stay warp-uniform.
+__device__ __forceinline__ void umma_bf16_ss_leader(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                    uint32_t idesc, uint32_t accumulate, uint32_t leader) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 q, %5, 0;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(leader)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_leader(uint32_t bar, uint32_t leader) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %1, 0;\n\t"
+      "@q tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar),
+      "r"(leader)
       : "memory");
 }
 
