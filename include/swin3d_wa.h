@@ -152,6 +152,16 @@ int s3w_poll_device_error(s3w_stream_t stream);
  */
 long long s3w_set_wait_limit_ns(long long ns);
 
+/*
+ * Failure injection for tests (process-wide; returns the previous setting).  With a
+ * nonzero value, every swin3d_window_attn_fwd launched after the call first waits on a
+ * barrier that nothing signals, so that wait expires after the limit set above and the
+ * kernel takes the timeout path (S3W_ERR_DEVICE_TIMEOUT in the error word, early exit,
+ * context usable).  0 restores normal operation.  Nothing faults, traps or hangs: the
+ * wait is bounded like every other one.
+ */
+int s3w_set_test_stall(int on);
+
 /* Library version as major*10000 + minor*100 + patch. */
 int s3w_version(void);
 

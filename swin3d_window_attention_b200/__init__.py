@@ -10,6 +10,7 @@ from .api import (  # noqa: F401
     library_path,
     load_library,
     poll_device_error,
+    set_test_stall,
     set_wait_limit_ns,
     status_string,
     swin3d_window_attn_fwd,

@@ -45,6 +45,8 @@ def load_library():
     lib.swin3d_window_attn_fwd_legacy_mma.restype = I
     lib.s3w_set_wait_limit_ns.argtypes = [LL]
     lib.s3w_set_wait_limit_ns.restype = LL
+    lib.s3w_set_test_stall.argtypes = [ctypes.c_int]
+    lib.s3w_set_test_stall.restype = ctypes.c_int
     lib.adaln_residual_fwd.argtypes = [P, I, P, P, P, P, I, I, LL, I, F, P]
     lib.adaln_residual_fwd.restype = I
     lib.s3w_status_string.argtypes = [I]
@@ -152,3 +154,10 @@ def poll_device_error(stream=None) -> int:
 def set_wait_limit_ns(ns: int) -> int:
     """Set the kernels' bounded-wait limit (ns); returns the previous one."""
     return int(load_library().s3w_set_wait_limit_ns(int(ns)))
+
+
+def set_test_stall(on: bool) -> bool:
+    """Failure injection for tests: later attention launches first wait on a barrier that
+    nothing signals, so they take the bounded-wait timeout path.  Returns the previous
+    setting."""
+    return bool(load_library().s3w_set_test_stall(1 if on else 0))

@@ -47,6 +47,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // Time limit of every bounded wait inside the kernels (nanoseconds); 1 s by default.
 long long g_wait_limit_ns = 1000000000ll;
+int g_test_stall = 0;
 
 }  // namespace
 
@@ -118,6 +119,7 @@ int make_geometry(const void* q, const void* k, const void* v, void* o, int B, i
   if (per_sample * B * heads > INT32_MAX) return S3W_ERR_UNSUPPORTED;  // tile index is 32-bit
 
   s3w::WinGeom& g = *out;
+  g = s3w::WinGeom{};
   g.B = B; g.T = T; g.H = H; g.W = W;
   g.wt = win_t; g.wh = win_h; g.ww = win_w;
   g.st = shift_t; g.sh = shift_h; g.sw = shift_w;
@@ -149,6 +151,12 @@ long long s3w_set_wait_limit_ns(long long ns) {
   return prev;
 }
 
+int s3w_set_test_stall(int on) {
+  const int prev = g_test_stall;
+  g_test_stall = on ? 1 : 0;
+  return prev;
+}
+
 int swin3d_window_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int T, int H, int W,
                            int win_t, int win_h, int win_w, int shift_t, int shift_h, int shift_w, int heads,
                            int head_dim, long long qkv_token_stride, long long o_token_stride, float scale,
@@ -160,6 +168,7 @@ int swin3d_window_attn_fwd(const void* q, const void* k, const void* v, void* o,
   DeviceState* ds = nullptr;
   rc = device_state(&ds);
   if (rc != S3W_OK) return rc;
+  g.test_stall = g_test_stall;
   cudaError_t e = s3w::launch_window_attn_tc(g, q, k, v, o, out_dtype == S3W_F32, ds->err, g_wait_limit_ns,
                                              ds->num_sms, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? S3W_OK : S3W_ERR_CUDA;

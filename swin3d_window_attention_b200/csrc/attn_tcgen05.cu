@@ -483,7 +483,9 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     // Step j issues S(j) (if tile j exists) and then PV(j-1): S(0); S(1), PV(0); S(2), PV(1); ...
     // The whole warp runs this (every wait's outcome is agreed by a vote); lane 0 alone
     // issues the MMAs and commits.
-    bool ok = true;
+    // Failure injection (tests): wait on the drain barrier, which nothing signals before the
+    // loop below has run, so the bounded wait expires and the CTA takes the timeout path.
+    bool ok = !g.test_stall || __all_sync(0xffffffffu, mbar_wait_bounded(drain_bar, 0, limit_ns));
     const long long my_tiles =
         static_cast<long long>(blockIdx.x) < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     for (long long j = 0; ok && j <= my_tiles; ++j) {

@@ -55,6 +55,7 @@ struct WinGeom {
   float scale_log2;        // scale * log2(e)
   int o_rows_32b;          // 1 if every output row start is 32-byte aligned
   FastDiv div_heads, div_per_sample, div_nww, div_nwh;   // tile -> (sample, window, head)
+  int test_stall;          // failure injection: first wait on a barrier nothing signals
 };
 
 // Per-axis region label on the shifted, padded grid.

@@ -166,19 +166,22 @@ def test_full_size_sampled_windows(cuda_ok, case):
 
 
 def test_bounded_wait_timeout_is_reported_and_context_survives(cuda_ok):
-    """A zero wait limit makes the kernel's first unsatisfied wait expire: the call must
-    unwind, report S3W_ERR_DEVICE_TIMEOUT through the error word, and leave the context
-    usable for a normal call right after."""
+    """With the stall injection on, the kernel's first wait is on a barrier nothing signals
+    and expires after the (short) limit: the call must unwind, report
+    S3W_ERR_DEVICE_TIMEOUT through the error word, and leave the context usable for a
+    normal call right after."""
     B, T, H, W, heads, hd, window, shift = 1, 4, 36, 72, 8, 64, (2, 6, 12), (1, 3, 6)
     C = heads * hd
     bits, dev = make_qkv(B, T, H, W, C, base=60)
     o = torch.zeros((B, T, H, W, C), dtype=torch.bfloat16, device="cuda")
     assert s3w.poll_device_error() == 0
-    prev = s3w.set_wait_limit_ns(0)
+    prev = s3w.set_wait_limit_ns(1_000_000)
+    prev_stall = s3w.set_test_stall(True)
     try:
         s3w.swin3d_window_attn_fwd(*dev, o, heads, hd, window, shift)
         status = s3w.poll_device_error()
     finally:
+        s3w.set_test_stall(prev_stall)
         s3w.set_wait_limit_ns(prev)
     assert status == 5
     assert s3w.poll_device_error() == 0          # the word was cleared by the poll
