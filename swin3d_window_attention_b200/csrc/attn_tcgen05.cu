@@ -99,8 +99,8 @@ struct SlotConst {
 constexpr int OFF_SLOTC = OFF_TABLE + kStages * kTableBytes;
 constexpr int OFF_BARS = OFF_SLOTC + ((static_cast<int>(sizeof(SlotConst)) + 15) & ~15);
 // barriers: load[3] (TMA bytes), empty[3], table[3], s_full, s_empty, p_full, p_empty,
-// o_full, o_empty, drain, row max written[2] (one per key half)
-constexpr int kNumBars = 3 * kStages + 9;
+// o_full, o_empty, drain, row max written[2] (one per key half), tail p_full, tail p_empty
+constexpr int kNumBars = 3 * kStages + 11;
 // Row max of each key half of the main rows, exchanged between the two warps that share a
 // row: [tile parity][key half][row].
 constexpr int OFF_XCHG = OFF_BARS + kNumBars * 8;
@@ -185,6 +185,10 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
   const uint32_t o_empty = bar0 + 8u * (3 * kStages + 5);
   const uint32_t drain_bar = bar0 + 8u * (3 * kStages + 6);
   auto xmax_bar = [&](int h) { return bar0 + 8u * (3 * kStages + 7 + h); };   // key half h wrote its row maxima
+  // P of the main rows and of the tail rows are handed over separately, so the main rows'
+  // next P may be written as soon as their own PV MMAs have read it.
+  const uint32_t p_full_t = bar0 + 8u * (3 * kStages + 9);
+  const uint32_t p_empty_t = bar0 + 8u * (3 * kStages + 10);
   float* xmax = reinterpret_cast<float*>(sm + OFF_XCHG);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sm + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
@@ -204,8 +208,10 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     }
     mbar_init(s_full, 1);
     mbar_init(s_empty, n_soft);
-    mbar_init(p_full, n_soft);
+    mbar_init(p_full, 256);
     mbar_init(p_empty, 1);
+    mbar_init(p_full_t, 32);
+    mbar_init(p_empty_t, 1);
     mbar_init(o_full, 1);
     mbar_init(o_empty, n_soft);
     mbar_init(drain_bar, 1);
@@ -470,13 +476,16 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
 #pragma unroll
       for (int kk = 0; kk < kN / 16; ++kk)
         umma_bf16_ss_leader(tmem + TM_O0, p_desc(dp0, dp0b, kk, OFF_P0B1 - OFF_P0B0), v_desc(kk), idesc_o, kk > 0, leader);
+      umma_commit_leader(p_empty, leader);
       if (has_tail) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(p_full_t, jt & 1, limit_ns))) return false;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kN / 16; ++kk)
           umma_bf16_ss_leader(tmem + TM_O1, p_desc(dp1, dp1b, kk, OFF_P1B1 - OFF_P1B0), v_desc(kk), idesc_o, kk > 0, leader);
       }
+      if (has_tail) umma_commit_leader(p_empty_t, leader);
       umma_commit_leader(o_full, leader);
-      umma_commit_leader(p_empty, leader);
       umma_commit_leader(empty_bar(s), leader);
       return true;
     };
@@ -556,10 +565,10 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         __nv_bfloat16* dst =
             static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD + col;
         uint4 u;
-        u.x = pack_bf16x2(vals[0] * scl, vals[1] * scl);
-        u.y = pack_bf16x2(vals[2] * scl, vals[3] * scl);
-        u.z = pack_bf16x2(vals[4] * scl, vals[5] * scl);
-        u.w = pack_bf16x2(vals[6] * scl, vals[7] * scl);
+        u.x = pack_bf16x2_int(vals[0] * scl, vals[1] * scl);
+        u.y = pack_bf16x2_int(vals[2] * scl, vals[3] * scl);
+        u.z = pack_bf16x2_int(vals[4] * scl, vals[5] * scl);
+        u.w = pack_bf16x2_int(vals[6] * scl, vals[7] * scl);
         *reinterpret_cast<uint4*>(dst) = u;
       }
     };
@@ -589,7 +598,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       reg_fence1(&l);
       tc_fence_before();
       mbar_arrive(o_empty);
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float inv = l > 0.f ? rcp_approx(l) : 0.f;
       if (tok >= 0) {
 #pragma unroll
         for (int m = 0; m < HD / 32; ++m) {
@@ -598,7 +607,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
             if (g.o_rows_32b) {   // 16 bf16 = one 32-byte store
               uint32_t u[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) u[e] = pack_bf16x2(ov[16 * m + 2 * e] * inv, ov[16 * m + 2 * e + 1] * inv);
+              for (int e = 0; e < 8; ++e) u[e] = pack_bf16x2_int(ov[16 * m + 2 * e] * inv, ov[16 * m + 2 * e + 1] * inv);
               st_global_v8(static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tok) * g.o_stride + head * HD + col, u);
               continue;
             }
@@ -723,14 +732,14 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         }
         if (mrow == -INFINITY) mrow = 0.f;
         // P may only be overwritten once the previous tile's PV MMA has consumed it.
-        ok = mbar_wait_bounded(p_empty, par ^ 1, limit_ns);
+        ok = mbar_wait_bounded(is_tail ? p_empty_t : p_empty, par ^ 1, limit_ns);
         if (!__all_sync(0xffffffffu, ok)) {
           aborted = true;
           break;
         }
         row_exp(x, mrow);
         fence_proxy_async_smem();
-        mbar_arrive(p_full);
+        mbar_arrive(is_tail ? p_full_t : p_full);
       }
       if (have_prev) {
         if (!epilogue(prev_it, prev_head, prev_tok)) {
