@@ -36,7 +36,7 @@ inline FastDiv make_fastdiv(uint32_t d) {
   f.shift = 31 + l;
   return f;
 }
-__device__ __forceinline__ int fdiv(int n, const FastDiv& f) {
+__host__ __device__ __forceinline__ int fdiv(int n, const FastDiv& f) {
   return static_cast<int>((static_cast<unsigned long long>(static_cast<uint32_t>(n)) * f.m) >> f.shift);
 }
 
