@@ -1,6 +1,6 @@
 // Thin inline-PTX wrappers for the sm_100a features the window-attention kernel uses:
-// mbarriers with time-bounded waits, cp.async gathers, the tcgen05 tensor-core MMA with
-// TMEM accumulators, TMEM allocation and TMEM -> register loads.
+// mbarriers with time-bounded waits, TMA tensor loads, the tcgen05 tensor-core MMA with
+// TMEM accumulators, TMEM allocation and TMEM -> register loads, packed fp32x2 arithmetic.
 #pragma once
 #include <cstdint>
 
@@ -87,19 +87,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-__device__ __forceinline__ void cp_async_16_zfill(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
-               : "memory");
-}
-// Arrive on `bar` once every cp.async issued so far by this thread has landed (the
-// pending count is raised first, so together with a plain arrive the net count is one).
-__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
 // ---- TMEM ------------------------------------------------------------------------
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
@@ -158,16 +145,6 @@ __device__ __forceinline__ void tmem_ld_16x32bx2_x16(uint32_t taddr, float* v) {
         "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
       : "r"(taddr));
 }
-// 16 lanes x 256 bits (8 columns): thread t gets lanes base + t/4 and base + 8 + t/4,
-// columns 2*(t%4) and 2*(t%4)+1: v = {(r, c), (r, c+1), (r+8, c), (r+8, c+1)}.
-__device__ __forceinline__ void tmem_ld_16x256b(uint32_t taddr, float* v) {
-  asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];"
-               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3])
-               : "r"(taddr));
-}
-__device__ __forceinline__ void reg_fence4(float* v) {
-  asm volatile("" : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]));
-}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 // Emits nothing; ties 16 registers to a point after the preceding volatile asm (the
 // tcgen05.wait::ld), so no use of them can be scheduled before the load has landed.
@@ -175,16 +152,6 @@ __device__ __forceinline__ void reg_fence16(float* v) {
   asm volatile("" : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]),
                "+f"(v[7]), "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]),
                "+f"(v[14]), "+f"(v[15]));
-}
-
-// ---- tcgen05.mma (kind::f16, bf16 x bf16 -> fp32 in TMEM, A and B from shared memory) --
-__device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
 }
 
 // The same, executed by a whole warp with only the `leader` lane issuing: the warp stays
@@ -247,15 +214,6 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
   asm("mov.b64 {%0,%1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
   return r;
 }
-__device__ __forceinline__ float2 add2(float2 a, float2 b) {
-  uint64_t d;
-  asm("{\n\t.reg .b64 a, b;\n\tmov.b64 a, {%1,%2};\n\tmov.b64 b, {%3,%4};\n\tadd.rn.f32x2 %0, a, b;\n\t}"
-      : "=l"(d) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  float2 r;
-  asm("mov.b64 {%0,%1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
-  return r;
-}
-
 // max of three fp32 values in one instruction.
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
