@@ -119,3 +119,51 @@ def torch_bf16_to_bits(t) -> np.ndarray:
     import torch
 
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def _to_i64(u: int) -> int:
+    """A uint64 constant as the int64 with the same bit pattern."""
+    return u - (1 << 64) if u >= (1 << 63) else u
+
+
+def normal_f32_torch(n: int, device, seed: int = SEED, tensor_index: int = 0, sigma: float = 1.0,
+                     chunk_pairs: int = 1 << 25):
+    """The same stream as :func:`normal_f32`, evaluated with torch int64 / float64 ops on
+    ``device`` (for inputs too large to draw on the host in a test).  int64 arithmetic
+    wraps like uint64; right shifts are made logical by masking.  The float64 log, sqrt,
+    cos and sin may differ from numpy's in the last bit, so a float32 sample can differ by
+    one unit in rare cases: tests that use this hand the same device tensor to both sides."""
+    import torch
+
+    def lsr(z, k):
+        return (z >> k) & ((1 << (64 - k)) - 1)
+
+    def mix(x):
+        z = x + _to_i64(int(_GOLDEN))
+        z = (z ^ lsr(z, 30)) * _to_i64(int(_M1))
+        z = (z ^ lsr(z, 27)) * _to_i64(int(_M2))
+        return z ^ lsr(z, 31)
+
+    key = _to_i64(int(stream_key(seed, tensor_index)))
+    out = torch.empty(n, dtype=torch.float32, device=device)
+    npairs = (n + 1) // 2
+    for p0 in range(0, npairs, chunk_pairs):
+        p1 = min(npairs, p0 + chunk_pairs)
+        idx = torch.arange(p0, p1, dtype=torch.int64, device=device)
+        z = mix(key ^ (idx * _to_i64(int(_PAIR))))
+        u1 = (lsr(z, 40).to(torch.float64) + 0.5) * (1.0 / (1 << 24))
+        u2 = ((lsr(z, 16) & 0xFFFFFF).to(torch.float64) + 0.5) * (1.0 / (1 << 24))
+        r = torch.sqrt(-2.0 * torch.log(u1)) * sigma
+        ang = 2.0 * np.pi * u2
+        pair = torch.stack([(r * torch.cos(ang)).to(torch.float32), (r * torch.sin(ang)).to(torch.float32)], 1)
+        lo, hi = 2 * p0, min(n, 2 * p1)
+        out[lo:hi] = pair.reshape(-1)[: hi - lo]
+    return out
+
+
+def normal_bf16_torch(shape, device, seed: int = SEED, tensor_index: int = 0, sigma: float = 1.0):
+    """bf16 tensor of the stream on ``device`` (float32 rounded to nearest, ties to even)."""
+    import torch
+
+    n = int(np.prod(shape))
+    return normal_f32_torch(n, device, seed, tensor_index, sigma).to(torch.bfloat16).reshape(shape)
