@@ -136,21 +136,30 @@ def make_device_inputs(torch, dev):
 
 
 
+def kernel_code_sha256(text):
+    """sha256 of a source file's code: comments and blank lines removed, so that editing a
+    comment does not separate a capture from the kernel it measured."""
+    import hashlib
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines()]
+    return hashlib.sha256("\n".join(ln for ln in lines if ln.strip()).encode()).hexdigest()
+
+
 def recorded_traffic():
     """DRAM bytes per attention launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
-    committed ncu summary, or None if the kernel source changed since that capture."""
-    import hashlib
+    committed ncu summary, or None if the kernel's code changed since that capture."""
     import re
     summ = os.path.join(ROOT, "profiles", "window_attn_tc_stage1_full.md")
     src = os.path.join(ROOT, "swin3d_window_attention_b200", "csrc", "attn_tcgen05.cu")
     if not (os.path.exists(summ) and os.path.exists(src)):
         return None
     text = open(summ).read()
-    sha = re.search(r"sha256 `([0-9a-f]{64})`", text)
+    sha = re.search(r"code sha256 `([0-9a-f]{64})`", text)
     nbytes = re.search(r"dram_bytes_per_launch: (\d+)", text)
     if not sha or not nbytes:
         return None
-    if hashlib.sha256(open(src, "rb").read()).hexdigest() != sha.group(1):
+    if kernel_code_sha256(open(src).read()) != sha.group(1):
         return None
     return int(nbytes.group(1))
 

@@ -13,29 +13,33 @@
 //
 // Work unit ("tile"): one (sample, window, head).  Roles (warp -> SM sub-partition w % 4):
 //   softmax warps 0-7  warp w owns TMEM lanes 32 (w % 4) .. +31 = query rows of
-//                      S0 = Q[0:128] K^T, and of each row the keys of half w / 4 (72 keys).
-//                      It reads its 72 logits out of TMEM once (releasing S for the next
-//                      tile), takes the masked max, swaps it with the warp holding the other
-//                      half, then exp2, the partial row sum and P rounded to bf16 into shared
-//                      memory.  One tile later (the PV MMA overlaps the next softmax) it adds
-//                      the partner's row sum, loads half of the row's O columns, scales by
-//                      1/rowsum and stores them to the query's original grid position;
-//                      padded slots are dropped.
+//                      S0 = Q[0:128] K^T, and of each row the keys of half w / 4 (key
+//                      groups 2k + h of 8 keys, 72 keys).  It reads its 72 logits out of
+//                      TMEM once (releasing S for the next tile), takes the masked max, swaps
+//                      it with the warp holding the other half, then exp2 and P rounded to
+//                      bf16 into shared memory.  One tile later (the PV MMA overlaps the next
+//                      softmax) it loads half of the row's O columns and the row sum (an MMA
+//                      output column, see below), scales by 1/rowsum and stores them to the
+//                      query's original grid position; padded slots are dropped.
 //   tail warp 8        the same for the 16 tail rows (S1 = Q[128:144] K^T in TMEM lanes
-//                      0..15, reachable from warp 8 like from warp 0), read with the 16x256b
-//                      shape so all 32 lanes share them.
-//   MMA warp 9         one thread issues S(t+1) as soon as tile t+1 is loaded and S(t) has
-//                      left TMEM, then PV(t) = P V once P(t) is in shared memory (V read as
-//                      an MN-major operand); completion is signalled by tcgen05.commit.
+//                      0..15, reachable from warp 8 like from warp 0), read with the 16x32bx2
+//                      shape: threads 0..15 hold half 0 of rows 128..143, threads 16..31
+//                      half 1; the two halves swap row maxima by a shuffle.
+//   MMA warp 9         the warp runs the issue loop, lane 0 issues: S(t+1) as soon as tile
+//                      t+1 is loaded and S(t) has left TMEM, then PV(t) = P V once P(t) is in
+//                      shared memory (main rows and tail rows handed over separately), with V
+//                      read as an MN-major operand followed by 16 columns of ones, so O's
+//                      columns from 64 on are the row sums of the bf16 P; completion is
+//                      signalled by tcgen05.commit.
 //   TMA warp 10        one thread loads the tile's Q, K and V with TMA: one box per T-slab
 //                      of the window (win_h x win_w tokens) per tensor, cut where the window
 //                      wraps around a seam of the shifted grid, straight from grid layout into
 //                      a 3-stage ring in the tensor core's 128-byte swizzled K-major layout;
 //                      padded coordinates are out of bounds and read as zero.  It runs ahead
 //                      as far as the ring allows.
-//   table warp 11      writes the slot -> grid-token table, a bitmask of the real slots and
-//                      the window's "last along a shifted axis" flags (the mask of a query
-//                      follows from these) for the stage being loaded.
+//   table warp 11      writes the slot -> grid-token table, a bitmask of the real slots, the
+//                      window's "last along a shifted axis" flags and, from these, the key
+//                      masks per region combination and key half, for the stage being loaded.
 // Synchronisation is by mbarriers only; every wait is bounded by a time limit and a
 // timeout unwinds the whole CTA (error word set, copies drained, TMEM freed).
 #include <cuda.h>
@@ -123,7 +127,7 @@ constexpr int kTailWarp = 8;           // tail rows 128..143 (TMEM lane quarter 
 constexpr int kMmaWarp = 9;
 constexpr int kTmaWarp = 10;
 constexpr int kFirstProducerWarp = 11;
-constexpr int kProducerThreads = 32;   // table writer (warp 7)
+constexpr int kProducerThreads = 32;   // table writer (warp 11)
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");

@@ -1,7 +1,6 @@
 """Host-side pieces of bench.py that need no GPU: the clock sampler's parsing and window
 filter, and the lookup of the DRAM traffic recorded by an ncu capture."""
 import datetime
-import hashlib
 import os
 import time
 
@@ -39,11 +38,13 @@ def test_recorded_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
     src_dir.mkdir(parents=True)
     (tmp_path / "profiles").mkdir()
     src = src_dir / "attn_tcgen05.cu"
-    src.write_text("// kernel v1\n")
-    sha = hashlib.sha256(src.read_bytes()).hexdigest()
+    src.write_text("int a = 1;  // kernel v1\n")
+    sha = bench.kernel_code_sha256(src.read_text())
     (tmp_path / "profiles" / "window_attn_tc_stage1_full.md").write_text(
-        f"- kernel source: `x`, sha256 `{sha}`\n- dram_bytes_per_launch: 1234567  (algorithmic: 1)\n")
+        f"- kernel source: `x`, code sha256 `{sha}`\n- dram_bytes_per_launch: 1234567  (algorithmic: 1)\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.recorded_traffic() == 1234567
-    src.write_text("// kernel v2\n")           # the kernel changed since the capture
+    src.write_text("// a new comment\nint a = 1;  /* edited */\n\n")   # comments only: same code
+    assert bench.recorded_traffic() == 1234567
+    src.write_text("int a = 2;\n")             # the code changed since the capture
     assert bench.recorded_traffic() is None
