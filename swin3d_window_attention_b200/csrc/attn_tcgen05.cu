@@ -432,6 +432,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     constexpr uint32_t idesc_s = idesc_bf16_f32(128, kN, false, false);
     // N = 64 V columns (the box is 64 channels wide for head_dim 32 too) + 16 ones columns
     constexpr uint32_t idesc_o = idesc_bf16_f32(128, kOnesCol + 16, false, true);
+    static_assert(kN / 16 == 9, "the PV chain covers 144 keys");
     // Operand descriptors are linear in the address field (bits 0..13 = address / 16, every
     // operand below 256 KB), so each MMA's descriptor is a base plus a constant: the stage
     // moves it by kStageBytes / 16, a K step by 32 B (K-major) or 16 keys = 2048 B (V).
@@ -451,21 +452,11 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       fence_proxy_async_smem();
       tc_fence_after();
       const uint64_t qd = dq0 + s * kStageStep, kd = qd + (kTileBytes >> 4);
-#pragma unroll
-      for (int kk = 0; kk < HD / 16; ++kk) umma_bf16_ss_leader(tmem + TM_S0, qd + 2 * kk, kd + 2 * kk, idesc_s, kk > 0, leader);
-      if (has_tail) {
-        const uint64_t qtd = qd + ((128 * kRowBytes) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) umma_bf16_ss_leader(tmem + TM_S1, qtd + 2 * kk, kd + 2 * kk, idesc_s, kk > 0, leader);
-      }
+      umma_chain_qk<HD / 16>(tmem + TM_S0, qd, kd, idesc_s, leader);
+      if (has_tail) umma_chain_qk<HD / 16>(tmem + TM_S1, qd + ((128 * kRowBytes) >> 4), kd, idesc_s, leader);
       umma_commit_leader(s_full, leader);
       issued = true;
       return true;
-    };
-    // keys 16kk .. 16kk + 15 of P: blocks of 64 keys (128B swizzle), the last 16 keys in the
-    // 32B-swizzled block
-    auto p_desc = [](uint64_t d128, uint64_t d32, int kk, int block_bytes) {
-      return kk < 8 ? d128 + static_cast<uint64_t>(((kk >> 2) * block_bytes + (kk & 3) * 32) >> 4) : d32;
     };
     auto issue_pv = [&](int jt) -> bool {  // O(jt) = P V of the tile in stage jt % kStages
       const int s = jt % kStages;
@@ -473,20 +464,14 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(o_empty, (jt & 1) ^ 1, limit_ns))) return false;
       tc_fence_after();
       // Moving V by d (bytes / 16) moves the ones block's leading offset by -d.
-      auto v_desc = [&](int kk) {
-        const uint64_t d = s * kStageStep + 128 * kk;
-        return dv0 + d - (d << 16);
-      };
-#pragma unroll
-      for (int kk = 0; kk < kN / 16; ++kk)
-        umma_bf16_ss_leader(tmem + TM_O0, p_desc(dp0, dp0b, kk, OFF_P0B1 - OFF_P0B0), v_desc(kk), idesc_o, kk > 0, leader);
+      const uint64_t dstage = s * kStageStep;
+      const uint64_t vd = dv0 + dstage - (dstage << 16);
+      umma_chain_pv(tmem + TM_O0, dp0, vd, idesc_o, leader, dp0b, ((OFF_P0B1 - OFF_P0B0) >> 4) - 6);
       umma_commit_leader(p_empty, leader);
       if (has_tail) {
         if (!__all_sync(0xffffffffu, mbar_wait_bounded(p_full_t, jt & 1, limit_ns))) return false;
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kN / 16; ++kk)
-          umma_bf16_ss_leader(tmem + TM_O1, p_desc(dp1, dp1b, kk, OFF_P1B1 - OFF_P1B0), v_desc(kk), idesc_o, kk > 0, leader);
+        umma_chain_pv(tmem + TM_O1, dp1, vd, idesc_o, leader, dp1b, ((OFF_P1B1 - OFF_P1B0) >> 4) - 6);
       }
       if (has_tail) umma_commit_leader(p_empty_t, leader);
       umma_commit_leader(o_full, leader);

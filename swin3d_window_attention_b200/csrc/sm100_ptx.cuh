@@ -164,6 +164,59 @@ __device__ __forceinline__ void umma_bf16_ss_leader(uint32_t d_tmem, uint64_t a_
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(leader)
       : "memory");
 }
+// Whole MMA chains in one asm block, so the descriptor steps are plain 64-bit adds between
+// the MMAs (each tcgen05.mma otherwise costs a block of operand moves).  Executed by the
+// whole warp; only `leader` issues.  The first MMA of a chain overwrites D, the rest
+// accumulate.
+#define S3W_MMA_(A, B, P) "@q tcgen05.mma.cta_group::1.kind::f16 [%0], " A ", " B ", %3, " P ";\n\t"
+// S = Q K^T over head_dim / 16 K steps of 32 bytes (K-major, 128B swizzle)
+template <int KSTEPS>
+__device__ __forceinline__ void umma_chain_qk(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc,
+                                              uint32_t leader) {
+  static_assert(KSTEPS == 2 || KSTEPS == 4, "head_dim 32 or 64");
+  if constexpr (KSTEPS == 4) {
+    asm volatile(
+        "{\n\t.reg .pred q, f, t;\n\t.reg .b64 a, b;\n\t"
+        "setp.ne.b32 q, %4, 0;\n\tsetp.ne.b32 f, %4, %4;\n\tsetp.eq.b32 t, %4, %4;\n\t"
+        "mov.b64 a, %1;\n\tmov.b64 b, %2;\n\t" S3W_MMA_("a", "b", "f")
+        "add.s64 a, a, 2;\n\tadd.s64 b, b, 2;\n\t" S3W_MMA_("a", "b", "t")
+        "add.s64 a, a, 2;\n\tadd.s64 b, b, 2;\n\t" S3W_MMA_("a", "b", "t")
+        "add.s64 a, a, 2;\n\tadd.s64 b, b, 2;\n\t" S3W_MMA_("a", "b", "t") "}" ::"r"(d_tmem),
+        "l"(a0), "l"(b0), "r"(idesc), "r"(leader)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred q, f, t;\n\t.reg .b64 a, b;\n\t"
+        "setp.ne.b32 q, %4, 0;\n\tsetp.ne.b32 f, %4, %4;\n\tsetp.eq.b32 t, %4, %4;\n\t"
+        "mov.b64 a, %1;\n\tmov.b64 b, %2;\n\t" S3W_MMA_("a", "b", "f")
+        "add.s64 a, a, 2;\n\tadd.s64 b, b, 2;\n\t" S3W_MMA_("a", "b", "t") "}" ::"r"(d_tmem),
+        "l"(a0), "l"(b0), "r"(idesc), "r"(leader)
+        : "memory");
+  }
+}
+// O = P V over 144 keys in 9 K steps of 16 keys.  P: steps of 32 bytes inside a 64-key
+// block, `block_step` (descriptor units) to the next block after every fourth step, and the
+// last 16 keys from `p_last` (a separately swizzled block).  V: each step moves the address
+// field by 2048 / 16 and the leading byte offset (the ones block behind it) by the opposite.
+__device__ __forceinline__ void umma_chain_pv(uint32_t d_tmem, uint64_t p0, uint64_t v0, uint32_t idesc,
+                                              uint32_t leader, uint64_t p_last, uint64_t block_step) {
+  asm volatile(
+      "{\n\t.reg .pred q, f, t;\n\t.reg .b64 a, b;\n\t"
+      "setp.ne.b32 q, %4, 0;\n\tsetp.ne.b32 f, %4, %4;\n\tsetp.eq.b32 t, %4, %4;\n\t"
+      "mov.b64 a, %1;\n\tmov.b64 b, %2;\n\t" S3W_MMA_("a", "b", "f")
+      "add.s64 a, a, 2;\n\tadd.s64 b, b, -8388480;\n\t" S3W_MMA_("a", "b", "t")
+      "add.s64 a, a, 2;\n\tadd.s64 b, b, -8388480;\n\t" S3W_MMA_("a", "b", "t")
+      "add.s64 a, a, 2;\n\tadd.s64 b, b, -8388480;\n\t" S3W_MMA_("a", "b", "t")
+      "add.s64 a, a, %6;\n\tadd.s64 b, b, -8388480;\n\t" S3W_MMA_("a", "b", "t")
+      "add.s64 a, a, 2;\n\tadd.s64 b, b, -8388480;\n\t" S3W_MMA_("a", "b", "t")
+      "add.s64 a, a, 2;\n\tadd.s64 b, b, -8388480;\n\t" S3W_MMA_("a", "b", "t")
+      "add.s64 a, a, 2;\n\tadd.s64 b, b, -8388480;\n\t" S3W_MMA_("a", "b", "t")
+      "add.s64 b, b, -8388480;\n\t" S3W_MMA_("%5", "b", "t") "}" ::"r"(d_tmem),
+      "l"(p0), "l"(v0), "r"(idesc), "r"(leader), "l"(p_last), "l"(block_step)
+      : "memory");
+}
+#undef S3W_MMA_
+
 __device__ __forceinline__ void umma_commit_leader(uint32_t bar, uint32_t leader) {
   asm volatile(
       "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %1, 0;\n\t"
