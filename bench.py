@@ -1,30 +1,45 @@
 #!/usr/bin/env python3
 """Benchmark of the Swin3D shifted-window attention hot path on B200.
 
-One step = one pass of the whole path over one batch of the Aurora 0.25-degree
-encoder stage-1 workload (B=1, grid 4x180x360, C=512 = 8 heads x 64, window (2,6,12)):
+Headline step (the workload the metric is quoted on): one pass of the whole path over the
+Aurora 0.25-degree encoder stage-1 grid (B=1, grid 4x180x360, C=512 = 8 heads x 64,
+window (2,6,12)):
 
     window attention, shift (0,0,0)  -> AdaLN + residual (fp32 residual stream, in place)
     window attention, shift (1,3,6)  -> AdaLN + residual
 
-Each attention call reads fresh seeded bf16 Q/K/V (N(0,1)), the AdaLN calls take the
-attention output, per-sample FiLM scale/shift N(0,0.1) and the fp32 residual stream.
-Every input tensor is larger than the 126 MB L2, so no flush is needed between steps.
+Each attention call reads its own seeded bf16 Q/K/V (N(0,1)); the AdaLN calls take the
+attention output, per-sample FiLM scale/shift N(0,0.1) and the fp32 residual stream.  Every
+input tensor is larger than the 126 MB L2, so no flush is needed between steps.
 
-Output: one JSON line (rank 0).  ``value`` is windows per second over all ranks (each
-step processes 2 x 1800 windows x 8 heads per rank).  ``--impl reference`` times the
-fp64 CPU oracle on a bounded sample of the same workload instead.
+``value`` is windows per second over all ranks (each step processes 2 x 1800 windows of 8
+heads per rank).  Besides the headline the JSON line carries:
+
+* ``attn`` / ``adaln``: per-launch statistics of the two kernels inside the timed region;
+* ``roofline``: the binding roofline of the attention kernel, max(bytes/BW, FLOPs/peak),
+  with the DRAM traffic of the committed ncu capture while it still matches the code;
+* ``configs``: the other workloads of the set, each timed on its own (N=1 only): the tiny
+  grid, stage 2 with AdaLN at C=1024, stage 3 with padding, the six-block stage-1 stack at
+  B=4, each with its algorithmic bytes, FLOPs and roofline fraction;
+* ``e2e``: the headline step through the public API with pinned host buffers;
+* ``cpu_baseline``: the fp64 oracle on the host cores, on bounded samples of the same
+  workloads (rank 0, N=1).
+
+``--impl reference`` times the fp64 CPU oracle on samples of the headline workload as the
+reference arm (same sampler as ``cpu_baseline``).
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
+import math
 import os
+import re
 import statistics
 import subprocess
 import sys
 import tempfile
-import threading
 import time
 
 import numpy as np
@@ -32,28 +47,139 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-# Workload: Aurora 0.25-degree encoder stage 1.
-B, T, H, W = 1, 4, 180, 360
-HEADS, HD = 8, 64
-C = HEADS * HD
 WINDOW = (2, 6, 12)
-SHIFTS = ((0, 0, 0), (1, 3, 6))
-N_TOK = 144
-L = T * H * W
-N_WIN = B * (T // 2) * (H // 6) * (W // 12)          # 1800 windows per call
-ATTN_BYTES = 4 * B * L * C * 2                         # read Q, K, V once, write O once (bf16)
-ATTN_FLOPS = N_WIN * HEADS * 4 * N_TOK * N_TOK * HD    # QK^T and PV, dense in each window
-ADALN_BYTES = B * L * C * (2 + 4 + 4)                  # bf16 x, fp32 residual in, fp32 out
+N_TOK = WINDOW[0] * WINDOW[1] * WINDOW[2]
+UNSHIFTED, SHIFTED = (0, 0, 0), (1, 3, 6)
+SHIFTS = (UNSHIFTED, SHIFTED)
+
+# The benchmark set: grid, heads x head_dim.  "stage1" is the headline workload.
+WORKLOADS = {
+    "tiny": dict(B=1, T=2, H=15, W=30, heads=2, hd=32),
+    "stage1": dict(B=1, T=4, H=180, W=360, heads=8, hd=64),
+    "stage2": dict(B=1, T=4, H=90, W=180, heads=16, hd=64),
+    "stage3_padded": dict(B=2, T=4, H=45, W=90, heads=32, hd=64),
+    "stack_b4": dict(B=4, T=4, H=180, W=360, heads=8, hd=64),
+}
+STACK_BLOCKS = 6
+METRIC = "window-attn TFLOP/s, HBM GB/s & % of roofline on 1 B200; windows/s"
 WORKLOAD = ("Aurora 0.25deg encoder stage 1: B=1, grid T4xH180xW360, C=512 (8 heads x 64), window (2,6,12); "
             "per step: attn shift (0,0,0) + AdaLN fp32-out, attn shift (1,3,6) + AdaLN fp32-out")
+PROFILE = os.path.join("profiles", "window_attn_tc_stage1.json")
+KERNEL_SOURCES = [os.path.join("swin3d_window_attention_b200", "csrc", f)
+                  for f in ("attn_tcgen05.cu", "sm100_ptx.cuh", "s3w_common.cuh")]
+
+
+def geometry(w):
+    """Derived sizes of a workload: channels, tokens, windows (all samples)."""
+    C = w["heads"] * w["hd"]
+    tokens = w["B"] * w["T"] * w["H"] * w["W"]
+    windows = w["B"] * math.prod(-(-d // a) for d, a in zip((w["T"], w["H"], w["W"]), WINDOW))
+    return C, tokens, windows
+
+
+def attn_bytes(w, o_bytes=2):
+    """Read Q, K, V once and write O once (bf16 in): padding and the shift never touch HBM."""
+    C, tokens, _ = geometry(w)
+    return (3 * 2 + o_bytes) * tokens * C
+
+
+def attn_flops(w):
+    """4 N^2 d per (window, head): QK^T and PV, dense inside each window."""
+    _, _, windows = geometry(w)
+    return windows * w["heads"] * 4 * N_TOK * N_TOK * w["hd"]
+
+
+def adaln_bytes(w, x_bytes=2, out_bytes=4):
+    """x, the fp32 residual and the output, once each (scale/shift are negligible)."""
+    C, tokens, _ = geometry(w)
+    return tokens * C * (x_bytes + 4 + out_bytes)
+
+
+S1 = WORKLOADS["stage1"]
+C1, L1, N_WIN = geometry(S1)
+ATTN_BYTES, ATTN_FLOPS, ADALN_BYTES = attn_bytes(S1), attn_flops(S1), adaln_bytes(S1)
+CONFIG = {"workload": WORKLOAD, "global_batch": S1["B"], "windows_per_call": N_WIN, "heads": S1["heads"],
+          "head_dim": S1["hd"], "l2": "inputs larger than L2 (265 MB per tensor), no flush",
+          "parallelism": "single GPU"}
+
+
+def config_for(world):
+    c = dict(CONFIG)
+    c["global_batch"] = S1["B"] * world
+    if world > 1:
+        c["parallelism"] = f"replicas x{world}"
+    return c
 
 
 def load_peaks():
+    """Measured peaks of this machine's B200s if the driver wrote them, else the fallback."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
-    return 6650.0, 1590.0, "fallback"
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def roofline(nbytes, flops, ms, peaks):
+    """Binding roofline: the larger of bytes/BW and FLOPs/peak; frac = that time / measured."""
+    t = ms * 1e-3
+    t_bw = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    if t_bw >= t_tc:
+        r = {"bound": "hbm", "achieved": nbytes / t / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+             "frac": t_bw / t}
+    else:
+        r = {"bound": "tensor", "achieved": flops / t / 1e12, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+             "frac": t_tc / t}
+    r["frac_of_nominal_8tbs"] = nbytes / t / 8e12
+    r["tensor_frac"] = flops / t / 1e12 / peaks["bf16_tflops"]
+    return r
+
+
+def code_sha256(text):
+    """sha256 of source code with comments and blank lines removed, so that editing a
+    comment does not separate a capture from the code it measured."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines()]
+    return hashlib.sha256("\n".join(ln for ln in lines if ln.strip()).encode()).hexdigest()
+
+
+def kernel_code_sha256(root=None):
+    """Code hash of the attention kernel's translation unit (kernel source + its headers)."""
+    root = ROOT if root is None else root
+    return code_sha256("\n".join(open(os.path.join(root, f)).read() for f in KERNEL_SOURCES))
+
+
+def recorded_profile(root=None):
+    """The committed ncu capture of the attention kernel, or None if its code changed since."""
+    root = ROOT if root is None else root
+    p = os.path.join(root, PROFILE)
+    if not os.path.exists(p):
+        return None
+    try:
+        prof = json.load(open(p))
+        if prof.get("code_sha256") != kernel_code_sha256(root):
+            return None
+        return prof
+    except (OSError, ValueError, KeyError):
+        return None
+
+
+def recorded_traffic(root=None):
+    """DRAM bytes per attention launch (read + write) from the committed capture, or None."""
+    prof = recorded_profile(root)
+    if prof is None:
+        return None
+    return int(prof["dram_bytes_read"]) + int(prof["dram_bytes_write"])
+
+
+def launch_stats(ms):
+    s = sorted(ms)
+    q = lambda f: s[min(len(s) - 1, int(f * len(s)))]
+    return {"avg_launch_ms": statistics.fmean(s), "median_ms": statistics.median(s), "p10_ms": q(0.1),
+            "p90_ms": q(0.9), "min_ms": s[0], "max_ms": s[-1], "launches": len(s)}
 
 
 class ClockSampler:
@@ -117,51 +243,123 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
-def make_device_inputs(torch, dev):
-    """Seeded inputs: two Q/K/V sets (one per attention call), FiLM vectors, residual."""
+# ----------------------------------------------------------------------------- GPU arm
+def device_qkv(torch, w, dev, base):
+    """Seeded bf16 Q, K, V of a workload, drawn on the device."""
     from swin3d_window_attention_b200 import inputs
 
-    host = {}
-    for i, _ in enumerate(SHIFTS):
-        for j, name in enumerate("qkv"):
-            host[f"{name}{i}"] = inputs.normal_bf16_bits((B, T, H, W, C), tensor_index=100 + 10 * i + j)
-    host["scale"] = inputs.normal_f32_tensor((B, C), tensor_index=200, sigma=0.1)
-    host["shift"] = inputs.normal_f32_tensor((B, C), tensor_index=201, sigma=0.1)
-    host["res"] = inputs.normal_f32_tensor((B, L, C), tensor_index=202)
-    devt = {}
-    for kname, a in host.items():
-        t = inputs.bits_to_torch_bf16(a) if a.dtype == np.uint16 else torch.from_numpy(a)
-        devt[kname] = t.to(dev)
-    return host, devt
+    C = w["heads"] * w["hd"]
+    shape = (w["B"], w["T"], w["H"], w["W"], C)
+    return [inputs.normal_bf16_torch(shape, dev, tensor_index=base + j) for j in range(3)]
 
 
+def device_film(torch, w, dev, base, sigma):
+    from swin3d_window_attention_b200 import inputs
 
-def kernel_code_sha256(text):
-    """sha256 of a source file's code: comments and blank lines removed, so that editing a
-    comment does not separate a capture from the kernel it measured."""
-    import hashlib
-    import re
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines()]
-    return hashlib.sha256("\n".join(ln for ln in lines if ln.strip()).encode()).hexdigest()
+    C, tokens, _ = geometry(w)
+    sc = inputs.normal_f32_torch(w["B"] * C, dev, tensor_index=base, sigma=sigma).reshape(w["B"], C)
+    sh = inputs.normal_f32_torch(w["B"] * C, dev, tensor_index=base + 1, sigma=sigma).reshape(w["B"], C)
+    res = inputs.normal_f32_torch(tokens * C, dev, tensor_index=base + 2).reshape(w["B"], tokens // w["B"], C)
+    return sc, sh, res
 
 
-def recorded_traffic():
-    """DRAM bytes per attention launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
-    committed ncu summary, or None if the kernel's code changed since that capture."""
-    import re
-    summ = os.path.join(ROOT, "profiles", "window_attn_tc_stage1_full.md")
-    src = os.path.join(ROOT, "swin3d_window_attention_b200", "csrc", "attn_tcgen05.cu")
-    if not (os.path.exists(summ) and os.path.exists(src)):
-        return None
-    text = open(summ).read()
-    sha = re.search(r"code sha256 `([0-9a-f]{64})`", text)
-    nbytes = re.search(r"dram_bytes_per_launch: (\d+)", text)
-    if not sha or not nbytes:
-        return None
-    if kernel_code_sha256(open(src).read()) != sha.group(1):
-        return None
-    return int(nbytes.group(1))
+def timed(torch, stream, fn, reps, warmup=3):
+    """Per-call device times (ms) of fn, CUDA events on the launching stream."""
+    for _ in range(warmup):
+        fn()
+    ev = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        ev.append((a, b))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def bench_configs(torch, s3w, dev, stream, peaks, reps):
+    """Every workload of the set besides the headline, each timed on its own."""
+    out = {}
+    launches = 0
+    # tiny grid: launch-bound, latency reported
+    w = WORKLOADS["tiny"]
+    q, k, v = device_qkv(torch, w, dev, 900)
+    o = torch.empty_like(q)
+    ms = timed(torch, stream, lambda: s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTED),
+               reps)
+    launches += len(ms)
+    out["tiny"] = {"grid": "B=1 T2xH15xW30 (padded 2x18x36), 2 heads x 32, shift (1,3,6), 9 windows",
+                   "attn": launch_stats(ms), "latency_us_median": 1e3 * statistics.median(ms)}
+    del q, k, v, o
+
+    # stage 2: shifted attention + AdaLN at C = 1024
+    w = WORKLOADS["stage2"]
+    C, tokens, windows = geometry(w)
+    q, k, v = device_qkv(torch, w, dev, 910)
+    sc, sh, res = device_film(torch, w, dev, 920, 0.1)
+    o = torch.empty_like(q)
+    ms_a = timed(torch, stream, lambda: s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTED),
+                 reps)
+    x = o.view(w["B"], tokens // w["B"], C)
+    ms_n = timed(torch, stream, lambda: s3w.adaln_residual_fwd(x, res, sc, sh, res, eps=1e-5), reps)
+    launches += len(ms_a) + len(ms_n)
+    a_med, n_med = statistics.median(ms_a), statistics.median(ms_n)
+    out["stage2"] = {"grid": "B=1 T4xH90xW180, 16 heads x 64, shift (1,3,6), 450 windows; AdaLN C=1024 fp32 out",
+                     "attn": {**launch_stats(ms_a), "bytes": attn_bytes(w), "flops": attn_flops(w),
+                              "windows_per_s": windows / (a_med * 1e-3),
+                              "roofline": roofline(attn_bytes(w), attn_flops(w), a_med, peaks)},
+                     "adaln": {**launch_stats(ms_n), "bytes": adaln_bytes(w),
+                               "roofline": roofline(adaln_bytes(w), 0, n_med, peaks)}}
+    del q, k, v, o, x, sc, sh, res
+
+    # stage 3: padded grid (45 -> 48, 90 -> 96), padded keys masked, padded outputs dropped
+    w = WORKLOADS["stage3_padded"]
+    _, _, windows = geometry(w)
+    q, k, v = device_qkv(torch, w, dev, 930)
+    o = torch.empty_like(q)
+    ms_a = timed(torch, stream, lambda: s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTED),
+                 reps)
+    launches += len(ms_a)
+    a_med = statistics.median(ms_a)
+    out["stage3_padded"] = {
+        "grid": "B=2 T4xH45xW90 (padded 4x48x96), 32 heads x 64, shift (1,3,6), 256 windows",
+        "attn": {**launch_stats(ms_a), "bytes": attn_bytes(w), "flops": attn_flops(w),
+                 "windows_per_s": windows / (a_med * 1e-3),
+                 "roofline": roofline(attn_bytes(w), attn_flops(w), a_med, peaks)}}
+    del q, k, v, o
+
+    # six-block stage-1 stack at B = 4: fresh Q/K/V per block, fp32 residual chained
+    w = WORKLOADS["stack_b4"]
+    C, tokens, windows = geometry(w)
+    qkv = [device_qkv(torch, w, dev, 1000 + 10 * b) for b in range(STACK_BLOCKS)]
+    films = [device_film(torch, w, dev, 1100 + 10 * b, 1.0)[:2] for b in range(STACK_BLOCKS)]
+    res = device_film(torch, w, dev, 1190, 1.0)[2]
+    o = torch.empty_like(qkv[0][0])
+    x = o.view(w["B"], tokens // w["B"], C)
+
+    def stack():
+        for b in range(STACK_BLOCKS):
+            q, k, v = qkv[b]
+            s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTS[b % 2])
+            s3w.adaln_residual_fwd(x, res, films[b][0], films[b][1], res, eps=1e-5)
+
+    stack_reps = max(3, reps // 4)
+    ms_s = timed(torch, stream, stack, stack_reps, warmup=2)
+    launches += 2 * STACK_BLOCKS * stack_reps
+    s_med = statistics.median(ms_s)
+    nbytes = STACK_BLOCKS * (attn_bytes(w) + adaln_bytes(w))
+    flops = STACK_BLOCKS * attn_flops(w)
+    out["stack_b4"] = {
+        "grid": "B=4 T4xH180xW360, 8 heads x 64, 6 x (attn alternating shift + AdaLN fp32 out), 7200 windows per call",
+        "ms_per_stack": launch_stats(ms_s), "bytes": nbytes, "flops": flops,
+        "floor_ms_at_measured_hbm": nbytes / (peaks["hbm_gbs"] * 1e9) * 1e3,
+        "windows_per_s": STACK_BLOCKS * windows / (s_med * 1e-3),
+        "roofline": roofline(nbytes, flops, s_med, peaks)}
+    del qkv, films, res, o, x
+    torch.cuda.empty_cache()
+    return out, launches
+
 
 def bench_cuda(args):
     import torch
@@ -185,23 +383,36 @@ def bench_cuda(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     s3w.load_library()
     stream = torch.cuda.current_stream(dev)
-    host, d = make_device_inputs(torch, dev)
-    o = torch.empty((B, T, H, W, C), dtype=torch.bfloat16, device=dev)
+    peaks = load_peaks()
+
+    # headline inputs: one Q/K/V set per attention call, FiLM vectors, residual stream
+    d = {}
+    for i, _ in enumerate(SHIFTS):
+        d[f"q{i}"], d[f"k{i}"], d[f"v{i}"] = device_qkv(torch, S1, dev, 100 + 10 * i)
+    d["scale"], d["shift"], d["res"] = device_film(torch, S1, dev, 200, 0.1)
+    o = torch.empty((S1["B"], S1["T"], S1["H"], S1["W"], C1), dtype=torch.bfloat16, device=dev)
     res = d["res"]
+    x = o.view(S1["B"], L1 // S1["B"], C1)
     launches_per_step = 4
-    attn_events = []
+    attn_ev, adaln_ev = [], []
+
+    def ev_pair():
+        return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
     def step(record=False):
         for i, shift in enumerate(SHIFTS):
             if record:
-                e0 = torch.cuda.Event(enable_timing=True)
-                e1 = torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-            s3w.swin3d_window_attn_fwd(d[f"q{i}"], d[f"k{i}"], d[f"v{i}"], o, HEADS, HD, WINDOW, shift)
+                a0, a1 = ev_pair()
+                a0.record(stream)
+            s3w.swin3d_window_attn_fwd(d[f"q{i}"], d[f"k{i}"], d[f"v{i}"], o, S1["heads"], S1["hd"], WINDOW, shift)
             if record:
-                e1.record(stream)
-                attn_events.append((e0, e1))
-            s3w.adaln_residual_fwd(o.view(B, L, C), res, d["scale"], d["shift"], res, eps=1e-5)
+                a1.record(stream)
+                attn_ev.append((a0, a1))
+            s3w.adaln_residual_fwd(x, res, d["scale"], d["shift"], res, eps=1e-5)
+            if record:
+                a2 = torch.cuda.Event(enable_timing=True)
+                a2.record(stream)
+                adaln_ev.append((a1, a2))
 
     for _ in range(args.warmup):
         step()
@@ -214,6 +425,8 @@ def bench_cuda(args):
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
     wall0 = time.time()
     t0.record(stream)
     for _ in range(args.steps):
@@ -221,6 +434,8 @@ def bench_cuda(args):
     t1.record(stream)
     torch.cuda.synchronize()
     wall1 = time.time()
+    if dist:
+        dist.barrier()
     ms = t0.elapsed_time(t1)
     clk = clocks.stop((wall0, wall1))
     if s3w.poll_device_error() != 0:
@@ -229,30 +444,22 @@ def bench_cuda(args):
         tt = torch.tensor([ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         ms = float(tt.item())
-        dist.barrier()
-    attn_ms = [a.elapsed_time(b) for a, b in attn_events]
-    attn_avg_ms = sum(attn_ms) / len(attn_ms)
+    attn_ms = [a.elapsed_time(b) for a, b in attn_ev]
+    adaln_ms = [a.elapsed_time(b) for a, b in adaln_ev]
+    attn = launch_stats(attn_ms)
+    adaln = launch_stats(adaln_ms)
+    attn_med, adaln_med = attn["median_ms"], adaln["median_ms"]
 
     # For context: the same attention call on the legacy mma.sync baseline kernel.
-    leg = []
-    for i in range(3):
-        a0 = torch.cuda.Event(enable_timing=True)
-        a1 = torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        s3w.swin3d_window_attn_fwd_legacy_mma(d["q1"], d["k1"], d["v1"], o, HEADS, HD, WINDOW, SHIFTS[1])
-        a1.record(stream)
-        leg.append((a0, a1))
-    torch.cuda.synchronize()
-    legacy_ms = min(a.elapsed_time(b) for a, b in leg)
+    leg = timed(torch, stream, lambda: s3w.swin3d_window_attn_fwd_legacy_mma(
+        d["q1"], d["k1"], d["v1"], o, S1["heads"], S1["hd"], WINDOW, SHIFTED), 3, warmup=1)
 
-    # End-to-end through the public API with host buffers: every step copies its inputs
-    # from pinned host memory and reads the step's result (the residual stream) back.
-    pinned = {k: (torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) if v.dtype == np.uint16
-                  else torch.from_numpy(v)).pin_memory() for k, v in host.items()}
-    res_out = torch.empty((B, L, C), dtype=torch.float32).pin_memory()
+    # End to end through the public API with host buffers: every step copies its inputs from
+    # pinned host memory and reads the step's result (the residual stream) back.
+    pinned = {k: t.cpu().pin_memory() for k, t in d.items()}
+    res_out = torch.empty(res.shape, dtype=torch.float32).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
     d2h = res_out.numel() * 4
-    e2e_steps = max(1, min(args.steps, 5))
 
     def e2e_step():
         for kname, t in pinned.items():
@@ -264,28 +471,39 @@ def bench_cuda(args):
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
+    e0, e1 = ev_pair()
     e0.record(stream)
-    for _ in range(e2e_steps):
+    for _ in range(args.steps):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    e2e_ms = e0.elapsed_time(e1) / args.steps
     if dist:
         tt = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         e2e_ms = float(tt.item())
+    del pinned, res_out
 
-    hbm_peak, tc_peak, peak_src = load_peaks()
+    configs, extra_launches = None, 0
+    if world == 1 and not args.no_configs:
+        del d, o, x, res
+        torch.cuda.empty_cache()
+        configs, extra_launches = bench_configs(torch, s3w, dev, stream, peaks, args.config_reps)
+        if s3w.poll_device_error() != 0:
+            raise SystemExit("device error word set during the per-config runs")
+
     ms_step = ms / args.steps
     windows_per_step = len(SHIFTS) * N_WIN
-    value = windows_per_step * world / (ms_step * 1e-3)
-    attn_gbs = ATTN_BYTES / (attn_avg_ms * 1e-3) / 1e9
-    attn_tflops = ATTN_FLOPS / (attn_avg_ms * 1e-3) / 1e12
+    rl = roofline(ATTN_BYTES, ATTN_FLOPS, attn_med, peaks)
+    prof = recorded_profile()
+    rl.update({"traffic": None if prof is None else int(prof["dram_bytes_read"]) + int(prof["dram_bytes_write"]),
+               "traffic_source": None if prof is None else PROFILE, "peak_source": peaks["source"],
+               "kernel": "window_attn_tc_kernel<64, bf16 out> (window attention)",
+               "algorithmic_bytes_per_launch": ATTN_BYTES, "flops_per_launch": ATTN_FLOPS,
+               "timing": "median of the per-launch CUDA-event times inside the timed region"})
     line = {
-        "metric": "window-attn TFLOP/s, HBM GB/s & % of roofline on 1 B200; windows/s",
-        "value": value,
+        "metric": METRIC,
+        "value": windows_per_step * world / (ms_step * 1e-3),
         "unit": "windows/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -296,21 +514,21 @@ def bench_cuda(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 Q/K/V, N(0,0.1) FiLM, N(0,1) fp32 residual)",
-        "config": {"workload": WORKLOAD, "global_batch": B * world, "windows_per_call": N_WIN, "heads": HEADS,
-                   "head_dim": HD, "l2": "inputs larger than L2 (265 MB per tensor), no flush",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-        "attn": {"avg_launch_ms": attn_avg_ms, "hbm_gbs": attn_gbs, "tflops": attn_tflops,
-                 "windows_per_s": N_WIN / (attn_avg_ms * 1e-3),
-                 "hbm_frac": attn_gbs / hbm_peak, "tensor_frac": attn_tflops / tc_peak,
-                 "legacy_mma_baseline_ms": legacy_ms},
-        "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": attn_gbs / hbm_peak, "traffic": recorded_traffic(), "peak_source": peak_src,
-                     "kernel": "window attention", "algorithmic_bytes_per_launch": ATTN_BYTES},
+        "config": config_for(world),
+        "attn": {**attn, "bytes": ATTN_BYTES, "flops": ATTN_FLOPS, "hbm_gbs": ATTN_BYTES / (attn_med * 1e-3) / 1e9,
+                 "tflops": ATTN_FLOPS / (attn_med * 1e-3) / 1e12, "windows_per_s": N_WIN / (attn_med * 1e-3),
+                 "legacy_mma_baseline_ms": min(leg)},
+        "adaln": {**adaln, "bytes": ADALN_BYTES, "hbm_gbs": ADALN_BYTES / (adaln_med * 1e-3) / 1e9,
+                  "frac": ADALN_BYTES / (adaln_med * 1e-3) / 1e9 / peaks["hbm_gbs"], "peak_source": peaks["source"]},
+        "roofline": rl,
         "e2e": {"value": windows_per_step * world / (e2e_ms * 1e-3), "unit": "windows/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": args.steps},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }
+    if configs is not None:
+        line["configs"] = configs
+        line["gpu_launches_outside_timed_region"] = extra_launches + len(leg) + 1
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     if dist:
@@ -319,72 +537,127 @@ def bench_cuda(args):
         print(json.dumps(line), flush=True)
 
 
-_CPU_INPUTS = []
+# ----------------------------------------------------------------------------- CPU oracle
+class OracleSampler:
+    """The fp64 oracle timed on bounded samples of a workload's windows.
 
+    One sample = a batch of random windows (all heads) of the workload's grid through
+    ``oracle.window_attn``, plus AdaLN on those windows' tokens where the workload has
+    AdaLN.  Both benchmark arms use this one procedure: a short untimed warm-up, then
+    batches until the time budget is spent.  Host inputs are seeded draws of the workload's
+    shape (made once, not timed)."""
 
-def cpu_sample(seconds_budget):
-    """Time the fp64 oracle on a bounded sample of the workload: whole windows (all heads)
-    of both attention calls plus AdaLN on those windows' tokens.  Returns (windows, s, threads)."""
-    import oracle
-    from swin3d_window_attention_b200 import inputs
+    BATCH = 8
 
-    oracle.build()
-    rng = np.random.default_rng(0)
-    # The oracle indexes the full grid, so one full-size input set is built once (not timed).
-    if not _CPU_INPUTS:
-        _CPU_INPUTS.extend([inputs.normal_bf16_bits((B, T, H, W, C), tensor_index=100 + j) for j in range(3)])
-        _CPU_INPUTS.append(inputs.normal_f32_tensor((B, C), tensor_index=200, sigma=0.1))
-        _CPU_INPUTS.append(inputs.normal_f32_tensor((B, C), tensor_index=201, sigma=0.1))
-    q, k, v, sc, sh = _CPU_INPUTS
-    done = 0
-    t_start = time.perf_counter()
-    batch = 8
-    while True:
-        for shift in SHIFTS:
-            ids = rng.integers(0, N_WIN, size=batch)
-            out, tok, _ = oracle.window_attn(q, k, v, HEADS, HD, WINDOW, shift, window_ids=ids)
-            x = out.reshape(1, -1, C)
-            res = np.zeros((1, x.shape[1], C), dtype=np.float32)
-            oracle.adaln(x, res, sc, sh, eps=1e-5)
+    def __init__(self):
+        import oracle
+
+        oracle.build()
+        self.oracle = oracle
+        self.cache = {}
+
+    def inputs(self, name):
+        if name not in self.cache:
+            import torch
+
+            from swin3d_window_attention_b200 import inputs
+
+            w = WORKLOADS[name]
+            C = w["heads"] * w["hd"]
+            shape = (w["B"], w["T"], w["H"], w["W"], C)
+            qkv = [inputs.torch_bf16_to_bits(inputs.normal_bf16_torch(shape, "cpu", tensor_index=1300 + j))
+                   for j in range(3)]
+            film = [inputs.normal_f32_tensor((w["B"], C), tensor_index=1310 + j, sigma=0.1) for j in range(2)]
+            self.cache[name] = (qkv, film)
+            del torch
+        return self.cache[name]
+
+    def run(self, name, shifts, adaln, seconds, seed=0):
+        """Windows per second of the oracle; returns (windows, seconds, threads)."""
+        w = WORKLOADS[name]
+        C, _, windows = geometry(w)
+        (q, k, v), (sc, sh) = self.inputs(name)
+        rng = np.random.default_rng(seed)
+        batch = min(self.BATCH, windows)
+
+        def one(shift):
+            ids = rng.integers(0, windows, size=batch)
+            out, tok, _ = self.oracle.window_attn(q, k, v, w["heads"], w["hd"], WINDOW, shift, window_ids=ids)
+            if adaln:
+                xo = out.reshape(1, -1, C)
+                self.oracle.adaln(xo, np.zeros(xo.shape, dtype=np.float32), sc[:1], sh[:1], eps=1e-5)
+
+        one(shifts[0])   # warm-up: threads started, pages touched
+        done, i = 0, 0
+        t0 = time.perf_counter()
+        while True:
+            one(shifts[i % len(shifts)])
+            i += 1
             done += batch
-        el = time.perf_counter() - t_start
-        if el >= seconds_budget:
-            break
-    return done, el, oracle.num_threads()
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                return done, el, self.oracle.num_threads()
 
 
-def cpu_baseline(seconds_budget):
-    wins, el, thr = cpu_sample(seconds_budget)
-    return {"value": wins / el, "unit": "windows/s", "cores": thr, "kind": "oracle",
-            "sample": f"{wins} random windows (all 8 heads, both shifts alternating) + AdaLN on their tokens, "
-                      f"{el:.1f} s on {thr} threads"}
+_SAMPLER = []
+
+
+def sampler():
+    if not _SAMPLER:
+        _SAMPLER.append(OracleSampler())
+    return _SAMPLER[0]
+
+
+def cpu_baseline(seconds):
+    """The oracle on the headline workload and on every other workload of the set."""
+    smp = sampler()
+    wins, el, thr = smp.run("stage1", SHIFTS, True, seconds)
+    rate = wins / el
+    per = {}
+    other = max(2.0, seconds / 5)
+    for name, shifts, adaln in (("tiny", (SHIFTED,), False), ("stage2", (SHIFTED,), True),
+                                ("stage3_padded", (SHIFTED,), False)):
+        wn, e, _ = smp.run(name, shifts, adaln, other)
+        per[name] = {"windows_per_s": wn / e, "sample": f"{wn} random windows in {e:.1f} s"}
+    per["stage1"] = {"windows_per_s": rate, "sample": f"{wins} random windows in {el:.1f} s"}
+    # One block of the B=4 stack has the per-window work of stage 1 (same grid and heads).
+    stack_windows = STACK_BLOCKS * geometry(WORKLOADS["stack_b4"])[2]
+    per["stack_b4"] = {"windows_per_s": rate, "extrapolated": True,
+                       "seconds_per_stack": stack_windows / rate,
+                       "sample": "one block timed on stage-1 windows (same per-window work), x6 blocks extrapolated"}
+    return {"value": rate, "unit": "windows/s", "cores": thr, "kind": "oracle",
+            "sample": f"{wins} random stage-1 windows (8 heads each, both shifts alternating) + AdaLN on their "
+                      f"tokens, {el:.1f} s on {thr} threads, after one untimed batch",
+            "configs": per}
 
 
 def bench_reference(args):
-    """The fp64 oracle as the reference arm, on the host cores, same metric and unit."""
+    """The fp64 oracle as the reference arm, on the host cores: same metric, unit, config
+    and sampler as the CUDA arm's cpu_baseline."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
+    smp = sampler()
+    per_step = max(0.5, args.cpu_seconds / max(1, args.steps))
     for _ in range(args.warmup):
-        cpu_sample(0.5)
+        smp.run("stage1", SHIFTS, True, 0.2)
     wins_total, el_total, thr = 0, 0.0, 1
-    for _ in range(args.steps):
-        w, el, thr = cpu_sample(per_step)
-        wins_total += w
+    for k in range(args.steps):
+        wn, el, thr = smp.run("stage1", SHIFTS, True, per_step, seed=k)
+        wins_total += wn
         el_total += el
     value = wins_total / el_total
     line = {
         "impl": "reference",
-        "metric": "window-attn TFLOP/s, HBM GB/s & % of roofline on 1 B200; windows/s",
+        "metric": METRIC,
         "value": value, "unit": "windows/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * el_total / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, same generator as the CUDA arm)",
-        "config": {"workload": WORKLOAD, "global_batch": B, "windows_per_call": N_WIN, "heads": HEADS,
-                   "head_dim": HD},
+        "config": config_for(world),
         "cpu_baseline": {"value": value, "unit": "windows/s", "cores": thr, "kind": "oracle",
-                         "sample": f"{wins_total} random windows over {args.steps} steps of ~{per_step:.1f} s"},
+                         "sample": f"{wins_total} random stage-1 windows + AdaLN on their tokens over {args.steps} "
+                                   f"steps of ~{per_step:.1f} s on {thr} threads"},
         "e2e": {"value": value, "unit": "windows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -393,11 +666,13 @@ def bench_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--config-reps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -69,6 +69,12 @@ typedef enum { S3W_BF16 = 0, S3W_F32 = 1 } s3w_dtype;
 /*
  * Shifted-window attention forward.
  *
+ * Defines: "Flash-Aurora: Toward Efficient Inference for Geospatial Foundation Models",
+ * section "CuTe DSL window attention" (per window and head: S = scale * Q K^T, the Swin
+ * shift mask, softmax in FP32, O = softmax(S) V; window (2,6,12) -> N = 144; BF16_MIXED)
+ * and section "Kernel fusion for backbone memory traffic" (cyclic shift, pad, 3D window
+ * partition and the inverse merge folded into the kernel).  Semantics: steps 1-5 above.
+ *
  * q, k, v   device pointers, in_dtype elements (S3W_BF16 only), grid layout with
  *           qkv_token_stride elements between consecutive tokens (>= heads*head_dim, a
  *           multiple of 8 so that every token row starts on a 16-byte boundary; q, k and v
@@ -81,7 +87,12 @@ typedef enum { S3W_BF16 = 0, S3W_F32 = 1 } s3w_dtype;
  * shift_*   0 <= shift < window on each axis.
  * heads     >= 1.  head_dim: 32 or 64.
  * scale     logit scale; a value <= 0 selects 1/sqrt(head_dim).
+ * in_dtype, out_dtype  values of s3w_dtype, passed as int (the width of an enum is up to
+ *           the compiler; int keeps the ABI fixed).
  * stream    CUDA stream; the call only enqueues work.
+ *
+ * Separate token strides for q/k/v and for o let q, k, v be slices of one fused QKV
+ * buffer while o is a plain [tokens][C] tensor.
  *
  * Returns S3W_OK or an s3w_status; on error nothing is launched.
  */
@@ -95,22 +106,12 @@ int swin3d_window_attn_fwd(const void* q, const void* k, const void* v, void* o,
                            s3w_stream_t stream);
 
 /*
- * The same operation and the same arguments, checks and results as
- * swin3d_window_attn_fwd, computed on the legacy warp-level tensor path (mma.sync,
- * one CTA per (window, head), loads and math not overlapped).  It is the measured
- * baseline the tcgen05 path is compared with; it has no bounded waits.
- */
-int swin3d_window_attn_fwd_legacy_mma(const void* q, const void* k, const void* v, void* o,
-                                      int B, int T, int H, int W,
-                                      int win_t, int win_h, int win_w,
-                                      int shift_t, int shift_h, int shift_w,
-                                      int heads, int head_dim,
-                                      long long qkv_token_stride, long long o_token_stride,
-                                      float scale, int in_dtype, int out_dtype,
-                                      s3w_stream_t stream);
-
-/*
- * Fused AdaLN + residual forward ("Kernel fusion for backbone memory traffic").
+ * Fused AdaLN + residual forward.
+ *
+ * Defines: "Flash-Aurora: Toward Efficient Inference for Geospatial Foundation Models",
+ * section "Kernel fusion for backbone memory traffic" (LayerNorm, FiLM modulation and the
+ * residual add without a full-width intermediate) and section "Mixed-precision
+ * inference" (FP32 activations between blocks, output_fp32).
  *
  * For every sample b and token l of x[B][L][C] (contiguous rows of C elements):
  *   mean = sum_c x / C,  var = sum_c (x - mean)^2 / C        (biased, two passes)
@@ -125,7 +126,8 @@ int swin3d_window_attn_fwd_legacy_mma(const void* q, const void* k, const void* 
  * out       device, out_dtype, [B][L][C], 16-byte aligned.
  * B >= 1, tokens_per_sample >= 0, C a multiple of 8 with 8 <= C <= 4096; eps >= 0.
  * With tokens_per_sample == 0 nothing is launched and the pointers are not used (they
- * may be NULL).
+ * may be NULL).  B * tokens_per_sample above (2^31 - 1) * 8 returns S3W_ERR_UNSUPPORTED.
+ * x_dtype, out_dtype: values of s3w_dtype, passed as int.
  */
 int adaln_residual_fwd(const void* x, int x_dtype, const float* residual,
                        const float* scale, const float* shift,
@@ -145,7 +147,7 @@ int s3w_poll_device_error(s3w_stream_t stream);
 
 /*
  * Time limit, in nanoseconds, of every bounded wait inside kernels launched after the
- * call (process-wide); returns the previous limit.  Default 1e9 (one second).  With 0, a
+ * call (process-wide, safe to call from any thread); returns the previous limit.  Default 1e9 (one second).  With 0, a
  * wait not satisfied at its first poll expires: the kernel unwinds early (copies drained,
  * tensor memory released), records S3W_ERR_DEVICE_TIMEOUT in the device error word and
  * leaves the CUDA context usable.  Meant for tests of that failure path.

@@ -3,11 +3,14 @@
 // failed check returns a status and enqueues nothing.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
+#include <climits>
 #include <cstdint>
 #include <mutex>
 
 #include "swin3d_wa.h"
+#include "swin3d_wa_baseline.h"
 #include "s3w_internal.h"
 
 namespace {
@@ -45,9 +48,10 @@ int device_state(DeviceState** out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Time limit of every bounded wait inside the kernels (nanoseconds); 1 s by default.
-long long g_wait_limit_ns = 1000000000ll;
-int g_test_stall = 0;
+// Time limit of every bounded wait inside the kernels (nanoseconds); 1 s by default.  Both
+// controls are process-wide and may be set from one host thread while another launches.
+std::atomic<long long> g_wait_limit_ns{1000000000ll};
+std::atomic<int> g_test_stall{0};
 
 }  // namespace
 
@@ -146,16 +150,10 @@ int make_geometry(const void* q, const void* k, const void* v, void* o, int B, i
 extern "C" {
 
 long long s3w_set_wait_limit_ns(long long ns) {
-  const long long prev = g_wait_limit_ns;
-  g_wait_limit_ns = ns < 0 ? 0 : ns;
-  return prev;
+  return g_wait_limit_ns.exchange(ns < 0 ? 0 : ns, std::memory_order_relaxed);
 }
 
-int s3w_set_test_stall(int on) {
-  const int prev = g_test_stall;
-  g_test_stall = on ? 1 : 0;
-  return prev;
-}
+int s3w_set_test_stall(int on) { return g_test_stall.exchange(on ? 1 : 0, std::memory_order_relaxed); }
 
 int swin3d_window_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int T, int H, int W,
                            int win_t, int win_h, int win_w, int shift_t, int shift_h, int shift_w, int heads,
@@ -168,8 +166,9 @@ int swin3d_window_attn_fwd(const void* q, const void* k, const void* v, void* o,
   DeviceState* ds = nullptr;
   rc = device_state(&ds);
   if (rc != S3W_OK) return rc;
-  g.test_stall = g_test_stall;
-  cudaError_t e = s3w::launch_window_attn_tc(g, q, k, v, o, out_dtype == S3W_F32, ds->err, g_wait_limit_ns,
+  g.test_stall = g_test_stall.load(std::memory_order_relaxed);
+  cudaError_t e = s3w::launch_window_attn_tc(g, q, k, v, o, out_dtype == S3W_F32, ds->err,
+                                             g_wait_limit_ns.load(std::memory_order_relaxed),
                                              ds->num_sms, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? S3W_OK : S3W_ERR_CUDA;
 }
@@ -202,13 +201,16 @@ int adaln_residual_fwd(const void* x, int x_dtype, const float* residual, const 
   if (!x || !residual || !scale || !shift || !out) return S3W_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(residual) || !aligned16(scale) || !aligned16(shift) || !aligned16(out))
     return S3W_ERR_MISALIGNED;
+  // One block of 8 rows each: the row count is bounded by the grid size limit (2^31 - 1
+  // blocks); checked before any product that could overflow.
+  constexpr long long kMaxRows = static_cast<long long>(INT32_MAX) * 8;
+  if (tokens_per_sample > kMaxRows / B) return S3W_ERR_UNSUPPORTED;
   // out may alias residual exactly; any other overlap with residual is rejected
   const long long n = static_cast<long long>(B) * tokens_per_sample * C;
   const char* r0 = reinterpret_cast<const char*>(residual);
   const char* o0 = reinterpret_cast<const char*>(out);
   const long long ob = out_dtype == S3W_F32 ? 4 : 2;
   if (o0 != r0 && o0 < r0 + n * 4 && r0 < o0 + n * ob) return S3W_ERR_INVALID_ARG;
-  if (B * tokens_per_sample > (1ll << 34)) return S3W_ERR_UNSUPPORTED;
   DeviceState* ds = nullptr;
   int rc = device_state(&ds);
   if (rc != S3W_OK) return rc;

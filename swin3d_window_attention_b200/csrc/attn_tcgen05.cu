@@ -64,16 +64,28 @@ constexpr int kTileBytes = kN * kRowBytes;          // 18432: one of Q / K / V
 constexpr int kStageBytes = 3 * kTileBytes;         // 55296
 constexpr int kMaskWords = 5;    // 144 key bits
 
-// Shared-memory map (offsets from a 1024-byte aligned base).  The tail P blocks only hold
-// 16 rows; the rows 16..127 their M = 128 descriptors also cover fall on the buffers that
-// follow (valid memory, results of those rows are never used).
+// Shared-memory map (offsets from a 1024-byte aligned base).
+// Once S = Q K^T of a tile has been computed, its Q and K tiles are dead: the P of the 128
+// main rows (36 KB, exactly the size of Q + K) is written over them, in the tile's own
+// stage, so P of the next tile never waits for the PV MMA of this one.  In a stage:
+//   P rows 0..127, keys 0..63    at +0      (128B swizzle, over Q)
+//   P rows 0..127, keys 64..127  at +16384  (128B swizzle, over Q rows 128.. and K)
+//   P rows 0..127, keys 128..143 at +32768  (32B swizzle, 4 KB, over K)
+// The 16 tail rows' P of stage s lives in a block of its own at s * kTailPBytes.  Their
+// M = 128 descriptors also cover rows 16..127, which fall on the blocks and stages that
+// follow (valid memory; the results of those rows are never used).
+constexpr int kTailPBytes = 5120;
 constexpr int OFF_P1B0 = 0;        // tail P rows 0..15, keys 0..63   (128B swizzle)
 constexpr int OFF_P1B1 = 2048;     // tail P rows 0..15, keys 64..127 (128B swizzle)
 constexpr int OFF_P1B2 = 4096;     // tail P rows 0..15, keys 128..143 (32B swizzle)
-constexpr int OFF_P0B0 = 5120;     // P rows 0..127, keys 0..63
-constexpr int OFF_P0B1 = OFF_P0B0 + 16384;
-constexpr int OFF_P0B2 = OFF_P0B1 + 16384;   // keys 128..143, 32B swizzle, 4 KB
-constexpr int OFF_STAGE = OFF_P0B2 + 4096;   // 41984 (1024-aligned)
+constexpr int OFF_P0B0 = 0;        // main P, relative to the stage
+constexpr int OFF_P0B1 = 16384;
+constexpr int OFF_P0B2 = 32768;
+static_assert(OFF_P0B2 + 128 * 32 <= 2 * kTileBytes, "main P fits over Q and K");
+constexpr int OFF_STAGE = kStages * kTailPBytes;   // 15360 (1024-aligned)
+static_assert(OFF_STAGE % 1024 == 0 && kStageBytes % 1024 == 0, "swizzle atoms stay aligned");
+static_assert((kStages - 1) * kTailPBytes + 128 * kRowBytes <= OFF_STAGE + kStageBytes,
+              "the tail P descriptors' unused rows stay inside the stages");
 // 16 key rows of bf16 ones in the V operand's layout: the PV MMA reads them as 16 more
 // output columns (through the descriptor's leading byte offset), so every such column of O
 // is the row sum of P as rounded to bf16, the exact normaliser of the P the MMA used.
@@ -102,9 +114,15 @@ struct SlotConst {
 };
 constexpr int OFF_SLOTC = OFF_TABLE + kStages * kTableBytes;
 constexpr int OFF_BARS = OFF_SLOTC + ((static_cast<int>(sizeof(SlotConst)) + 15) & ~15);
-// barriers: load[3] (TMA bytes), empty[3], table[3], s_full, s_empty, p_full, p_empty,
-// o_full, o_empty, drain, row max written[2] (one per key half), tail p_full, tail p_empty
-constexpr int kNumBars = 3 * kStages + 11;
+// barriers: load[3] (TMA bytes), empty[3], table[3], s_full, s_empty, p_full[2] (tile
+// parity), o_full, o_empty, drain, row max written[2][2] (tile parity, key half), tail
+// p_full[2] (tile parity).
+// P and the row maxima of a tile are handed over on barriers of the tile's parity.  Nothing
+// stops one softmax warp from arriving for tile t+1 before another has arrived for tile t,
+// or the tail warp from completing tile t+1's P before the MMA warp has waited for tile
+// t's; but no warp can arrive for tile t+2 before every waiter of tile t has passed (that
+// needs S(t+2), which the MMA warp issues only after its waits of tile t).
+constexpr int kNumBars = 3 * kStages + 13;
 // Row max of each key half of the main rows, exchanged between the two warps that share a
 // row: [tile parity][key half][row].
 constexpr int OFF_XCHG = OFF_BARS + kNumBars * 8;
@@ -183,16 +201,15 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
   auto table_bar = [&](int s) { return bar0 + 8u * (2 * kStages + s); };  // the stage's table written
   const uint32_t s_full = bar0 + 8u * (3 * kStages + 0);
   const uint32_t s_empty = bar0 + 8u * (3 * kStages + 1);
-  const uint32_t p_full = bar0 + 8u * (3 * kStages + 2);
-  const uint32_t p_empty = bar0 + 8u * (3 * kStages + 3);
+  auto p_full = [&](int par) { return bar0 + 8u * (3 * kStages + 2 + par); };   // main-row P of a tile
   const uint32_t o_full = bar0 + 8u * (3 * kStages + 4);
   const uint32_t o_empty = bar0 + 8u * (3 * kStages + 5);
   const uint32_t drain_bar = bar0 + 8u * (3 * kStages + 6);
-  auto xmax_bar = [&](int h) { return bar0 + 8u * (3 * kStages + 7 + h); };   // key half h wrote its row maxima
+  // key half h of a tile of parity par wrote its row maxima
+  auto xmax_bar = [&](int par, int h) { return bar0 + 8u * (3 * kStages + 7 + 2 * par + h); };
   // P of the main rows and of the tail rows are handed over separately, so the main rows'
-  // next P may be written as soon as their own PV MMAs have read it.
-  const uint32_t p_full_t = bar0 + 8u * (3 * kStages + 9);
-  const uint32_t p_empty_t = bar0 + 8u * (3 * kStages + 10);
+  // PV MMA need not wait for the tail warp.
+  auto p_full_t = [&](int par) { return bar0 + 8u * (3 * kStages + 11 + par); };
   float* xmax = reinterpret_cast<float*>(sm + OFF_XCHG);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sm + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
@@ -212,14 +229,13 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     }
     mbar_init(s_full, 1);
     mbar_init(s_empty, n_soft);
-    mbar_init(p_full, 256);
-    mbar_init(p_empty, 1);
-    mbar_init(p_full_t, 32);
-    mbar_init(p_empty_t, 1);
+    for (int par = 0; par < 2; ++par) mbar_init(p_full(par), 256);
+    for (int par = 0; par < 2; ++par) mbar_init(p_full_t(par), 32);
     mbar_init(o_full, 1);
     mbar_init(o_empty, n_soft);
     mbar_init(drain_bar, 1);
-    for (int h = 0; h < 2; ++h) mbar_init(xmax_bar(h), 128);
+    for (int par = 0; par < 2; ++par)
+      for (int h = 0; h < 2; ++h) mbar_init(xmax_bar(par, h), 128);
     *abort_flag = 0;
     *prod_stop = 0;
     fence_barrier_init();
@@ -440,9 +456,12 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     // V of stage 0; its second 64-column atom along N (leading byte offset) is the ones block
     const uint64_t dv0 = smem_desc(sb + OFF_STAGE + 2 * kTileBytes, OFF_ONES - (OFF_STAGE + 2 * kTileBytes), 1024,
                                    kSwizzle128B);
-    const uint64_t dp0 = desc_kmajor_sw128(sb + OFF_P0B0), dp0b = desc_kmajor_sw32(sb + OFF_P0B2);
+    // P of the main rows over Q and K of stage 0; the tail rows' P block of stage 0
+    const uint64_t dp0 = desc_kmajor_sw128(sb + OFF_STAGE + OFF_P0B0);
+    const uint64_t dp0b = desc_kmajor_sw32(sb + OFF_STAGE + OFF_P0B2);
     const uint64_t dp1 = desc_kmajor_sw128(sb + OFF_P1B0), dp1b = desc_kmajor_sw32(sb + OFF_P1B2);
     constexpr uint64_t kStageStep = kStageBytes >> 4;
+    constexpr uint64_t kTailStep = kTailPBytes >> 4;
     const uint32_t leader = lane == 0 ? 1u : 0u;
     bool issued = false;
     auto issue_s = [&](int jt) -> bool {   // S(jt) = Q K^T of the tile in stage jt % kStages
@@ -460,20 +479,20 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     };
     auto issue_pv = [&](int jt) -> bool {  // O(jt) = P V of the tile in stage jt % kStages
       const int s = jt % kStages;
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded(p_full, jt & 1, limit_ns))) return false;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(p_full(jt & 1), (jt >> 1) & 1, limit_ns))) return false;
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(o_empty, (jt & 1) ^ 1, limit_ns))) return false;
       tc_fence_after();
       // Moving V by d (bytes / 16) moves the ones block's leading offset by -d.
       const uint64_t dstage = s * kStageStep;
       const uint64_t vd = dv0 + dstage - (dstage << 16);
-      umma_chain_pv(tmem + TM_O0, dp0, vd, idesc_o, leader, dp0b, ((OFF_P0B1 - OFF_P0B0) >> 4) - 6);
-      umma_commit_leader(p_empty, leader);
+      umma_chain_pv(tmem + TM_O0, dp0 + dstage, vd, idesc_o, leader, dp0b + dstage, ((OFF_P0B1 - OFF_P0B0) >> 4) - 6);
       if (has_tail) {
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(p_full_t, jt & 1, limit_ns))) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(p_full_t(jt & 1), (jt >> 1) & 1, limit_ns))) return false;
         tc_fence_after();
-        umma_chain_pv(tmem + TM_O1, dp1, vd, idesc_o, leader, dp1b, ((OFF_P1B1 - OFF_P1B0) >> 4) - 6);
+        const uint64_t dtail = s * kTailStep;
+        umma_chain_pv(tmem + TM_O1, dp1 + dtail, vd, idesc_o, leader, dp1b + dtail,
+                      ((OFF_P1B1 - OFF_P1B0) >> 4) - 6);
       }
-      if (has_tail) umma_commit_leader(p_empty_t, leader);
       umma_commit_leader(o_full, leader);
       umma_commit_leader(empty_bar(s), leader);
       return true;
@@ -518,9 +537,11 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     const int half = is_tail ? (lane >> 4) : ((warp >> 2) & 1);
     const int row = is_tail ? 128 + (lane & 15) : (warp & 3) * 32 + lane;
     const int lrow = is_tail ? (lane & 15) : row;   // row inside its P blocks
-    const uint32_t pb0 = sb + (is_tail ? OFF_P1B0 : OFF_P0B0);
-    const uint32_t pb1 = sb + (is_tail ? OFF_P1B1 : OFF_P0B1);
-    const uint32_t pb2 = sb + (is_tail ? OFF_P1B2 : OFF_P0B2);
+    // P blocks of stage 0 (main rows: over that stage's Q and K; tail rows: its tail block)
+    const uint32_t pb0 = sb + (is_tail ? OFF_P1B0 : OFF_STAGE + OFF_P0B0);
+    const uint32_t pb1 = sb + (is_tail ? OFF_P1B1 : OFF_STAGE + OFF_P0B1);
+    const uint32_t pb2 = sb + (is_tail ? OFF_P1B2 : OFF_STAGE + OFF_P0B2);
+    const uint32_t p_stage_step = is_tail ? kTailPBytes : kStageBytes;
     const uint32_t s_base = is_tail ? tmem + TM_S1 : tmem + lane_base + TM_S0 + 8 * half;
     // O columns of a thread: groups of 16, 32m + 16h .. +15 (m < head_dim / 32); the main
     // rows take them with 32x32b at that column, the tail with 16x32bx2 at column 32m.
@@ -554,10 +575,10 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         __nv_bfloat16* dst =
             static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD + col;
         uint4 u;
-        u.x = pack_bf16x2_int(vals[0] * scl, vals[1] * scl);
-        u.y = pack_bf16x2_int(vals[2] * scl, vals[3] * scl);
-        u.z = pack_bf16x2_int(vals[4] * scl, vals[5] * scl);
-        u.w = pack_bf16x2_int(vals[6] * scl, vals[7] * scl);
+        u.x = pack_bf16x2(vals[0] * scl, vals[1] * scl);
+        u.y = pack_bf16x2(vals[2] * scl, vals[3] * scl);
+        u.z = pack_bf16x2(vals[4] * scl, vals[5] * scl);
+        u.w = pack_bf16x2(vals[6] * scl, vals[7] * scl);
         *reinterpret_cast<uint4*>(dst) = u;
       }
     };
@@ -596,7 +617,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
             if (g.o_rows_32b) {   // 16 bf16 = one 32-byte store
               uint32_t u[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) u[e] = pack_bf16x2_int(ov[16 * m + 2 * e] * inv, ov[16 * m + 2 * e + 1] * inv);
+              for (int e = 0; e < 8; ++e) u[e] = pack_bf16x2(ov[16 * m + 2 * e] * inv, ov[16 * m + 2 * e + 1] * inv);
               st_global_v8(static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tok) * g.o_stride + head * HD + col, u);
               continue;
             }
@@ -640,7 +661,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       return fmaxf(a, b);
     };
     // exp2 and P (bf16) into the P blocks.  The row sum comes out of the PV MMA.
-    auto row_exp = [&](const float (&x)[72], float m) {
+    auto row_exp = [&](const float (&x)[72], float m, uint32_t pofs) {
       const float2 cc = make_float2(c, c), nm = make_float2(-m * c, -m * c);
       const uint32_t rsw = lrow & 7;
       const uint32_t row128 = static_cast<uint32_t>(lrow) * 128, row32 = static_cast<uint32_t>(lrow) * 32;
@@ -661,9 +682,9 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         const int g8 = 2 * k + half;   // 16-byte chunk of P along the keys
         uint32_t addr;
         if (k < 8)
-          addr = (k < 4 ? pb0 : pb1) + row128 + ((((g8 & 7) ^ rsw)) << 4);
+          addr = (k < 4 ? pb0 : pb1) + pofs + row128 + ((((g8 & 7) ^ rsw)) << 4);
         else
-          addr = pb2 + row32 + (((g8 - 16) ^ sw32) << 4);
+          addr = pb2 + pofs + row32 + (((g8 - 16) ^ sw32) << 4);
         asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(pk[0]), "r"(pk[1]), "r"(pk[2]),
                      "r"(pk[3])
                      : "memory");
@@ -709,8 +730,8 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         float mrow;
         if (!is_tail) {
           xmax[(par * 2 + half) * 128 + row] = mh;
-          mbar_arrive(xmax_bar(half));
-          ok = mbar_wait_bounded(xmax_bar(half ^ 1), par, limit_ns);
+          mbar_arrive(xmax_bar(par, half));
+          ok = mbar_wait_bounded(xmax_bar(par, half ^ 1), (it >> 1) & 1, limit_ns);
           if (!__all_sync(0xffffffffu, ok)) {
             aborted = true;
             break;
@@ -720,15 +741,11 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
           mrow = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 16));
         }
         if (mrow == -INFINITY) mrow = 0.f;
-        // P may only be overwritten once the previous tile's PV MMA has consumed it.
-        ok = mbar_wait_bounded(is_tail ? p_empty_t : p_empty, par ^ 1, limit_ns);
-        if (!__all_sync(0xffffffffu, ok)) {
-          aborted = true;
-          break;
-        }
-        row_exp(x, mrow);
+        // P goes to the tile's own stage (over its Q and K, consumed by S, which s_full
+        // guaranteed above): no wait for the previous tile's PV.
+        row_exp(x, mrow, static_cast<uint32_t>(s) * p_stage_step);
         fence_proxy_async_smem();
-        mbar_arrive(is_tail ? p_full_t : p_full);
+        mbar_arrive(is_tail ? p_full_t(par) : p_full(par));
       }
       if (have_prev) {
         if (!epilogue(prev_it, prev_head, prev_tok)) {

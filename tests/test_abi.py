@@ -89,6 +89,8 @@ def _adaln(**over):
     (dict(C=8192), api.S3W_ERR_UNSUPPORTED),
     (dict(sc=FAKE + 4), api.S3W_ERR_MISALIGNED),
     (dict(out=FAKE + 16 * 512), api.S3W_ERR_INVALID_ARG),   # partial overlap with residual
+    (dict(L=(2 ** 31 - 1) * 8 + 1), api.S3W_ERR_UNSUPPORTED),   # more row blocks than a grid holds
+    (dict(B=4, L=2 ** 62), api.S3W_ERR_UNSUPPORTED),             # B * L * C would overflow int64
 ])
 def test_adaln_rejects_bad_arguments_on_host(over, expect):
     # the overlap case keeps out != residual while the two ranges intersect

@@ -1,8 +1,11 @@
 """The six-block encoder stack at full size: B=4, 4 x 180 x 360, 8 heads x 64; block k runs
 attention on fresh seeded Q/K/V with the shift alternating (0,0,0), (1,3,6), ..., then AdaLN
 (fp32 out) on its output into the fp32 residual stream, which chains through the six blocks.
-Checked on sampled windows: each block's attention against the oracle, and the residual
-stream at the sampled tokens against the oracle's own chain (attention -> AdaLN, six times).
+Checked on sampled windows: each block's attention against the oracle; each block's AdaLN
+at max-abs 1e-5 against the oracle's AdaLN fed the GPU's own bf16 attention output and the
+GPU's residual before the block (so the AdaLN bar is the FP32 one, independent of the
+attention error); and the residual stream at the sampled tokens against the oracle's own
+chain (attention -> AdaLN, six times).
 
 Tolerance of the chained residual: each block adds y (1 + scale) + shift, y the normalised
 attention output.  The attention output carries the attention tolerance (max-abs 1e-2 at
@@ -19,7 +22,7 @@ import oracle
 import swin3d_window_attention_b200 as s3w
 from swin3d_window_attention_b200 import inputs
 
-from .helpers import ATTN_MAX_ABS, ATTN_REL_L2, attn_errors, edge_window_ids, window_geometry
+from .helpers import ADALN_F32_MAX_ABS, ATTN_MAX_ABS, ATTN_REL_L2, attn_errors, edge_window_ids, window_geometry
 
 pytestmark = pytest.mark.gpu
 
@@ -58,6 +61,11 @@ def test_encoder_stack_six_blocks_sampled(cuda_ok):
         if k == 0:
             res_host0 = res.cpu().numpy()
         s3w.swin3d_window_attn_fwd(q, kk, v, o, HEADS, HD, WINDOW, shift)
+        torch.cuda.synchronize()
+        if toks is not None:
+            toks_d = torch.from_numpy(toks).to(dev)
+            res_before = res.view(B * L, C)[toks_d].cpu().numpy()
+            x_gpu = inputs.torch_bf16_to_bits(o.view(B * L, C)[toks_d])
         s3w.adaln_residual_fwd(o.view(B, L, C), res, scale, shift_v, res, eps=1e-5)
         torch.cuda.synchronize()
         assert s3w.poll_device_error() == 0
@@ -66,6 +74,19 @@ def test_encoder_stack_six_blocks_sampled(cuda_ok):
             _, tok0, _ = oracle.window_attn(qb, kb, vb, HEADS, HD, WINDOW, shift, window_ids=ids0)
             toks = np.unique(tok0[tok0 >= 0])
             ref_res = res_host0.reshape(B * L, C)[toks].astype(np.float64)
+        if k == 0:
+            toks_d = torch.from_numpy(toks).to(dev)
+            res_before = res_host0.reshape(B * L, C)[toks]
+            x_gpu = inputs.torch_bf16_to_bits(o.view(B * L, C)[toks_d])
+        # this block's AdaLN on the GPU's own attention output and residual: the FP32 bar
+        sc_h, sh_h = scale.cpu().numpy(), shift_v.cpu().numpy()
+        samp = toks // L
+        res_after = res.view(B * L, C)[toks_d].cpu().numpy()
+        for b in np.unique(samp):
+            sel = samp == b
+            want = oracle.adaln(x_gpu[sel][None], res_before[sel][None], sc_h[b:b + 1], sh_h[b:b + 1])[0]
+            err = float(np.abs(res_after[sel] - want).max())
+            assert err <= ADALN_F32_MAX_ABS, (k, int(b), err)
         ids = windows_of_tokens(toks, shift)
         out, tok, _ = oracle.window_attn(qb, kb, vb, HEADS, HD, WINDOW, shift, window_ids=ids)
         real = tok >= 0
@@ -76,8 +97,6 @@ def test_encoder_stack_six_blocks_sampled(cuda_ok):
         # the oracle's chain at the sampled tokens: AdaLN of the oracle's attention output
         att = dict(zip(tok[real].tolist(), out[real]))
         x = np.stack([att[int(t)] for t in toks])
-        sc_h, sh_h = scale.cpu().numpy(), shift_v.cpu().numpy()
-        samp = toks // L
         new = np.empty_like(ref_res)
         for b in np.unique(samp):
             sel = samp == b
