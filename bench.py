@@ -66,7 +66,7 @@ WORKLOAD = ("Aurora 0.25deg encoder stage 1: B=1, grid T4xH180xW360, C=512 (8 he
             "per step: attn shift (0,0,0) + AdaLN fp32-out, attn shift (1,3,6) + AdaLN fp32-out")
 PROFILE = os.path.join("profiles", "window_attn_tc_stage1.json")
 KERNEL_SOURCES = [os.path.join("swin3d_window_attention_b200", "csrc", f)
-                  for f in ("attn_tcgen05.cu", "sm100_ptx.cuh", "s3w_common.cuh")]
+                  for f in ("attn_tcgen05.cu", "attn_common.cuh", "sm100_ptx.cuh", "s3w_common.cuh")]
 
 
 def geometry(w):
@@ -77,10 +77,10 @@ def geometry(w):
     return C, tokens, windows
 
 
-def attn_bytes(w, o_bytes=2):
-    """Read Q, K, V once and write O once (bf16 in): padding and the shift never touch HBM."""
+def attn_bytes(w, o_bytes=2, in_bytes=2):
+    """Read Q, K, V once and write O once: padding and the shift never touch HBM."""
     C, tokens, _ = geometry(w)
-    return (3 * 2 + o_bytes) * tokens * C
+    return (3 * in_bytes + o_bytes) * tokens * C
 
 
 def attn_flops(w):
@@ -253,6 +253,14 @@ def device_qkv(torch, w, dev, base):
     return [inputs.normal_bf16_torch(shape, dev, tensor_index=base + j) for j in range(3)]
 
 
+def inputs_f32(torch, w, dev, index):
+    """A seeded fp32 grid tensor of a workload (the TF32_ACC_FP32 mode's inputs), on the device."""
+    from swin3d_window_attention_b200 import inputs
+
+    C, tokens, _ = geometry(w)
+    return inputs.normal_f32_torch(tokens * C, dev, tensor_index=index).reshape(w["B"], w["T"], w["H"], w["W"], C)
+
+
 def device_film(torch, w, dev, base, sigma):
     from swin3d_window_attention_b200 import inputs
 
@@ -327,6 +335,23 @@ def bench_configs(torch, s3w, dev, stream, peaks, reps):
         "attn": {**launch_stats(ms_a), "bytes": attn_bytes(w), "flops": attn_flops(w),
                  "windows_per_s": windows / (a_med * 1e-3),
                  "roofline": roofline(attn_bytes(w), attn_flops(w), a_med, peaks)}}
+    del q, k, v, o
+
+    # TF32_ACC_FP32 mode on the stage-1 grid: fp32 Q/K/V in, fp32 O out
+    w = WORKLOADS["stage1"]
+    C, tokens, windows = geometry(w)
+    q, k, v = (inputs_f32(torch, w, dev, 940 + j) for j in range(3))
+    o = torch.empty_like(q)
+    ms_a = timed(torch, stream, lambda: s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTED),
+                 reps)
+    launches += len(ms_a)
+    a_med = statistics.median(ms_a)
+    nbytes = attn_bytes(w, o_bytes=4, in_bytes=4)
+    out["stage1_tf32"] = {
+        "grid": "B=1 T4xH180xW360, 8 heads x 64, shift (1,3,6), 1800 windows; fp32 Q/K/V/O, TF32 MMAs (TF32_ACC_FP32)",
+        "attn": {**launch_stats(ms_a), "bytes": nbytes, "flops": attn_flops(w), "windows_per_s": windows / (a_med * 1e-3),
+                 "roofline": roofline(nbytes, attn_flops(w), a_med,
+                                      {**peaks, "bf16_tflops": peaks["bf16_tflops"] / 2})}}
     del q, k, v, o
 
     # six-block stage-1 stack at B = 4: fresh Q/K/V per block, fp32 residual chained

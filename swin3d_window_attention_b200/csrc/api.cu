@@ -108,10 +108,10 @@ int make_geometry(const void* q, const void* k, const void* v, void* o, int B, i
   const long long N = static_cast<long long>(win_t) * win_h * win_w;
   if (N > 144) return S3W_ERR_UNSUPPORTED;
   if (head_dim != 32 && head_dim != 64) return S3W_ERR_UNSUPPORTED;
-  if (in_dtype != S3W_BF16) return S3W_ERR_UNSUPPORTED;
+  const int ib = in_dtype == S3W_F32 ? 4 : 2;
   const int ob = out_dtype == S3W_F32 ? 4 : 2;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return S3W_ERR_MISALIGNED;
-  if ((qkv_token_stride * 2) % 16 != 0 || (o_token_stride * ob) % 16 != 0) return S3W_ERR_MISALIGNED;
+  if ((qkv_token_stride * ib) % 16 != 0 || (o_token_stride * ob) % 16 != 0) return S3W_ERR_MISALIGNED;
   // grid token indices are 32-bit inside the kernels; padded sizes must stay in int range
   if (static_cast<long long>(B) * T * H * W > INT32_MAX) return S3W_ERR_UNSUPPORTED;
   const long long Pt = (T + win_t - 1) / win_t * static_cast<long long>(win_t);
@@ -167,9 +167,11 @@ int swin3d_window_attn_fwd(const void* q, const void* k, const void* v, void* o,
   rc = device_state(&ds);
   if (rc != S3W_OK) return rc;
   g.test_stall = g_test_stall.load(std::memory_order_relaxed);
-  cudaError_t e = s3w::launch_window_attn_tc(g, q, k, v, o, out_dtype == S3W_F32, ds->err,
-                                             g_wait_limit_ns.load(std::memory_order_relaxed),
-                                             ds->num_sms, reinterpret_cast<cudaStream_t>(stream));
+  const long long limit = g_wait_limit_ns.load(std::memory_order_relaxed);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = in_dtype == S3W_F32
+                      ? s3w::launch_window_attn_tf32(g, q, k, v, o, out_dtype == S3W_F32, ds->err, limit, ds->num_sms, st)
+                      : s3w::launch_window_attn_tc(g, q, k, v, o, out_dtype == S3W_F32, ds->err, limit, ds->num_sms, st);
   return e == cudaSuccess ? S3W_OK : S3W_ERR_CUDA;
 }
 
@@ -181,6 +183,7 @@ int swin3d_window_attn_fwd_legacy_mma(const void* q, const void* k, const void* 
   int rc = make_geometry(q, k, v, o, B, T, H, W, win_t, win_h, win_w, shift_t, shift_h, shift_w, heads, head_dim,
                          qkv_token_stride, o_token_stride, scale, in_dtype, out_dtype, &g);
   if (rc != S3W_OK) return rc;
+  if (in_dtype != S3W_BF16) return S3W_ERR_UNSUPPORTED;   // the baseline path is BF16 only
   if (g.windows * heads > (1ll << 31) - 1) return S3W_ERR_UNSUPPORTED;
   DeviceState* ds = nullptr;
   rc = device_state(&ds);

@@ -45,10 +45,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
-#include <cudaTypedefs.h>
 
-#include <mutex>
-
+#include "attn_common.cuh"
 #include "s3w_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -56,13 +54,11 @@ namespace s3w {
 namespace {
 
 using namespace sm100;
+using namespace attn;
 
-constexpr int kN = 144;          // slots per window tile (queries and keys)
 constexpr int kStages = 3;
-constexpr int kRowBytes = 128;   // one token row of one head in shared memory (swizzle width)
-constexpr int kTileBytes = kN * kRowBytes;          // 18432: one of Q / K / V
+constexpr int kTileBytes = kChunkTileBytes;         // 18432: one of Q / K / V (one head = 128 B rows)
 constexpr int kStageBytes = 3 * kTileBytes;         // 55296
-constexpr int kMaskWords = 5;    // 144 key bits
 
 // Shared-memory map (offsets from a 1024-byte aligned base).
 // Once S = Q K^T of a tile has been computed, its Q and K tiles are dead: the P of the 128
@@ -93,27 +89,8 @@ constexpr int OFF_ONES = OFF_STAGE + kStages * kStageBytes;
 constexpr int kOnesBytes = 16 * kRowBytes;
 constexpr int OFF_TABLE = OFF_ONES + kOnesBytes;
 
-// Per tile: grid token of every slot (-1 = padded), which slots are real, and along which
-// shifted axes the window is the last one (where Swin's mask splits it in two regions).
-struct Table {
-  int tok[kN];
-  uint32_t real[kMaskWords];
-  uint32_t last;
-  // The key mask a softmax thread applies, per (region combination of the query, key half):
-  // bytes 0..8 = key groups 2k + half (k = 0..8), one bit per key; w = 1 if any key is masked.
-  uint4 maskq[16];
-};
-constexpr int kTableBytes = (static_cast<int>(sizeof(Table)) + 15) & ~15;
-// Per CTA, the same for every tile: the (t, h, w) offset of each slot inside the window
-// and, per axis, the slots of the wrapped-around part (offset >= window - shift).  A query
-// in the last window along a shifted axis may only see keys on its own side of that split.
-struct SlotConst {
-  uint32_t coord[kN];                 // rt | rh << 8 | rw << 16
-  uint32_t hi[3][kMaskWords];
-  uint32_t all[kMaskWords];           // slots < N
-};
 constexpr int OFF_SLOTC = OFF_TABLE + kStages * kTableBytes;
-constexpr int OFF_BARS = OFF_SLOTC + ((static_cast<int>(sizeof(SlotConst)) + 15) & ~15);
+constexpr int OFF_BARS = OFF_SLOTC + kSlotConstBytes;
 // barriers: load[3] (TMA bytes), empty[3], table[3], s_full, s_empty, p_full[2] (tile
 // parity), o_full, o_empty, drain, row max written[2][2] (tile parity, key half), tail
 // p_full[2] (tile parity).
@@ -139,17 +116,15 @@ constexpr uint32_t TM_S0 = 0, TM_S1 = 160, TM_O0 = 320, TM_O1 = 416;
 constexpr uint32_t kOnesCol = 64;
 constexpr uint32_t kTmemCols = 512;
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
 constexpr int kMainWarps = 8;          // rows 0..127: warp w holds lanes 32 (w % 4) .., keys 72 (w / 4) ..
 constexpr int kTailWarp = 8;           // tail rows 128..143 (TMEM lane quarter 0, like warp 0)
 constexpr int kMmaWarp = 9;
 constexpr int kTmaWarp = 10;
 constexpr int kFirstProducerWarp = 11;
 constexpr int kProducerThreads = 32;   // table writer (warp 11)
-
-__device__ __forceinline__ void named_bar_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
+constexpr int kFirstEpiWarp = 12;      // warps 12..15: O of TMEM lane quarter warp % 4 to global memory
+constexpr int kEpiThreads = 128;
 
 // Operand descriptors.  K-major 128B swizzle: 8-row x 128-byte atoms, 1024 bytes apart.
 // K-major 32B swizzle: 8-row x 32-byte atoms, 256 bytes apart.  MN-major 128B swizzle (V,
@@ -157,35 +132,6 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
 // K; the leading byte offset is the distance to the next 64 elements along N.
 __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t addr) { return smem_desc(addr, 16, 1024, kSwizzle128B); }
 __device__ __forceinline__ uint64_t desc_kmajor_sw32(uint32_t addr) { return smem_desc(addr, 16, 256, kSwizzle32B); }
-
-// Keys visible to a query in slot r: real slots, restricted on every axis where the window
-// is the last one of a shifted axis to the query's side of the wrap-around split.
-// hi_bits: bit a set iff slot r is in the wrapped-around part of axis a.
-__device__ __forceinline__ void build_mask(const Table& tb, const SlotConst& sc, uint32_t last, uint32_t hi_bits,
-                                           uint32_t (&m)[kMaskWords]) {
-#pragma unroll
-  for (int w = 0; w < kMaskWords; ++w) {
-    uint32_t x = tb.real[w];
-#pragma unroll
-    for (int a = 0; a < 3; ++a)
-      if ((last >> a) & 1u) x &= ((hi_bits >> a) & 1u) ? sc.hi[a][w] : (sc.all[w] & ~sc.hi[a][w]);
-    m[w] = x;
-  }
-}
-
-// Tensor maps of Q, K and V over the grid as a 5-D tensor (channel, W, H, T, sample),
-// one per box shape.  A window is loaded one T-slab (win_h x win_w tokens) at a time:
-// a whole slab in one box where the window does not wrap around a seam; a slab cut at
-// the H seam in two boxes (win_h - shift_h rows, then shift_h rows); and where the window
-// wraps around the W seam, one box per (t, h) run cut in two (win_w - shift_w, then
-// shift_w tokens), since a box narrower than the window would pack its rows too densely.
-// Box width is 64 channels (one head of 64; for head_dim 32 the head plus its
-// neighbour, 128 bytes either way), 128-byte swizzle, out-of-bounds elements (padding)
-// read as zero.
-enum : int { kBoxSlab = 0, kBoxSeamH1 = 1, kBoxSeamH2 = 2, kBoxSeamW1 = 3, kBoxSeamW2 = 4, kBoxShapes = 5 };
-struct TmaMaps {
-  CUtensorMap m[3][kBoxShapes];   // [tensor q/k/v][box shape]
-};
 
 template <int HD, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -224,7 +170,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(load_bar(s), 1);                        // the TMA thread's expect_tx arrival + bytes
-      mbar_init(empty_bar(s), 1 + n_soft);              // PV commit + every softmax thread (table read)
+      mbar_init(empty_bar(s), 1 + n_soft + kEpiThreads);  // PV commit + softmax and epilogue threads (table read)
       mbar_init(table_bar(s), kProducerThreads);
     }
     mbar_init(s_full, 1);
@@ -232,7 +178,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     for (int par = 0; par < 2; ++par) mbar_init(p_full(par), 256);
     for (int par = 0; par < 2; ++par) mbar_init(p_full_t(par), 32);
     mbar_init(o_full, 1);
-    mbar_init(o_empty, n_soft);
+    mbar_init(o_empty, kEpiThreads);
     mbar_init(drain_bar, 1);
     for (int par = 0; par < 2; ++par)
       for (int h = 0; h < 2; ++h) mbar_init(xmax_bar(par, h), 128);
@@ -242,29 +188,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     fence_proxy_async_smem();
   }
   SlotConst* slotc = reinterpret_cast<SlotConst*>(sm + OFF_SLOTC);
-  {
-    auto split_at = [&](int a) { return a == 0 ? g.wt - g.st : (a == 1 ? g.wh - g.sh : g.ww - g.sw); };
-    auto slot_off = [&](int r, int a) {   // offset of slot r along axis a
-      return a == 2 ? r % g.ww : (a == 1 ? (r / g.ww) % g.wh : r / (g.ww * g.wh));
-    };
-    if (tid < kN) slotc->coord[tid] = tid < g.N ? (slot_off(tid, 0) | slot_off(tid, 1) << 8 | slot_off(tid, 2) << 16) : 0u;
-    if (tid >= 160 && tid < 160 + 3 * kMaskWords) {
-      const int a = (tid - 160) / kMaskWords, w = (tid - 160) % kMaskWords;
-      uint32_t bits = 0;
-      for (int b = 0; b < 32; ++b) {
-        const int r = 32 * w + b;
-        if (r < g.N && slot_off(r, a) >= split_at(a)) bits |= 1u << b;
-      }
-      slotc->hi[a][w] = bits;
-    }
-    if (tid >= 192 && tid < 192 + kMaskWords) {
-      const int w = tid - 192;
-      uint32_t bits = 0;
-      for (int b = 0; b < 32; ++b)
-        if (32 * w + b < g.N) bits |= 1u << b;
-      slotc->all[w] = bits;
-    }
-  }
+  init_slot_consts(g, slotc, tid);
   for (int i = tid; i < kOnesBytes / 16; i += kThreads)   // bf16 1.0 = 0x3f80
     *reinterpret_cast<uint4*>(sm + OFF_ONES + 16 * i) = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);
   fence_proxy_async_smem();
@@ -289,157 +213,13 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // Window coordinates of a tile (32-bit: the tile count is checked on the host) and the
-  // shifted padded coordinate of its slot offset 0 plus the shift: slot (rt, rh, rw) holds
-  // the original coordinate (base + offset) mod P on each axis.
-  struct TileCoord {
-    int head, bsmp, itw, ih, iw, bt, bh, bw;
-  };
-  auto tile_coord = [&](long long tile) {
-    TileCoord tc;
-    const int t32 = static_cast<int>(tile);
-    const int win = fdiv(t32, g.div_heads);
-    tc.head = t32 - win * g.heads;
-    tc.bsmp = fdiv(win, g.div_per_sample);
-    const int rem = win - tc.bsmp * (g.nwt * g.nwh * g.nww);
-    const int q1 = fdiv(rem, g.div_nww);
-    tc.iw = rem - q1 * g.nww;
-    tc.itw = fdiv(q1, g.div_nwh);
-    tc.ih = q1 - tc.itw * g.nwh;
-    tc.bt = tc.itw * g.wt + g.st;
-    tc.bh = tc.ih * g.wh + g.sh;
-    tc.bw = tc.iw * g.ww + g.sw;
-    return tc;
-  };
-
+  const Ring ring{sb + OFF_STAGE, load_bar(0), empty_bar(0), table_bar(0)};
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------------ TMA loads
-    // One thread loads each tile's Q, K and V: one box per (t, h) run of window tokens per
-    // tensor (two where the run wraps around the W seam), straight from grid layout into
-    // the stage; padded coordinates are out of bounds and read as zero.
-    if (lane == 0) {
-#pragma unroll
-      for (int a = 0; a < 3; ++a)
-#pragma unroll
-        for (int b = 0; b < kBoxShapes; ++b) prefetch_tmap(&maps.m[a][b]);
-      const uint32_t tile_bytes = static_cast<uint32_t>(3 * g.N * kRowBytes);
-      const uint32_t run_bytes = static_cast<uint32_t>(g.ww) * kRowBytes;
-      int it = 0;
-      for (long long tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
-        const int s = it % kStages;
-        if (*abort_flag) break;
-        if (!mbar_wait_bounded(empty_bar(s), ((it / kStages) & 1) ^ 1, limit_ns)) {
-          record_error(err, kStatusTimeout);
-          *abort_flag = 1;
-          break;
-        }
-        const TileCoord tc = tile_coord(tile);
-        const uint32_t stage = sb + OFF_STAGE + s * kStageBytes;
-        const uint32_t bar = load_bar(s);
-        mbar_arrive_expect_tx(bar, tile_bytes);
-        // The window's first slot sits at (bt, bh, bw), inside the padded grid on every
-        // axis; a window wraps around an axis's seam only if it is the last one along a
-        // shifted axis.
-        const bool wrap_w = tc.bw + g.ww > g.Pw;
-        const bool wrap_h = tc.bh + g.wh > g.Ph;
-        const int n1w = g.Pw - tc.bw, n1h = g.Ph - tc.bh;
-        const int c0 = tc.head * HD;
-#pragma unroll 1
-        for (int rt = 0; rt < g.wt; ++rt) {
-          int t = tc.bt + rt;
-          t -= t >= g.Pt ? g.Pt : 0;
-          const uint32_t slab = stage + rt * g.wh * run_bytes;
-          if (!wrap_w) {
-#pragma unroll 1
-            for (int tsr = 0; tsr < 3; ++tsr) {
-              const uint32_t d = slab + tsr * kTileBytes;
-              if (!wrap_h) {
-                tma_load_5d(d, &maps.m[tsr][kBoxSlab], c0, tc.bw, tc.bh, t, tc.bsmp, bar);
-              } else {
-                tma_load_5d(d, &maps.m[tsr][kBoxSeamH1], c0, tc.bw, tc.bh, t, tc.bsmp, bar);
-                tma_load_5d(d + n1h * run_bytes, &maps.m[tsr][kBoxSeamH2], c0, tc.bw, 0, t, tc.bsmp, bar);
-              }
-            }
-          } else {
-            int h = tc.bh;
-#pragma unroll 1
-            for (int rh = 0; rh < g.wh; ++rh) {
-              const uint32_t dst = slab + rh * run_bytes;
-#pragma unroll 1
-              for (int tsr = 0; tsr < 3; ++tsr) {
-                const uint32_t d = dst + tsr * kTileBytes;
-                tma_load_5d(d, &maps.m[tsr][kBoxSeamW1], c0, tc.bw, h, t, tc.bsmp, bar);
-                tma_load_5d(d + n1w * kRowBytes, &maps.m[tsr][kBoxSeamW2], c0, 0, h, t, tc.bsmp, bar);
-              }
-              ++h;
-              h -= h >= g.Ph ? g.Ph : 0;
-            }
-          }
-        }
-      }
-      // Before the CTA may exit, every load issued must have landed.  On the normal path
-      // the MMA warp has consumed them all; after an abort, wait (bounded, independently of
-      // the test limit) for the last stages issued.
-      for (int j = it > kStages ? it - kStages : 0; j < it; ++j)
-        if (!mbar_wait_bounded(load_bar(j % kStages), (j / kStages) & 1, 2000000000ull))
-          record_error(err, kStatusTimeout);
-    }
-  } else if (warp >= kFirstProducerWarp) {
+    if (lane == 0) tma_loader<1, 64, kStages, kStageBytes>(g, maps, ring, HD, num_tiles, abort_flag, err, limit_ns);
+  } else if (warp == kFirstProducerWarp) {
     // ------------------------------------------------------------------ tile tables
-    const int p = tid - kFirstProducerWarp * 32;
-    int it = 0;
-    for (long long tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
-      const int s = it % kStages;
-      if (p == 0) {
-        const bool ok = mbar_wait_bounded(empty_bar(s), ((it / kStages) & 1) ^ 1, limit_ns);
-        if (!ok) {
-          record_error(err, kStatusTimeout);
-          *abort_flag = 1;
-        }
-        *prod_stop = (!ok || *abort_flag) ? 1 : 0;
-      }
-      named_bar_sync(1, kProducerThreads);
-      if (*prod_stop) break;
-      const TileCoord tc = tile_coord(tile);
-      auto resolve = [&](int r) -> int {   // grid token of slot r, -1 if padded
-        if (r >= g.N) return -1;
-        const uint32_t cd = slotc->coord[r];
-        int t = tc.bt + static_cast<int>(cd & 0xffu);
-        int h = tc.bh + static_cast<int>((cd >> 8) & 0xffu);
-        int w = tc.bw + static_cast<int>(cd >> 16);
-        t -= t >= g.Pt ? g.Pt : 0;
-        h -= h >= g.Ph ? g.Ph : 0;
-        w -= w >= g.Pw ? g.Pw : 0;
-        if (t >= g.T || h >= g.H || w >= g.W) return -1;
-        return ((tc.bsmp * g.T + t) * g.H + h) * g.W + w;
-      };
-      Table& tb = tables[s];
-#pragma unroll 1
-      for (int r = p; r < kN; r += kProducerThreads) tb.tok[r] = resolve(r);
-      if (p == 0)
-        tb.last = ((tc.itw == g.nwt - 1 && g.st > 0) ? 1u : 0u) | ((tc.ih == g.nwh - 1 && g.sh > 0) ? 2u : 0u) |
-                  ((tc.iw == g.nww - 1 && g.sw > 0) ? 4u : 0u);
-#pragma unroll 1
-      for (int wd = p >> 5; wd < kMaskWords; wd += kProducerThreads / 32) {
-        const int r = 32 * wd + lane;
-        const unsigned m = __ballot_sync(0xffffffffu, r < kN && resolve(r) >= 0);
-        if (lane == 0) tb.real[wd] = m;
-      }
-      __syncwarp();
-      if (lane < 16) {
-        // combination c of the query's wrapped-around sides (bit a: axis a), key half h
-        const uint32_t c = static_cast<uint32_t>(lane) >> 1, h = static_cast<uint32_t>(lane) & 1u;
-        uint32_t mw[kMaskWords];
-        build_mask(tb, *slotc, tb.last, c, mw);
-        uint32_t kb[9];
-#pragma unroll
-        for (int k = 0; k < 9; ++k) kb[k] = (mw[k >> 1] >> (16 * (k & 1) + 8 * h)) & 0xffu;
-        const uint32_t all = kb[0] & kb[1] & kb[2] & kb[3] & kb[4] & kb[5] & kb[6] & kb[7] & kb[8];
-        tb.maskq[lane] = make_uint4(kb[0] | kb[1] << 8 | kb[2] << 16 | kb[3] << 24,
-                                    kb[4] | kb[5] << 8 | kb[6] << 16 | kb[7] << 24, kb[8], all == 0xffu ? 0u : 1u);
-      }
-      mbar_arrive(table_bar(s));   // table written (release)
-    }
+    table_writer<kStages>(g, tables, slotc, ring, num_tiles, abort_flag, prod_stop, err, limit_ns, lane);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     // Issue order: S(t+1) goes out as soon as tile t+1 is loaded and S(t) has been read
@@ -521,16 +301,117 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       if (!mbar_wait_bounded(drain_bar, 0, 2000000000ull)) record_error(err, kStatusTimeout);
     }
     __syncwarp();
+  } else if (warp >= kFirstEpiWarp) {
+    // ------------------------------------------------------------------ epilogue
+    // Warp 12 + q reads TMEM lane quarter q of O0 (query rows 32q .. 32q + 31, one row per
+    // thread: the head's columns and the row sum, an MMA output column), releases O, scales
+    // by 1/rowsum and stores each row to its query's original grid position; padded slots are
+    // dropped.  Warp 12 also takes the 16 tail rows of O1 (TMEM lanes 0..15), half a row per
+    // thread (16x32bx2 shape).  The grid tokens are read from the tile's table before the
+    // stage is released.
+    const int q = warp - kFirstEpiWarp;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const int row = q * 32 + lane;
+    const bool do_tail = has_tail && q == 0;
+    const int thalf = lane >> 4;
+    auto store16 = [&](int tk, int head, int col, const float* vals, float scl) {
+      // 16 consecutive outputs of one row starting at column `col`
+      if constexpr (OUT_F32) {
+        float* dst = static_cast<float*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD + col;
+#pragma unroll
+        for (int h8 = 0; h8 < 16; h8 += 8) {
+          if (g.o_rows_32b) {
+            uint32_t u[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) u[e] = __float_as_uint(vals[h8 + e] * scl);
+            st_global_v8(dst + h8, u);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; e += 4)
+              *reinterpret_cast<float4*>(dst + h8 + e) =
+                  make_float4(vals[h8 + e] * scl, vals[h8 + e + 1] * scl, vals[h8 + e + 2] * scl, vals[h8 + e + 3] * scl);
+          }
+        }
+      } else {
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD + col;
+        uint32_t u[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) u[e] = pack_bf16x2_rne_int(vals[2 * e] * scl, vals[2 * e + 1] * scl);
+        if (g.o_rows_32b) {
+          st_global_v8(dst, u);
+        } else {
+          *reinterpret_cast<uint4*>(dst) = make_uint4(u[0], u[1], u[2], u[3]);
+          *reinterpret_cast<uint4*>(dst + 8) = make_uint4(u[4], u[5], u[6], u[7]);
+        }
+      }
+    };
+    int it = 0;
+    bool aborted = false;
+    for (long long tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int s = it % kStages;
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) {
+        aborted = true;
+        break;
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(table_bar(s), (it / kStages) & 1, limit_ns))) {
+        aborted = true;
+        break;
+      }
+      const int tok = tables[s].tok[row];
+      const int tok_t = do_tail ? tables[s].tok[128 + (lane & 15)] : -1;
+      mbar_arrive(empty_bar(s));
+      const int head = static_cast<int>(tile) - fdiv(static_cast<int>(tile), g.div_heads) * g.heads;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(o_full, it & 1, limit_ns))) {
+        aborted = true;
+        break;
+      }
+      tc_fence_after();
+      float ov[HD], l;
+      float ot[HD / 2], lt = 0.f;
+#pragma unroll
+      for (int m = 0; m < HD / 16; ++m) tmem_ld16(tmem + lane_base + TM_O0 + 16 * m, ov + 16 * m);
+      tmem_ld1(tmem + lane_base + TM_O0 + kOnesCol, &l);
+      if (do_tail) {
+#pragma unroll
+        for (int m = 0; m < HD / 32; ++m) tmem_ld_16x32bx2_x16(tmem + TM_O1 + 32 * m, ot + 16 * m);
+        tmem_ld_16x32bx2_x1(tmem + TM_O1 + kOnesCol, &lt);
+      }
+      tmem_wait_ld();
+#pragma unroll
+      for (int m = 0; m < HD / 16; ++m) reg_fence16(ov + 16 * m);
+      reg_fence1(&l);
+      if (do_tail) {
+#pragma unroll
+        for (int m = 0; m < HD / 32; ++m) reg_fence16(ot + 16 * m);
+        reg_fence1(&lt);
+      }
+      tc_fence_before();
+      mbar_arrive(o_empty);
+      if (tok >= 0) {
+        const float inv = l > 0.f ? rcp_approx(l) : 0.f;
+#pragma unroll
+        for (int m = 0; m < HD / 16; ++m) store16(tok, head, 16 * m, ov + 16 * m, inv);
+      }
+      if (tok_t >= 0) {
+        const float inv = lt > 0.f ? rcp_approx(lt) : 0.f;
+#pragma unroll
+        for (int m = 0; m < HD / 32; ++m) store16(tok_t, head, 32 * m + 16 * thalf, ot + 16 * m, inv);
+      }
+    }
+    if (aborted) {
+      if (lane == 0) record_error(err, kStatusTimeout);
+      *abort_flag = 1;
+    }
   } else if (warp < kMainWarps || (warp == kTailWarp && has_tail)) {
-    // ------------------------------------------------------------------ softmax + epilogue
+    // ------------------------------------------------------------------ softmax
     // Every softmax thread owns one (query row, key half) and runs the same code.  Half h
     // holds the key groups 2k + h (k = 0..8) of 8 keys each, 72 keys.  Main warp w: row
     // 32 (w % 4) + lane (its TMEM lane in S0 = Q[0:128] K^T), half w / 4, read with the
     // 32x32b shape at column 16k + 8h; its partner (same row, other half) is warp w ^ 4,
-    // and the two swap row max and row sum through shared memory.  Tail warp 8: row
-    // 128 + lane % 16 (TMEM lane lane % 16 of S1 = Q[128:144] K^T), half lane / 16, read
-    // with the 16x32bx2 shape (threads 16..31 see the columns 8 further on); its partner is
-    // lane ^ 16 of the same warp (a shuffle).
+    // and the two swap row maxima through shared memory.  Tail warp 8: row 128 + lane % 16
+    // (TMEM lane lane % 16 of S1 = Q[128:144] K^T), half lane / 16, read with the 16x32bx2
+    // shape (threads 16..31 see the columns 8 further on); its partner is lane ^ 16 of the
+    // same warp (a shuffle).
     const bool is_tail = warp == kTailWarp;
     const float c = g.scale_log2;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -543,9 +424,6 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     const uint32_t pb2 = sb + (is_tail ? OFF_P1B2 : OFF_STAGE + OFF_P0B2);
     const uint32_t p_stage_step = is_tail ? kTailPBytes : kStageBytes;
     const uint32_t s_base = is_tail ? tmem + TM_S1 : tmem + lane_base + TM_S0 + 8 * half;
-    // O columns of a thread: groups of 16, 32m + 16h .. +15 (m < head_dim / 32); the main
-    // rows take them with 32x32b at that column, the tail with 16x32bx2 at column 32m.
-    const uint32_t o_base = is_tail ? tmem + TM_O1 : tmem + lane_base + TM_O0 + 16 * half;
     const uint32_t my_hi = [&] {
       uint32_t h = 0;
 #pragma unroll
@@ -553,81 +431,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       return h;
     }();
     int it = 0;
-    // state of the previous tile, finished one iteration later
-    bool have_prev = false;
-    int prev_it = 0, prev_head = 0, prev_tok = -1;
     bool aborted = false;
-
-    auto store8 = [&](int tk, int head, int col, const float* vals, float scl) {
-      // 8 consecutive outputs of one row starting at column `col`.
-      if constexpr (OUT_F32) {
-        float* dst = static_cast<float*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD + col;
-        if (g.o_rows_32b) {
-          uint32_t u[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) u[e] = __float_as_uint(vals[e] * scl);
-          st_global_v8(dst, u);
-        } else {
-          *reinterpret_cast<float4*>(dst) = make_float4(vals[0] * scl, vals[1] * scl, vals[2] * scl, vals[3] * scl);
-          *reinterpret_cast<float4*>(dst + 4) = make_float4(vals[4] * scl, vals[5] * scl, vals[6] * scl, vals[7] * scl);
-        }
-      } else {
-        __nv_bfloat16* dst =
-            static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD + col;
-        uint4 u;
-        u.x = pack_bf16x2(vals[0] * scl, vals[1] * scl);
-        u.y = pack_bf16x2(vals[2] * scl, vals[3] * scl);
-        u.z = pack_bf16x2(vals[4] * scl, vals[5] * scl);
-        u.w = pack_bf16x2(vals[6] * scl, vals[7] * scl);
-        *reinterpret_cast<uint4*>(dst) = u;
-      }
-    };
-
-    // Epilogue of a finished tile: this thread's O columns and the row sum (column 64 of O)
-    // from TMEM, scaled by 1/rowsum, stored to the grid position of the query slot
-    // (padded slots dropped).
-    auto epilogue = [&](int pit, int head, int tok) -> bool {
-      bool ok = mbar_wait_bounded(o_full, pit & 1, limit_ns);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) return false;
-      tc_fence_after();
-      float ov[HD / 2];
-      float l;
-      if (!is_tail) {
-#pragma unroll
-        for (int m = 0; m < HD / 32; ++m) tmem_ld16(o_base + 32 * m, ov + 16 * m);
-        tmem_ld1(o_base - 16 * half + kOnesCol, &l);
-      } else {
-#pragma unroll
-        for (int m = 0; m < HD / 32; ++m) tmem_ld_16x32bx2_x16(o_base + 32 * m, ov + 16 * m);
-        tmem_ld_16x32bx2_x1(o_base + kOnesCol, &l);
-      }
-      tmem_wait_ld();
-#pragma unroll
-      for (int m = 0; m < HD / 32; ++m) reg_fence16(ov + 16 * m);
-      reg_fence1(&l);
-      tc_fence_before();
-      mbar_arrive(o_empty);
-      const float inv = l > 0.f ? rcp_approx(l) : 0.f;
-      if (tok >= 0) {
-#pragma unroll
-        for (int m = 0; m < HD / 32; ++m) {
-          const int col = 32 * m + 16 * half;
-          if constexpr (!OUT_F32) {
-            if (g.o_rows_32b) {   // 16 bf16 = one 32-byte store
-              uint32_t u[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) u[e] = pack_bf16x2(ov[16 * m + 2 * e] * inv, ov[16 * m + 2 * e + 1] * inv);
-              st_global_v8(static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tok) * g.o_stride + head * HD + col, u);
-              continue;
-            }
-          }
-          store8(tok, head, col, ov + 16 * m, inv);
-          store8(tok, head, col + 8, ov + 16 * m + 8, inv);
-        }
-      }
-      return true;
-    };
 
     // The thread's 72 logits are read from TMEM once (nine 8-column loads) and stay in
     // registers.  If any thread of the warp has a masked key (near the shift seams and the
@@ -691,73 +495,53 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       }
     };
 
-    // Iteration `it` does the softmax of tile `it` (if any) and then the epilogue of tile
-    // it-1, so the PV MMA of a tile overlaps the next tile's softmax.  One call site each.
     // S is read out of TMEM into registers in one go, so it is released (s_empty) before
     // the exponentials, and the MMA warp can compute the next tile's S underneath them.
-    for (long long tile = blockIdx.x;; tile += gridDim.x, ++it) {
-      const bool have_cur = tile < num_tiles;
-      int head = 0, tok = -1;
-      if (have_cur) {
-        const int s = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
-        if (__any_sync(0xffffffffu, *abort_flag != 0)) {
-          aborted = true;
-          break;
-        }
-        bool ok = mbar_wait_bounded(table_bar(s), ph, limit_ns);
-        if (!__all_sync(0xffffffffu, ok)) {
-          aborted = true;
-          break;
-        }
-        head = static_cast<int>(tile) - fdiv(static_cast<int>(tile), g.div_heads) * g.heads;
-        const Table& tb = tables[s];
-        tok = tb.tok[row];
-        const uint4 mq = tb.maskq[my_hi * 2 + half];
-        mbar_arrive(empty_bar(s));
+    for (long long tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int s = it % kStages;
+      const uint32_t ph = (it / kStages) & 1;
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) {
+        aborted = true;
+        break;
+      }
+      bool ok = mbar_wait_bounded(table_bar(s), ph, limit_ns);
+      if (!__all_sync(0xffffffffu, ok)) {
+        aborted = true;
+        break;
+      }
+      const uint4 mq = tables[s].maskq[my_hi * 2 + half];
+      mbar_arrive(empty_bar(s));
 
-        ok = mbar_wait_bounded(s_full, it & 1, limit_ns);
+      ok = mbar_wait_bounded(s_full, it & 1, limit_ns);
+      if (!__all_sync(0xffffffffu, ok)) {
+        aborted = true;
+        break;
+      }
+      tc_fence_after();
+      float x[72];
+      const float mh = row_max(x, mq);
+      tc_fence_before();
+      mbar_arrive(s_empty);   // S of this thread is in registers: the next S may be written
+      const int par = it & 1;
+      float mrow;
+      if (!is_tail) {
+        xmax[(par * 2 + half) * 128 + row] = mh;
+        mbar_arrive(xmax_bar(par, half));
+        ok = mbar_wait_bounded(xmax_bar(par, half ^ 1), (it >> 1) & 1, limit_ns);
         if (!__all_sync(0xffffffffu, ok)) {
           aborted = true;
           break;
         }
-        tc_fence_after();
-        float x[72];
-        const float mh = row_max(x, mq);
-        tc_fence_before();
-        mbar_arrive(s_empty);   // S of this thread is in registers: the next S may be written
-        const int par = it & 1;
-        float mrow;
-        if (!is_tail) {
-          xmax[(par * 2 + half) * 128 + row] = mh;
-          mbar_arrive(xmax_bar(par, half));
-          ok = mbar_wait_bounded(xmax_bar(par, half ^ 1), (it >> 1) & 1, limit_ns);
-          if (!__all_sync(0xffffffffu, ok)) {
-            aborted = true;
-            break;
-          }
-          mrow = fmaxf(mh, xmax[(par * 2 + (half ^ 1)) * 128 + row]);
-        } else {
-          mrow = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 16));
-        }
-        if (mrow == -INFINITY) mrow = 0.f;
-        // P goes to the tile's own stage (over its Q and K, consumed by S, which s_full
-        // guaranteed above): no wait for the previous tile's PV.
-        row_exp(x, mrow, static_cast<uint32_t>(s) * p_stage_step);
-        fence_proxy_async_smem();
-        mbar_arrive(is_tail ? p_full_t(par) : p_full(par));
+        mrow = fmaxf(mh, xmax[(par * 2 + (half ^ 1)) * 128 + row]);
+      } else {
+        mrow = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 16));
       }
-      if (have_prev) {
-        if (!epilogue(prev_it, prev_head, prev_tok)) {
-          aborted = true;
-          break;
-        }
-      }
-      if (!have_cur) break;
-      have_prev = true;
-      prev_it = it;
-      prev_head = head;
-      prev_tok = tok;
+      if (mrow == -INFINITY) mrow = 0.f;
+      // P goes to the tile's own stage (over its Q and K, consumed by S, which s_full
+      // guaranteed above): no wait for the previous tile's PV.
+      row_exp(x, mrow, static_cast<uint32_t>(s) * p_stage_step);
+      fence_proxy_async_smem();
+      mbar_arrive(is_tail ? p_full_t(par) : p_full(par));
     }
     if (aborted) {
       if (lane == 0) record_error(err, kStatusTimeout);
@@ -769,49 +553,6 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    cudaDriverEntryPointQueryResult qres;
-    void* ptr = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
-        qres == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
-
-cudaError_t make_maps(const WinGeom& g, const void* const ptrs[3], TmaMaps* maps) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-  if (!enc) return cudaErrorNotSupported;
-  const cuuint64_t es = 2;  // bf16
-  const cuuint64_t C = static_cast<cuuint64_t>(g.heads) * g.head_dim;
-  const cuuint64_t dims[5] = {C, static_cast<cuuint64_t>(g.W), static_cast<cuuint64_t>(g.H),
-                              static_cast<cuuint64_t>(g.T), static_cast<cuuint64_t>(g.B)};
-  const cuuint64_t row = static_cast<cuuint64_t>(g.qkv_stride) * es;
-  const cuuint64_t strides[4] = {row, row * g.W, row * g.W * g.H, row * g.W * g.H * g.T};
-  // box (W, H) extents per shape; a seam shape of an unshifted axis is never used and
-  // gets the whole window instead
-  const cuuint32_t ww = static_cast<cuuint32_t>(g.ww), wh = static_cast<cuuint32_t>(g.wh);
-  const cuuint32_t sw = static_cast<cuuint32_t>(g.sw), sh = static_cast<cuuint32_t>(g.sh);
-  const cuuint32_t boxwh[kBoxShapes][2] = {{ww, wh},
-                                           {ww, wh - sh},
-                                           {ww, sh > 0 ? sh : wh},
-                                           {ww - sw, 1},
-                                           {sw > 0 ? sw : ww, 1}};
-  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  for (int t = 0; t < 3; ++t)
-    for (int b = 0; b < kBoxShapes; ++b) {
-      const cuuint32_t box[5] = {64, boxwh[b][0], boxwh[b][1], 1, 1};
-      CUresult r = enc(&maps->m[t][b], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptrs[t]), dims, strides,
-                       box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-      if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    }
-  return cudaSuccess;
 }
 
 template <int HD, bool OUT_F32>
@@ -832,7 +573,7 @@ cudaError_t launch_window_attn_tc(const WinGeom& g, const void* q, const void* k
                                   bool out_f32, int* err, long long spin_limit, int num_sms, cudaStream_t stream) {
   TmaMaps maps;
   const void* ptrs[3] = {q, k, v};
-  cudaError_t e = make_maps(g, ptrs, &maps);
+  cudaError_t e = make_maps(g, ptrs, false, &maps);
   if (e != cudaSuccess) return e;
   if (g.head_dim == 64)
     return out_f32 ? launch_t<64, true>(g, maps, o, err, spin_limit, num_sms, stream)

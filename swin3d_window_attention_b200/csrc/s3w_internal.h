@@ -12,6 +12,11 @@ cudaError_t launch_window_attn_tc(const WinGeom& g, const void* q, const void* k
                                   void* o, bool out_f32, int* err, long long spin_limit,
                                   int num_sms, cudaStream_t stream);
 
+// Window attention in the TF32_ACC_FP32 mode: fp32 Q/K/V, tcgen05 kind::tf32 (attn_tf32.cu).
+cudaError_t launch_window_attn_tf32(const WinGeom& g, const void* q, const void* k, const void* v,
+                                    void* o, bool out_f32, int* err, long long spin_limit,
+                                    int num_sms, cudaStream_t stream);
+
 // Window attention on the legacy warp-level mma.sync path (attn_mma.cu); kept as the
 // measured baseline the tcgen05 kernel is compared with.
 cudaError_t launch_window_attn_mma(const WinGeom& g, const void* q, const void* k, const void* v,

@@ -45,8 +45,8 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity
 }
 
 // Slow path of mbar_wait_bounded, kept out of line so that the many wait sites of the
-// kernels stay small in the instruction cache.
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+// kernels stay small in the instruction cache (internal linkage: one copy per kernel file).
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
@@ -281,6 +281,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
   const uint32_t a = __float_as_uint(lo) + 0x8000u;
   const uint32_t b = __float_as_uint(hi) + 0x8000u;
   return __byte_perm(a, b, 0x7632);
+}
+
+// Two finite fp32 values -> packed bf16x2 rounded to nearest, ties to even, on the integer
+// pipe: add 0x7fff plus the lowest kept bit to the bit pattern, keep the upper halves.
+__device__ __forceinline__ uint32_t pack_bf16x2_rne_int(float lo, float hi) {
+  const uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
+  const uint32_t ra = a + 0x7fffu + ((a >> 16) & 1u);
+  const uint32_t rb = b + 0x7fffu + ((b >> 16) & 1u);
+  return __byte_perm(ra, rb, 0x7632);
 }
 
 // 32-byte global store (one full sector per thread).

@@ -62,13 +62,20 @@ def _attn(**over):
     (dict(scale=float("nan")), api.S3W_ERR_INVALID_ARG),
     (dict(ww=13, sw=6), api.S3W_ERR_UNSUPPORTED),   # N = 156 > 144
     (dict(hd=48, qs=384, os_=384), api.S3W_ERR_UNSUPPORTED),
-    (dict(ind=1), api.S3W_ERR_UNSUPPORTED),         # fp32 Q/K/V not built
+    (dict(ind=1, qs=514), api.S3W_ERR_MISALIGNED),  # fp32 token rows not on 16-byte boundaries
     (dict(q=FAKE + 8), api.S3W_ERR_MISALIGNED),
     (dict(o=FAKE + 2), api.S3W_ERR_MISALIGNED),
     (dict(qs=516), api.S3W_ERR_MISALIGNED),         # token rows not on 16-byte boundaries
 ])
 def test_attn_rejects_bad_arguments_on_host(over, expect):
     assert _attn(**over) == expect
+
+
+def test_legacy_baseline_is_bf16_only():
+    lib = s3w.load_library()
+    rc = lib.swin3d_window_attn_fwd_legacy_mma(FAKE, FAKE, FAKE, FAKE, 1, 4, 12, 24, 2, 6, 12, 1, 3, 6, 8, 64, 512,
+                                               512, 0.0, api.S3W_F32, 0, None)
+    assert rc == api.S3W_ERR_UNSUPPORTED
 
 
 def _adaln(**over):

@@ -1,0 +1,321 @@
+"""Randomised model of the mbarrier protocols of the two tensor-core attention kernels.
+
+Each role of one CTA (TMA loader, table writer, MMA issuer, the softmax warps) is a generator
+that follows the kernel's sequence of waits and arrivals; MMA commits and TMA completions land
+later, each stream in issue order.  A seeded random scheduler with per-role speeds interleaves
+them.  The checks: no deadlock; a parity wait passes only when exactly the phase it waits for
+has completed (so it can neither pass on, nor miss, another phase); every arrival of one phase
+belongs to one tile.  mbarrier semantics modelled: a phase completes when its count of
+arrivals is reached; try_wait.parity(p) passes iff the current phase parity differs from p.
+
+The BF16 kernel (3 stages, P over the stage's Q/K, P and row-max hand-over barriers per tile
+parity, O read out by four epilogue warps) and the TF32 kernel (2 stages, P over S in TMEM, S(t+1) after PV(t) completes) are
+modelled; the single-barrier variant of the BF16 protocol must be caught.
+"""
+import random
+
+import pytest
+
+STAGES = 3
+
+
+class Bar:
+    def __init__(self, name, count):
+        self.name, self.count, self.pending, self.done = name, count, count, 0
+        self.tile = None
+
+    def arrive(self, tile, n=1):
+        if self.tile is None:
+            self.tile = tile
+        assert self.tile == tile, f"{self.name}: phase {self.done} mixes tiles {self.tile} and {tile}"
+        self.pending -= n
+        assert self.pending >= 0, f"{self.name}: too many arrivals"
+        if self.pending == 0:
+            self.done += 1
+            self.pending = self.count
+            self.tile = None
+
+
+def model(ntiles, has_tail=True, variant="new", seed=0, max_steps=2_000_000):
+    rng = random.Random(seed)
+    n_soft_warps = 9 if has_tail else 8
+    nsoft = 32 * n_soft_warps
+    B = {}
+
+    def mk(name, count):
+        B[name] = Bar(name, count)
+
+    nepi = 128
+    for s in range(STAGES):
+        mk(f"load{s}", 1)
+        mk(f"empty{s}", 1 + nsoft + nepi)
+        mk(f"table{s}", 32)
+    mk("s_full", 1)
+    mk("s_empty", nsoft)
+    for p in range(2):
+        mk(f"p_full{p}", 256)
+        mk(f"p_full_t{p}", 32)
+        for h in range(2):
+            mk(f"xmax{p}{h}", 128)
+    mk("o_full", 1)
+    mk("o_empty", nepi)
+
+    def tma():
+        for it in range(ntiles):
+            s = it % STAGES
+            yield ("wait", f"empty{s}", ((it // STAGES) & 1) ^ 1, it // STAGES - 1)
+            yield ("tma", f"load{s}", it)
+
+    def table():
+        for it in range(ntiles):
+            s = it % STAGES
+            yield ("wait", f"empty{s}", ((it // STAGES) & 1) ^ 1, it // STAGES - 1)
+            yield ("arrive", f"table{s}", it, 32)
+
+    def mma():
+        for j in range(ntiles + 1):
+            if j < ntiles:
+                s = j % STAGES
+                yield ("wait", f"load{s}", (j // STAGES) & 1, j // STAGES)
+                yield ("wait", "s_empty", (j & 1) ^ 1, j - 1)
+                yield ("commit", [("s_full", j)])
+            if j > 0:
+                jt = j - 1
+                s = jt % STAGES
+                if variant == "single":
+                    yield ("wait", "p_full0", jt & 1, jt)
+                else:
+                    yield ("wait", f"p_full{jt & 1}", (jt >> 1) & 1, jt >> 1)
+                yield ("wait", "o_empty", (jt & 1) ^ 1, jt - 1)
+                if has_tail:
+                    if variant == "single":
+                        yield ("wait", "p_full_t0", jt & 1, jt)
+                    else:
+                        yield ("wait", f"p_full_t{jt & 1}", (jt >> 1) & 1, jt >> 1)
+                yield ("commit", [("o_full", jt), (f"empty{s}", jt)])
+
+    def softmax(w):
+        tail = w == 8
+        half = 0 if tail else (w >> 2) & 1
+        for it in range(ntiles):
+            s = it % STAGES
+            yield ("wait", f"table{s}", (it // STAGES) & 1, it // STAGES)
+            yield ("arrive", f"empty{s}", it, 32)
+            yield ("wait", "s_full", it & 1, it)
+            yield ("arrive", "s_empty", it, 32)
+            par = it & 1
+            if not tail:
+                yield ("arrive", f"xmax{par}{half}", it, 32)
+                yield ("wait", f"xmax{par}{half ^ 1}", (it >> 1) & 1, it >> 1)
+            pp = 0 if variant == "single" else par
+            yield ("arrive", f"p_full_t{pp}" if tail else f"p_full{pp}", it, 32)
+
+    def epilogue():
+        # the four epilogue warps (warps 12..15): tokens from the table, then O
+        for it in range(ntiles):
+            s = it % STAGES
+            yield ("wait", f"table{s}", (it // STAGES) & 1, it // STAGES)
+            yield ("arrive", f"empty{s}", it, 32)
+            yield ("wait", "o_full", it & 1, it)
+            yield ("arrive", "o_empty", it, 32)
+
+    actors = {"tma": tma(), "table": table(), "mma": mma()}
+    for w in range(n_soft_warps):
+        actors[f"w{w}"] = softmax(w)
+    for e in range(4):
+        actors[f"epi{e}"] = epilogue()
+    cur = {k: None for k in actors}
+    asyncq = []          # in-order tensor-core completions: (bar, tile)
+    tmaq = []            # TMA completions (in order among themselves)
+    weight = {k: rng.choice([0.05, 0.3, 1.0, 1.0, 3.0]) for k in actors}
+    finished = set()
+    steps = 0
+    while len(finished) < len(actors) or asyncq or tmaq:
+        steps += 1
+        assert steps < max_steps
+        runnable = []
+        for k, g in actors.items():
+            if k in finished:
+                continue
+            if cur[k] is None:
+                try:
+                    cur[k] = next(g)
+                except StopIteration:
+                    finished.add(k)
+                    continue
+            op = cur[k]
+            if op[0] == "wait":
+                b = B[op[1]]
+                ok = (b.done & 1) != op[2]
+                if ok:
+                    assert b.done == op[3] + 1, f"{k}: wait on {op[1]} for phase {op[3]} passed with {b.done} done"
+                else:
+                    assert b.done == op[3], f"{k}: wait on {op[1]} for phase {op[3]} blocked with {b.done} done"
+                    continue
+            runnable.append(k)
+        choices = runnable + (["async"] if asyncq else []) + (["tmaq"] if tmaq else [])
+        if not choices and len(finished) == len(actors):
+            break
+        if not choices:
+            raise AssertionError("deadlock: " + ", ".join(f"{k}:{cur[k]}" for k in actors if k not in finished))
+        # per-actor speeds drawn per seed, to provoke races
+        k = rng.choices(choices, weights=[weight.get(c, 0.5) for c in choices])[0]
+        if k in ("async", "tmaq"):
+            q = asyncq if k == "async" else tmaq
+            bar, tile = q.pop(0)
+            B[bar].arrive(tile)
+            continue
+        op = cur[k]
+        cur[k] = None
+        if op[0] == "arrive":
+            B[op[1]].arrive(op[2], op[3])
+        elif op[0] == "commit":
+            asyncq.extend(op[1])
+        elif op[0] == "tma":
+            tmaq.append((op[1], op[2]))
+    return steps
+
+
+def model_tf32(ntiles, has_tail=True, seed=0, max_steps=2_000_000):
+    """The TF32 kernel: 2 stages, P over S in TMEM, S(t+1) after PV(t) completes."""
+    rng = random.Random(seed)
+    ST = 2
+    nw = 9 if has_tail else 8
+    nsoft = 32 * nw
+    B = {}
+
+    def mk(name, count):
+        B[name] = Bar(name, count)
+
+    for s in range(ST):
+        mk(f"load{s}", 1); mk(f"empty{s}", 1 + nsoft); mk(f"table{s}", 32)
+    for n, c in (("s_full", 1), ("p_full", 256), ("p_full_t", 32), ("o_full", 1), ("o_empty", nsoft),
+                 ("pv_done", 1), ("xmax0", 128), ("xmax1", 128)):
+        mk(n, c)
+
+    def tma():
+        for it in range(ntiles):
+            s = it % ST
+            yield ("wait", f"empty{s}", ((it // ST) & 1) ^ 1, it // ST - 1)
+            yield ("tma", f"load{s}", it)
+
+    def table():
+        for it in range(ntiles):
+            s = it % ST
+            yield ("wait", f"empty{s}", ((it // ST) & 1) ^ 1, it // ST - 1)
+            yield ("arrive", f"table{s}", it, 32)
+
+    def issue_s(j):
+        s = j % ST
+        yield ("wait", f"load{s}", (j // ST) & 1, j // ST)
+        if j > 0:
+            yield ("wait", "pv_done", (j - 1) & 1, j - 1)
+            yield ("sync_pv", j - 1)     # the waiter itself observed PV(j-1) complete
+        yield ("commit", [("s_full", j)])
+
+    def mma():
+        if ntiles:
+            yield from issue_s(0)
+        for t in range(ntiles):
+            s = t % ST
+            yield ("wait", "p_full", t & 1, t)
+            yield ("wait", "o_empty", (t & 1) ^ 1, t - 1)
+            if has_tail:
+                yield ("wait", "p_full_t", t & 1, t)
+            yield ("commit", [("o_full", t), (f"empty{s}", t), ("pv_done", t)])
+            if t + 1 < ntiles:
+                yield from issue_s(t + 1)
+
+    def softmax(w):
+        tail = w == 8
+        half = (w >> 2) & 1
+        prev = None
+        for it in range(ntiles + 1):
+            if it < ntiles:
+                s = it % ST
+                yield ("wait", f"table{s}", (it // ST) & 1, it // ST)
+                yield ("arrive", f"empty{s}", it, 32)
+                yield ("wait", "s_full", it & 1, it)
+                if not tail:
+                    yield ("arrive", f"xmax{half}", it, 32)
+                    yield ("wait", f"xmax{half ^ 1}", it & 1, it)
+                yield ("arrive", "p_full_t" if tail else "p_full", it, 32)
+            if prev is not None:
+                yield ("wait", "o_full", prev & 1, prev)
+                yield ("arrive", "o_empty", prev, 32)
+            if it < ntiles:
+                prev = it
+
+    actors = {"tma": tma(), "table": table(), "mma": mma()}
+    for w in range(nw):
+        actors[f"w{w}"] = softmax(w)
+    cur = {k: None for k in actors}
+    asyncq, tmaq, finished = [], [], set()
+    weight = {k: rng.choice([0.05, 0.3, 1.0, 1.0, 3.0]) for k in actors}
+    steps = 0
+    while len(finished) < len(actors) or asyncq or tmaq:
+        steps += 1
+        assert steps < max_steps
+        runnable = []
+        for k, g in actors.items():
+            if k in finished:
+                continue
+            if cur[k] is None:
+                try:
+                    cur[k] = next(g)
+                except StopIteration:
+                    finished.add(k)
+                    continue
+            op = cur[k]
+            if op[0] == "wait":
+                b = B[op[1]]
+                if (b.done & 1) != op[2]:
+                    assert b.done == op[3] + 1, f"{k}: wait {op[1]} phase {op[3]} passed with {b.done}"
+                else:
+                    assert b.done == op[3], f"{k}: wait {op[1]} phase {op[3]} blocked with {b.done}"
+                    continue
+            runnable.append(k)
+        choices = runnable + (["async"] if asyncq else []) + (["tmaq"] if tmaq else [])
+        if not choices and len(finished) == len(actors):
+            break
+        if not choices:
+            raise AssertionError("deadlock: " + ", ".join(f"{k}:{cur[k]}" for k in actors if k not in finished))
+        k = rng.choices(choices, weights=[weight.get(c, 0.5) for c in choices])[0]
+        if k in ("async", "tmaq"):
+            q = asyncq if k == "async" else tmaq
+            bar, tile = q.pop(0)
+            B[bar].arrive(tile)
+            continue
+        op = cur[k]
+        cur[k] = None
+        if op[0] == "arrive":
+            B[op[1]].arrive(op[2], op[3])
+        elif op[0] == "commit":
+            asyncq.extend(op[1])
+        elif op[0] == "tma":
+            tmaq.append((op[1], op[2]))
+
+
+
+def test_bf16_protocol_holds_under_random_schedules():
+    for seed in range(120):
+        for tail in (True, False):
+            model(ntiles=1 + seed % 13, has_tail=tail, seed=seed)
+
+
+def test_single_barrier_variant_is_caught():
+    """Without per-parity hand-over barriers a warp can lap another (the protocol this
+    replaced): the model must find it."""
+    fails = 0
+    for seed in range(60):
+        try:
+            model(ntiles=2 + seed % 12, has_tail=True, variant="single", seed=seed)
+        except AssertionError:
+            fails += 1
+    assert fails > 0
+
+
+def test_tf32_protocol_holds_under_random_schedules():
+    for seed in range(120):
+        for tail in (True, False):
+            model_tf32(ntiles=1 + seed % 11, has_tail=tail, seed=seed)

@@ -38,8 +38,8 @@ def test_recorded_traffic_follows_the_kernel_source(tmp_path):
     src_dir = tmp_path / "swin3d_window_attention_b200" / "csrc"
     src_dir.mkdir(parents=True)
     (tmp_path / "profiles").mkdir()
-    files = {"attn_tcgen05.cu": "int a = 1;  // kernel v1\n", "sm100_ptx.cuh": "int b = 1;\n",
-             "s3w_common.cuh": "int c = 1;\n"}
+    files = {"attn_tcgen05.cu": "int a = 1;  // kernel v1\n", "attn_common.cuh": "int d = 1;\n",
+             "sm100_ptx.cuh": "int b = 1;\n", "s3w_common.cuh": "int c = 1;\n"}
     for name, text in files.items():
         (src_dir / name).write_text(text)
     sha = bench.kernel_code_sha256(str(tmp_path))
