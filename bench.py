@@ -89,6 +89,14 @@ def attn_flops(w):
     return windows * w["heads"] * 4 * N_TOK * N_TOK * w["hd"]
 
 
+def fused_bytes(w, out_bytes=4):
+    """The fused attention + AdaLN call: Q, K, V, the fp32 residual and the output once each;
+    the attention output never leaves the chip (its bf16 copy goes through a per-CTA
+    workspace of 2 windows that stays in L2)."""
+    C, tokens, _ = geometry(w)
+    return tokens * C * (3 * 2 + 4 + out_bytes)
+
+
 def adaln_bytes(w, x_bytes=2, out_bytes=4):
     """x, the fp32 residual and the output, once each (scale/shift are negligible)."""
     C, tokens, _ = geometry(w)
@@ -354,6 +362,45 @@ def bench_configs(torch, s3w, dev, stream, peaks, reps):
                                       {**peaks, "bf16_tflops": peaks["bf16_tflops"] / 2})}}
     del q, k, v, o
 
+    # fused attention + AdaLN (one kernel per block) on the stage-1 grid: one launch, and the
+    # headline step (two blocks) made of fused calls against the two-call step
+    w = WORKLOADS["stage1"]
+    C, tokens, windows = geometry(w)
+    qkv = [device_qkv(torch, w, dev, 950 + 10 * b) for b in range(2)]
+    films = [device_film(torch, w, dev, 970 + 10 * b, 0.1)[:2] for b in range(2)]
+    res = device_film(torch, w, dev, 990, 1.0)[2]
+    o = torch.empty_like(qkv[0][0])
+    x = o.view(w["B"], tokens // w["B"], C)
+    ws = torch.empty(s3w.window_attn_adaln_workspace_bytes(w["B"], w["T"], w["H"], w["W"], w["heads"], w["hd"],
+                                                           WINDOW), dtype=torch.uint8, device=dev)
+
+    def fused_call(b):
+        q, k, v = qkv[b]
+        s3w.swin3d_window_attn_adaln_fwd(q, k, v, res, films[b][0], films[b][1], res, w["heads"], w["hd"], WINDOW,
+                                         SHIFTS[b], workspace=ws, eps=1e-5)
+
+    def two_call_block(b):
+        q, k, v = qkv[b]
+        s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTS[b])
+        s3w.adaln_residual_fwd(x, res, films[b][0], films[b][1], res, eps=1e-5)
+
+    ms_f = timed(torch, stream, lambda: fused_call(1), reps)
+    ms_fs = timed(torch, stream, lambda: [fused_call(b) for b in range(2)], reps)
+    ms_ts = timed(torch, stream, lambda: [two_call_block(b) for b in range(2)], reps)
+    launches += len(ms_f) + 2 * len(ms_fs) + 4 * len(ms_ts)
+    f_med = statistics.median(ms_f)
+    nbytes = fused_bytes(w)
+    out["stage1_fused"] = {
+        "grid": "B=1 T4xH180xW360, 8 heads x 64, shift (1,3,6), 1800 windows; attention + AdaLN in one kernel, "
+                "fp32 residual in place",
+        "fused": {**launch_stats(ms_f), "bytes": nbytes, "flops": attn_flops(w), "windows_per_s": windows / (f_med * 1e-3),
+                  "roofline": roofline(nbytes, attn_flops(w), f_med, peaks)},
+        "step_fused_ms": launch_stats(ms_fs), "step_two_call_ms": launch_stats(ms_ts),
+        "step_bytes_fused": 2 * nbytes, "step_bytes_two_call": 2 * (attn_bytes(w) + adaln_bytes(w)),
+        "step_windows_per_s_fused": 2 * windows / (statistics.median(ms_fs) * 1e-3),
+        "step_windows_per_s_two_call": 2 * windows / (statistics.median(ms_ts) * 1e-3)}
+    del qkv, films, res, o, x, ws
+
     # six-block stage-1 stack at B = 4: fresh Q/K/V per block, fp32 residual chained
     w = WORKLOADS["stack_b4"]
     C, tokens, windows = geometry(w)
@@ -369,9 +416,19 @@ def bench_configs(torch, s3w, dev, stream, peaks, reps):
             s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTS[b % 2])
             s3w.adaln_residual_fwd(x, res, films[b][0], films[b][1], res, eps=1e-5)
 
+    ws = torch.empty(s3w.window_attn_adaln_workspace_bytes(w["B"], w["T"], w["H"], w["W"], w["heads"], w["hd"],
+                                                           WINDOW), dtype=torch.uint8, device=dev)
+
+    def stack_fused():
+        for b in range(STACK_BLOCKS):
+            q, k, v = qkv[b]
+            s3w.swin3d_window_attn_adaln_fwd(q, k, v, res, films[b][0], films[b][1], res, w["heads"], w["hd"], WINDOW,
+                                             SHIFTS[b % 2], workspace=ws, eps=1e-5)
+
     stack_reps = max(3, reps // 4)
     ms_s = timed(torch, stream, stack, stack_reps, warmup=2)
-    launches += 2 * STACK_BLOCKS * stack_reps
+    ms_sf = timed(torch, stream, stack_fused, stack_reps, warmup=2)
+    launches += 3 * STACK_BLOCKS * stack_reps
     s_med = statistics.median(ms_s)
     nbytes = STACK_BLOCKS * (attn_bytes(w) + adaln_bytes(w))
     flops = STACK_BLOCKS * attn_flops(w)
@@ -380,8 +437,11 @@ def bench_configs(torch, s3w, dev, stream, peaks, reps):
         "ms_per_stack": launch_stats(ms_s), "bytes": nbytes, "flops": flops,
         "floor_ms_at_measured_hbm": nbytes / (peaks["hbm_gbs"] * 1e9) * 1e3,
         "windows_per_s": STACK_BLOCKS * windows / (s_med * 1e-3),
-        "roofline": roofline(nbytes, flops, s_med, peaks)}
-    del qkv, films, res, o, x
+        "roofline": roofline(nbytes, flops, s_med, peaks),
+        "fused": {"ms_per_stack": launch_stats(ms_sf), "bytes": STACK_BLOCKS * fused_bytes(w),
+                  "windows_per_s": STACK_BLOCKS * windows / (statistics.median(ms_sf) * 1e-3),
+                  "roofline": roofline(STACK_BLOCKS * fused_bytes(w), flops, statistics.median(ms_sf), peaks)}}
+    del qkv, films, res, o, x, ws
     torch.cuda.empty_cache()
     return out, launches
 

@@ -135,6 +135,54 @@ int adaln_residual_fwd(const void* x, int x_dtype, const float* residual,
                        int B, long long tokens_per_sample, int C, float eps,
                        s3w_stream_t stream);
 
+/*
+ * Shifted-window attention fused with AdaLN + residual: one launch computes, for every token,
+ *   x   = the window attention output of all heads (as swin3d_window_attn_fwd, rounded to
+ *         bf16 exactly as that call stores it),
+ *   out = residual + (x - mean) / sqrt(var + eps) * (1 + adaln_scale[b]) + adaln_shift[b]
+ *         (as adaln_residual_fwd), without writing x to global memory in full.
+ *
+ * Defines: "Flash-Aurora: Toward Efficient Inference for Geospatial Foundation Models",
+ * section "Kernel fusion for backbone memory traffic" (LayerNorm, FiLM modulation and the
+ * residual add without a full-width intermediate; FP32 activations between blocks) with the
+ * attention of section "CuTe DSL window attention" (BF16_MIXED).
+ *
+ * Each CTA takes whole windows, all heads of a window in a row, so every channel of a token
+ * passes through one CTA.  The statistics of each token's row are merged head by head in
+ * shared memory; the bf16 rows wait in `workspace` (per CTA, two windows deep) until the
+ * window's last head is in, then the row is normalised and written to `out`.
+ *
+ * q, k, v, qkv_token_stride, the grid, window, shift, heads, head_dim (32 or 64) and
+ *              attn_scale: as swin3d_window_attn_fwd; BF16 inputs only.
+ * residual     device fp32 [B][T*H*W][C], C = heads * head_dim (C % 8 == 0, C <= 4096).
+ * adaln_scale, adaln_shift  device fp32 [B][C].
+ * out          device, out_dtype (S3W_F32 or S3W_BF16), [B][T*H*W][C]; may alias residual
+ *              exactly (in-place update of the residual stream).
+ * o            optional device bf16 [B][T][H][W][C] (token stride C), 32-byte aligned: when
+ *              non-NULL the attention output is written there too; NULL skips it.
+ * workspace    device memory of at least swin3d_window_attn_adaln_workspace_bytes(...) bytes
+ *              for the current device, 32-byte aligned, owned by the caller; its contents on
+ *              entry do not matter.  Calls that overlap on the GPU must not share it.
+ * eps          >= 0.
+ * Returns S3W_OK or an s3w_status; on error nothing is launched.
+ */
+int swin3d_window_attn_adaln_fwd(const void* q, const void* k, const void* v, long long qkv_token_stride,
+                                 const float* residual, const float* adaln_scale, const float* adaln_shift,
+                                 void* out, int out_dtype, void* o, void* workspace, long long workspace_bytes,
+                                 int B, int T, int H, int W,
+                                 int win_t, int win_h, int win_w,
+                                 int shift_t, int shift_h, int shift_w,
+                                 int heads, int head_dim, float attn_scale, float eps,
+                                 s3w_stream_t stream);
+
+/*
+ * Bytes of workspace swin3d_window_attn_adaln_fwd needs on the current device for this grid
+ * (one CTA per SM up to the number of windows, 2 x 144 x C bf16 each).  A negative value is
+ * minus an s3w_status (invalid sizes, or no CUDA device).
+ */
+long long swin3d_window_attn_adaln_workspace_bytes(int B, int T, int H, int W, int win_t, int win_h, int win_w,
+                                                   int heads, int head_dim);
+
 /* Static English text for a status code (never NULL). */
 const char* s3w_status_string(int status);
 

@@ -13,6 +13,8 @@ from .api import (  # noqa: F401
     set_test_stall,
     set_wait_limit_ns,
     status_string,
+    swin3d_window_attn_adaln_fwd,
     swin3d_window_attn_fwd,
     swin3d_window_attn_fwd_legacy_mma,
+    window_attn_adaln_workspace_bytes,
 )

@@ -55,6 +55,11 @@ def load_library():
     lib.s3w_poll_device_error.restype = I
     lib.s3w_version.argtypes = []
     lib.s3w_version.restype = I
+    lib.swin3d_window_attn_adaln_fwd.argtypes = [P, P, P, LL, P, P, P, P, I, P, P, LL, I, I, I, I, I, I, I, I, I, I,
+                                                 I, I, F, F, P]
+    lib.swin3d_window_attn_adaln_fwd.restype = I
+    lib.swin3d_window_attn_adaln_workspace_bytes.argtypes = [I] * 9
+    lib.swin3d_window_attn_adaln_workspace_bytes.restype = LL
     _lib = lib
     return lib
 
@@ -125,6 +130,50 @@ def _attn(entry, q, k, v, o, heads, head_dim, window, shift, scale, stream, chec
                                     _dtype_code(q), _dtype_code(o), st)
     if check and rc != S3W_OK:
         raise S3WError(rc, entry)
+    return rc
+
+
+def window_attn_adaln_workspace_bytes(B, T, H, W, heads: int, head_dim: int, window=(2, 6, 12)) -> int:
+    """Workspace bytes of the fused attention + AdaLN call on the current device."""
+    n = int(load_library().swin3d_window_attn_adaln_workspace_bytes(B, T, H, W, *window, heads, head_dim))
+    if n < 0:
+        raise S3WError(-n, "swin3d_window_attn_adaln_workspace_bytes")
+    return n
+
+
+def swin3d_window_attn_adaln_fwd(q, k, v, residual, scale, shift, out, heads: int, head_dim: int,
+                                 window=(2, 6, 12), shift_=(0, 0, 0), o=None, workspace=None, eps: float = 1e-5,
+                                 attn_scale: float = 0.0, stream=None, check: bool = True) -> int:
+    """Window attention fused with AdaLN + residual.  q, k, v: bf16 [B, T, H, W, >=C] (one token
+    stride); residual: fp32 [B, L, C]; scale, shift: fp32 [B, C]; out: fp32/bf16 [B, L, C] (may
+    be ``residual``); o: optional bf16 [B, T, H, W, C] for the attention output.  workspace: a
+    CUDA tensor of at least window_attn_adaln_workspace_bytes(...) bytes (allocated here when
+    None)."""
+    import torch
+
+    lib = load_library()
+    C = heads * head_dim
+    B, T, H, W = q.shape[:4]
+    ts = _token_stride(q, C)
+    if _token_stride(k, C) != ts or _token_stride(v, C) != ts:
+        raise ValueError("q, k and v must share one token stride")
+    for t in (residual, out):
+        if not t.is_contiguous() or t.numel() != B * T * H * W * C:
+            raise ValueError("residual and out must be contiguous [B, L, C]")
+    if o is not None and (not o.is_contiguous() or o.dtype != torch.bfloat16 or tuple(o.shape) != (B, T, H, W, C)):
+        raise ValueError("o must be a contiguous bf16 [B, T, H, W, C] tensor")
+    need = window_attn_adaln_workspace_bytes(B, T, H, W, heads, head_dim, window)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = _stream_of(q) if stream is None else stream
+    rc = lib.swin3d_window_attn_adaln_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), ts, residual.data_ptr(),
+                                          scale.data_ptr(), shift.data_ptr(), out.data_ptr(), _dtype_code(out),
+                                          None if o is None else o.data_ptr(), workspace.data_ptr(), ws_bytes,
+                                          B, T, H, W, *window, *shift_, heads, head_dim, float(attn_scale),
+                                          float(eps), st)
+    if check and rc != S3W_OK:
+        raise S3WError(rc, "swin3d_window_attn_adaln_fwd")
     return rc
 
 

@@ -193,6 +193,58 @@ int swin3d_window_attn_fwd_legacy_mma(const void* q, const void* k, const void* 
   return e == cudaSuccess ? S3W_OK : S3W_ERR_CUDA;
 }
 
+long long swin3d_window_attn_adaln_workspace_bytes(int B, int T, int H, int W, int win_t, int win_h, int win_w,
+                                                  int heads, int head_dim) {
+  if (B < 1 || T < 1 || H < 1 || W < 1 || win_t < 1 || win_h < 1 || win_w < 1 || heads < 1 || head_dim < 1)
+    return -S3W_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  const int rc = device_state(&ds);
+  if (rc != S3W_OK) return -rc;
+  const long long windows = static_cast<long long>(B) * ((T + win_t - 1) / win_t) * ((H + win_h - 1) / win_h) *
+                            ((W + win_w - 1) / win_w);
+  const long long grid = s3w::window_attn_adaln_grid(windows, ds->num_sms);
+  return grid * 2 * 144 * static_cast<long long>(heads) * head_dim * 2;
+}
+
+int swin3d_window_attn_adaln_fwd(const void* q, const void* k, const void* v, long long qkv_token_stride,
+                                 const float* residual, const float* adaln_scale, const float* adaln_shift,
+                                 void* out, int out_dtype, void* o, void* workspace, long long workspace_bytes,
+                                 int B, int T, int H, int W, int win_t, int win_h, int win_w, int shift_t,
+                                 int shift_h, int shift_w, int heads, int head_dim, float attn_scale, float eps,
+                                 s3w_stream_t stream) {
+  if (!residual || !adaln_scale || !adaln_shift || !out || !workspace) return S3W_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || std::isinf(eps)) return S3W_ERR_INVALID_ARG;
+  if (out_dtype != S3W_BF16 && out_dtype != S3W_F32) return S3W_ERR_INVALID_ARG;
+  const long long C = static_cast<long long>(heads) * head_dim;
+  // attention checks (o, when given, is a bf16 grid tensor with token stride C)
+  s3w::WinGeom g;
+  int rc = make_geometry(q, k, v, o ? o : out, B, T, H, W, win_t, win_h, win_w, shift_t, shift_h, shift_w, heads,
+                         head_dim, qkv_token_stride, C, attn_scale, S3W_BF16, S3W_BF16, &g);
+  if (rc != S3W_OK) return rc;
+  if (C % 8 != 0 || C > 4096) return S3W_ERR_UNSUPPORTED;
+  if (!aligned16(residual) || !aligned16(adaln_scale) || !aligned16(adaln_shift) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 31u) != 0 || (o && (reinterpret_cast<uintptr_t>(o) & 31u) != 0))
+    return S3W_ERR_MISALIGNED;
+  // out may alias residual exactly; any other overlap with residual is rejected
+  const long long n = static_cast<long long>(B) * T * H * W * C;
+  const char* r0 = reinterpret_cast<const char*>(residual);
+  const char* o0 = reinterpret_cast<const char*>(out);
+  const long long ob = out_dtype == S3W_F32 ? 4 : 2;
+  if (o0 != r0 && o0 < r0 + n * 4 && r0 < o0 + n * ob) return S3W_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  rc = device_state(&ds);
+  if (rc != S3W_OK) return rc;
+  const long long grid = s3w::window_attn_adaln_grid(g.windows, ds->num_sms);
+  if (workspace_bytes < grid * 2 * 144 * C * 2) return S3W_ERR_INVALID_ARG;
+  g.test_stall = g_test_stall.load(std::memory_order_relaxed);
+  s3w::AdalnArgs fa{residual, adaln_scale, adaln_shift, out, static_cast<uint16_t*>(workspace), eps,
+                    out_dtype == S3W_F32 ? 1 : 0};
+  cudaError_t e = s3w::launch_window_attn_adaln(g, q, k, v, o, fa, ds->err,
+                                                g_wait_limit_ns.load(std::memory_order_relaxed), ds->num_sms,
+                                                reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? S3W_OK : S3W_ERR_CUDA;
+}
+
 int adaln_residual_fwd(const void* x, int x_dtype, const float* residual, const float* scale, const float* shift,
                        void* out, int out_dtype, int B, long long tokens_per_sample, int C, float eps,
                        s3w_stream_t stream) {

@@ -182,6 +182,22 @@ inline cudaError_t make_maps(const WinGeom& g, const void* const ptrs[3], bool f
   return cudaSuccess;
 }
 
+// The CTA's it-th tile, or -1 when it has none left.  Strided order (WINDOW_MAJOR false):
+// tile = blockIdx.x + it * gridDim.x.  Window-major order: the CTA takes whole windows,
+// window blockIdx.x + (it / heads) * gridDim.x, all its heads in a row (tile = window *
+// heads + head), so that every head of a token's row passes through one CTA.
+template <bool WINDOW_MAJOR>
+__device__ __forceinline__ long long cta_tile(const WinGeom& g, int it) {
+  if constexpr (!WINDOW_MAJOR) {
+    const long long t = blockIdx.x + static_cast<long long>(it) * gridDim.x;
+    return t < g.windows * g.heads ? t : -1;
+  } else {
+    const int k = fdiv(it, g.div_heads);
+    const long long w = blockIdx.x + static_cast<long long>(k) * gridDim.x;
+    return w < g.windows ? w * g.heads + (it - k * g.heads) : -1;
+  }
+}
+
 // Shared-memory addresses of a ring of stages and its barriers (8 bytes each, consecutive).
 struct Ring {
   uint32_t stage0;       // stage 0's Q tile
@@ -197,7 +213,7 @@ struct Ring {
 // x, chunk c at stage + x * CHUNKS * kChunkTileBytes + c * kChunkTileBytes, rows in slot
 // order.  Padded coordinates are out of bounds and read as zero.  On an abort, or after the
 // last tile, waits (bounded) for the loads still in flight before returning.
-template <int CHUNKS, int CHUNK_CH, int STAGES, int STAGE_BYTES>
+template <int CHUNKS, int CHUNK_CH, int STAGES, int STAGE_BYTES, bool WINDOW_MAJOR = false>
 __device__ __forceinline__ void tma_loader(const WinGeom& g, const TmaMaps& maps, const Ring& ring, int head_dim,
                                            long long num_tiles, volatile int* abort_flag, int* err,
                                            unsigned long long limit_ns) {
@@ -209,7 +225,8 @@ __device__ __forceinline__ void tma_loader(const WinGeom& g, const TmaMaps& maps
   const uint32_t tile_bytes = static_cast<uint32_t>(3 * CHUNKS * g.N * kRowBytes);
   const uint32_t run_bytes = static_cast<uint32_t>(g.ww) * kRowBytes;
   int it = 0;
-  for (long long tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+  for (long long tile = cta_tile<WINDOW_MAJOR>(g, 0); tile >= 0 && tile < num_tiles;
+       tile = cta_tile<WINDOW_MAJOR>(g, ++it)) {
     const int s = it % STAGES;
     if (*abort_flag) break;
     if (!mbar_wait_bounded(ring.empty_bar0 + 8u * s, ((it / STAGES) & 1) ^ 1, limit_ns)) {
@@ -279,12 +296,13 @@ __device__ __forceinline__ void tma_loader(const WinGeom& g, const TmaMaps& maps
 // Table writer (one warp, named barrier 1).  Per tile, once the stage is free: the slot ->
 // grid-token map, the bitmask of real slots, the "last window along a shifted axis" flags
 // and, from these, the key masks per (region combination, key half).
-template <int STAGES>
+template <int STAGES, bool WINDOW_MAJOR = false>
 __device__ __forceinline__ void table_writer(const WinGeom& g, Table* tables, const SlotConst* slotc, const Ring& ring,
                                              long long num_tiles, volatile int* abort_flag, volatile int* prod_stop,
                                              int* err, unsigned long long limit_ns, int lane) {
   int it = 0;
-  for (long long tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+  for (long long tile = cta_tile<WINDOW_MAJOR>(g, 0); tile >= 0 && tile < num_tiles;
+       tile = cta_tile<WINDOW_MAJOR>(g, ++it)) {
     const int s = it % STAGES;
     if (lane == 0) {
       const bool ok = mbar_wait_bounded(ring.empty_bar0 + 8u * s, ((it / STAGES) & 1) ^ 1, limit_ns);

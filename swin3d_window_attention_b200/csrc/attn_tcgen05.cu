@@ -19,8 +19,9 @@
 //                      it with the warp holding the other half, then exp2 and P rounded to
 //                      bf16 into shared memory.  One tile later (the PV MMA overlaps the next
 //                      softmax) it loads half of the row's O columns and the row sum (an MMA
-//                      output column, see below), scales by 1/rowsum and stores them to the
-//                      query's original grid position; padded slots are dropped.
+//                      output column, see below), scales by 1/rowsum, rounds to nearest even
+//                      and stores them to the query's original grid position; padded slots
+//                      are dropped.
 //   tail warp 8        the same for the 16 tail rows (S1 = Q[128:144] K^T in TMEM lanes
 //                      0..15, reachable from warp 8 like from warp 0), read with the 16x32bx2
 //                      shape: threads 0..15 hold half 0 of rows 128..143, threads 16..31
@@ -31,13 +32,14 @@
 //                      read as an MN-major operand followed by 16 columns of ones, so O's
 //                      columns from 64 on are the row sums of the bf16 P; completion is
 //                      signalled by tcgen05.commit.
-//   TMA warp 10        one thread loads the tile's Q, K and V with TMA: one box per T-slab
+//   TMA warp 10        (attn_common.cuh, shared with the TF32 kernel)
+//                      one thread loads the tile's Q, K and V with TMA: one box per T-slab
 //                      of the window (win_h x win_w tokens) per tensor, cut where the window
 //                      wraps around a seam of the shifted grid, straight from grid layout into
 //                      a 3-stage ring in the tensor core's 128-byte swizzled K-major layout;
 //                      padded coordinates are out of bounds and read as zero.  It runs ahead
 //                      as far as the ring allows.
-//   table warp 11      writes the slot -> grid-token table, a bitmask of the real slots, the
+//   table warp 11      (attn_common.cuh) writes the slot -> grid-token table, a bitmask of the real slots, the
 //                      window's "last along a shifted axis" flags and, from these, the key
 //                      masks per region combination and key half, for the stage being loaded.
 // Synchronisation is by mbarriers only; every wait is bounded by a time limit and a
@@ -57,31 +59,19 @@ using namespace sm100;
 using namespace attn;
 
 constexpr int kStages = 3;
-constexpr int kTileBytes = kChunkTileBytes;         // 18432: one of Q / K / V (one head = 128 B rows)
+constexpr int kTileBytes = kChunkTileBytes;         // 18432: one of Q / K / V
 constexpr int kStageBytes = 3 * kTileBytes;         // 55296
 
-// Shared-memory map (offsets from a 1024-byte aligned base).
-// Once S = Q K^T of a tile has been computed, its Q and K tiles are dead: the P of the 128
-// main rows (36 KB, exactly the size of Q + K) is written over them, in the tile's own
-// stage, so P of the next tile never waits for the PV MMA of this one.  In a stage:
-//   P rows 0..127, keys 0..63    at +0      (128B swizzle, over Q)
-//   P rows 0..127, keys 64..127  at +16384  (128B swizzle, over Q rows 128.. and K)
-//   P rows 0..127, keys 128..143 at +32768  (32B swizzle, 4 KB, over K)
-// The 16 tail rows' P of stage s lives in a block of its own at s * kTailPBytes.  Their
-// M = 128 descriptors also cover rows 16..127, which fall on the blocks and stages that
-// follow (valid memory; the results of those rows are never used).
-constexpr int kTailPBytes = 5120;
+// Shared-memory map (offsets from a 1024-byte aligned base).  The tail P blocks only hold
+// 16 rows; the rows 16..127 their M = 128 descriptors also cover fall on the buffers that
+// follow (valid memory, results of those rows are never used).
 constexpr int OFF_P1B0 = 0;        // tail P rows 0..15, keys 0..63   (128B swizzle)
 constexpr int OFF_P1B1 = 2048;     // tail P rows 0..15, keys 64..127 (128B swizzle)
 constexpr int OFF_P1B2 = 4096;     // tail P rows 0..15, keys 128..143 (32B swizzle)
-constexpr int OFF_P0B0 = 0;        // main P, relative to the stage
-constexpr int OFF_P0B1 = 16384;
-constexpr int OFF_P0B2 = 32768;
-static_assert(OFF_P0B2 + 128 * 32 <= 2 * kTileBytes, "main P fits over Q and K");
-constexpr int OFF_STAGE = kStages * kTailPBytes;   // 15360 (1024-aligned)
-static_assert(OFF_STAGE % 1024 == 0 && kStageBytes % 1024 == 0, "swizzle atoms stay aligned");
-static_assert((kStages - 1) * kTailPBytes + 128 * kRowBytes <= OFF_STAGE + kStageBytes,
-              "the tail P descriptors' unused rows stay inside the stages");
+constexpr int OFF_P0B0 = 5120;     // P rows 0..127, keys 0..63
+constexpr int OFF_P0B1 = OFF_P0B0 + 16384;
+constexpr int OFF_P0B2 = OFF_P0B1 + 16384;   // keys 128..143, 32B swizzle, 4 KB
+constexpr int OFF_STAGE = OFF_P0B2 + 4096;   // 41984 (1024-aligned)
 // 16 key rows of bf16 ones in the V operand's layout: the PV MMA reads them as 16 more
 // output columns (through the descriptor's leading byte offset), so every such column of O
 // is the row sum of P as rounded to bf16, the exact normaliser of the P the MMA used.
@@ -91,14 +81,11 @@ constexpr int OFF_TABLE = OFF_ONES + kOnesBytes;
 
 constexpr int OFF_SLOTC = OFF_TABLE + kStages * kTableBytes;
 constexpr int OFF_BARS = OFF_SLOTC + kSlotConstBytes;
-// barriers: load[3] (TMA bytes), empty[3], table[3], s_full, s_empty, p_full[2] (tile
-// parity), o_full, o_empty, drain, row max written[2][2] (tile parity, key half), tail
-// p_full[2] (tile parity).
-// P and the row maxima of a tile are handed over on barriers of the tile's parity.  Nothing
-// stops one softmax warp from arriving for tile t+1 before another has arrived for tile t,
-// or the tail warp from completing tile t+1's P before the MMA warp has waited for tile
-// t's; but no warp can arrive for tile t+2 before every waiter of tile t has passed (that
-// needs S(t+2), which the MMA warp issues only after its waits of tile t).
+// barriers: load[3] (TMA bytes), empty[3], table[3], s_full, s_empty, p_full, p_empty,
+// o_full, o_empty, drain, row max written[0][2], tail p_full, tail p_empty, row max
+// written[1][2] (row max barriers: [tile parity][key half]).  A softmax thread releases S (s_empty) before it waits for the other half's row
+// maximum, so the warps of one half can reach tile t+2 before a warp of the other half has
+// waited for tile t; one row-max barrier per tile parity keeps that wait on its own phase.
 constexpr int kNumBars = 3 * kStages + 13;
 // Row max of each key half of the main rows, exchanged between the two warps that share a
 // row: [tile parity][key half][row].
@@ -108,6 +95,14 @@ constexpr int OFF_MISC = OFF_XCHG + kXchgFloats * 4;   // tmem address, abort fl
 constexpr int kSmemBytes = OFF_MISC + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1024;       // slack for the 1024-byte alignment
 static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
+// Fused attention + AdaLN only: per window parity, the running statistics of every row's two
+// column halves, the rows' grid tokens, and the window-ready / window-free barriers.
+constexpr int OFF_WSTAT = kSmemBytes;                         // float2 [2 parity][2 half][kN]
+constexpr int OFF_WTOK = OFF_WSTAT + 2 * 2 * kN * 8;          // int [2 parity][kN]
+constexpr int OFF_WBAR = OFF_WTOK + 2 * kN * 4;               // win_full[2], win_free[2]
+constexpr int kSmemBytesFused = OFF_WBAR + 4 * 8;
+constexpr int kSmemAllocFused = kSmemBytesFused + 1024;
+static_assert(kSmemAllocFused <= 232448, "shared memory per CTA (fused)");
 
 // TMEM columns (fp32 accumulators, lane = row).  Every MMA destination is 32-aligned.  O
 // has 80 columns: the head's outputs (the first head_dim of 64), then from column 64 on 16
@@ -116,15 +111,17 @@ constexpr uint32_t TM_S0 = 0, TM_S1 = 160, TM_O0 = 320, TM_O1 = 416;
 constexpr uint32_t kOnesCol = 64;
 constexpr uint32_t kTmemCols = 512;
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 384;
 constexpr int kMainWarps = 8;          // rows 0..127: warp w holds lanes 32 (w % 4) .., keys 72 (w / 4) ..
 constexpr int kTailWarp = 8;           // tail rows 128..143 (TMEM lane quarter 0, like warp 0)
 constexpr int kMmaWarp = 9;
 constexpr int kTmaWarp = 10;
 constexpr int kFirstProducerWarp = 11;
 constexpr int kProducerThreads = 32;   // table writer (warp 11)
-constexpr int kFirstEpiWarp = 12;      // warps 12..15: O of TMEM lane quarter warp % 4 to global memory
-constexpr int kEpiThreads = 128;
+// Fused attention + AdaLN: warps 12..15 normalise finished windows (the AdaLN warps).
+constexpr int kThreadsFused = 512;
+constexpr int kFirstAdalnWarp = 12;
+constexpr int kAdalnThreads = 128;
 
 // Operand descriptors.  K-major 128B swizzle: 8-row x 128-byte atoms, 1024 bytes apart.
 // K-major 32B swizzle: 8-row x 32-byte atoms, 256 bytes apart.  MN-major 128B swizzle (V,
@@ -133,10 +130,210 @@ constexpr int kEpiThreads = 128;
 __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t addr) { return smem_desc(addr, 16, 1024, kSwizzle128B); }
 __device__ __forceinline__ uint64_t desc_kmajor_sw32(uint32_t addr) { return smem_desc(addr, 16, 256, kSwizzle32B); }
 
-template <int HD, bool OUT_F32>
-__global__ void __launch_bounds__(kThreads, 1)
+// ---------------------------------------------------------------- fused attention + AdaLN
+// "Flash-Aurora: Toward Efficient Inference for Geospatial Foundation Models", section
+// "Kernel fusion for backbone memory traffic": LayerNorm, FiLM modulation and the residual
+// add fused without a full-width intermediate.  The fused kernel takes whole windows (all
+// heads of every token of the window pass through one CTA).  Per head, the epilogue rounds
+// the thread's half-row of O to bf16 (the AdaLN input, exactly what the unfused path stores),
+// merges its statistics into a running (mean, M2) per (row, column half) (Chan, Golub and
+// LeVeque's pairwise update), and writes the bf16 values to the CTA's workspace.  When the
+// last head is in, the AdaLN warps normalise the window row by row:
+//   out = residual + (x - mean) / sqrt(var + eps) * (1 + scale_b) + shift_b.
+
+// Epilogue of one (window, head) tile in the fused kernel: the thread holds HD / 2 values of
+// O (its column half: groups of 16 at 32m + 16 half) already summed over the keys.
+template <int HD>
+__device__ __forceinline__ void fused_epilogue(const WinGeom& g, const AdalnArgs& fa, void* o, const float* ov,
+                                               float inv, int head, int tok, int row, int half, int wp,
+                                               float2* wstat, int* wtok, int C) {
+  constexpr int kVals = HD / 2;
+  uint32_t u[kVals / 2];
+  float sum = 0.f;
+#pragma unroll
+  for (int e = 0; e < kVals / 2; ++e) {
+    u[e] = pack_bf16x2(ov[2 * e] * inv, ov[2 * e + 1] * inv);
+    sum += __uint_as_float(u[e] << 16) + __uint_as_float(u[e] & 0xffff0000u);
+  }
+  const float mean_b = sum * (1.0f / kVals);
+  float m2_b = 0.f;
+#pragma unroll
+  for (int e = 0; e < kVals / 2; ++e) {
+    const float d0 = __uint_as_float(u[e] << 16) - mean_b, d1 = __uint_as_float(u[e] & 0xffff0000u) - mean_b;
+    m2_b = fmaf(d0, d0, fmaf(d1, d1, m2_b));
+  }
+  float2& st = wstat[(wp * 2 + half) * kN + row];
+  if (head == 0) {
+    st = make_float2(mean_b, m2_b);
+    if (half == 0) wtok[wp * kN + row] = tok;
+  } else {
+    // merge n_a = head * kVals values (mean_a, M2_a) with n_b = kVals values (mean_b, M2_b)
+    const float2 a = st;
+    const float na = static_cast<float>(head * kVals), nb = static_cast<float>(kVals);
+    const float n = na + nb, d = mean_b - a.x;
+    st = make_float2(a.x + d * (nb / n), a.y + m2_b + d * d * (na * nb / n));
+  }
+  if (tok < 0) return;
+  uint16_t* ws = fa.ws + ((static_cast<long long>(blockIdx.x) * 2 + wp) * kN + row) * C + head * HD;
+#pragma unroll
+  for (int m = 0; m < HD / 32; ++m) {
+    const int col = 32 * m + 16 * half;
+    uint32_t v8[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v8[e] = u[8 * m + e];
+    st_global_v8(ws + col, v8);
+    if (o != nullptr)
+      st_global_v8(static_cast<uint16_t*>(o) + static_cast<long long>(tok) * g.o_stride + head * HD + col, v8);
+  }
+}
+
+// The AdaLN warps (warps 12..15): per finished window, warp q normalises rows q, q + 4, ...,
+// two rows per pass; lane l takes the 8-channel groups l and l + 32 of each pass (then
+// l + 64, l + 96, ... for wider rows).  Every load of a pass is issued before its first
+// store (the output may be the residual itself, so the compiler could not reorder them),
+// and the residual rows kPrefetchPasses passes ahead are prefetched into L2, so a pass
+// costs about one L2 round trip.  The two column halves' running statistics of a row
+// combine into the row's mean and variance (biased, over C).
+// wbar0: the window barriers, win_full[2] then win_free[2].
+constexpr int kPrefetchPasses = 3;
+
+__device__ __forceinline__ void adaln_group(const AdalnArgs& fa, const float* scb, const float* shb, int tok, int cg,
+                                            float mean, float rstd, const uint4 xv, const float4 r0, const float4 r1,
+                                            int C) {
+  const float4 a0 = __ldg(reinterpret_cast<const float4*>(scb + cg * 8));
+  const float4 a1 = __ldg(reinterpret_cast<const float4*>(scb + cg * 8 + 4));
+  const float4 c0 = __ldg(reinterpret_cast<const float4*>(shb + cg * 8));
+  const float4 c1 = __ldg(reinterpret_cast<const float4*>(shb + cg * 8 + 4));
+  const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+  const float rr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+  const float sc[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+  const float sh[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  float y[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float x = (e & 1) ? __uint_as_float(xw[e >> 1] & 0xffff0000u) : __uint_as_float(xw[e >> 1] << 16);
+    y[e] = rr[e] + (x - mean) * rstd * (1.0f + sc[e]) + sh[e];
+  }
+  if (fa.out_f32) {
+    float* op = static_cast<float*>(fa.out) + static_cast<long long>(tok) * C + cg * 8;
+    __stcs(reinterpret_cast<float4*>(op), make_float4(y[0], y[1], y[2], y[3]));
+    __stcs(reinterpret_cast<float4*>(op + 4), make_float4(y[4], y[5], y[6], y[7]));
+  } else {
+    uint4 uo;
+    uo.x = pack_bf16x2(y[0], y[1]);
+    uo.y = pack_bf16x2(y[2], y[3]);
+    uo.z = pack_bf16x2(y[4], y[5]);
+    uo.w = pack_bf16x2(y[6], y[7]);
+    __stcs(reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(fa.out) + static_cast<long long>(tok) * C + cg * 8),
+           uo);
+  }
+}
+
+__device__ __forceinline__ void adaln_warps(const WinGeom& g, const AdalnArgs& fa, const float2* wstat,
+                                            const int* wtok, uint32_t wbar0, volatile int* abort_flag, int* err,
+                                            unsigned long long limit_ns, int warp, int lane, int C) {
+  auto win_full = [&](int wp) { return wbar0 + 8u * wp; };
+  auto win_free = [&](int wp) { return wbar0 + 8u * (2 + wp); };
+  const int q = warp - kFirstAdalnWarp;
+  const float nh = 0.5f * static_cast<float>(C);   // values per column half of a row
+  const int ng = C >> 3;                            // 8-channel groups per row
+  bool aborted = false;
+  for (int k = 0;; ++k) {
+    const long long win = blockIdx.x + static_cast<long long>(k) * gridDim.x;
+    if (win >= g.windows) break;
+    const int wp = k & 1;
+    if (__any_sync(0xffffffffu, *abort_flag != 0)) {
+      aborted = true;
+      break;
+    }
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(win_full(wp), (k >> 1) & 1, limit_ns))) {
+      aborted = true;
+      break;
+    }
+    const long long b = fdiv(static_cast<int>(win), g.div_per_sample);
+    const float* scb = fa.scale + b * C;
+    const float* shb = fa.shift + b * C;
+    const uint16_t* wsw = fa.ws + (static_cast<long long>(blockIdx.x) * 2 + wp) * kN * C;
+    const int* tokw = wtok + wp * kN;
+    // this warp's rows: j-th row q + 4j; rows at or beyond the window size are padding
+    // slots (rows 128.. exist only with a tail warp)
+    const int nrows = g.N > q ? (g.N - q + 3) / 4 : 0;
+    auto prefetch_row = [&](int j) {
+      if (j < nrows) {
+        const int tok = tokw[q + 4 * j];
+        if (tok >= 0) bulk_prefetch_l2(fa.residual + static_cast<long long>(tok) * C, static_cast<uint32_t>(C) * 4u);
+      }
+    };
+    if (lane < 2 * kPrefetchPasses) prefetch_row(lane);
+    for (int j = 0; j < nrows; j += 2) {
+      if (lane < 2) prefetch_row(j + 2 * kPrefetchPasses + lane);
+      const int ra = q + 4 * j, rb = ra + 4;
+      const int ta = tokw[ra];
+      const int tb = j + 1 < nrows ? tokw[rb] : -1;
+      auto stats = [&](int r, float& mean, float& rstd) {
+        const float2 s0 = wstat[(wp * 2 + 0) * kN + r], s1 = wstat[(wp * 2 + 1) * kN + r];
+        const float d = s1.x - s0.x;
+        mean = 0.5f * (s0.x + s1.x);
+        const float var = (s0.y + s1.y + d * d * (0.5f * nh)) / static_cast<float>(C);
+        rstd = 1.0f / sqrtf(var + fa.eps);
+      };
+      float ma = 0.f, sa = 0.f, mb = 0.f, sb = 0.f;
+      if (ta >= 0) stats(ra, ma, sa);
+      if (tb >= 0) stats(rb, mb, sb);
+      const float* resa = fa.residual + static_cast<long long>(ta >= 0 ? ta : 0) * C;
+      const float* resb = fa.residual + static_cast<long long>(tb >= 0 ? tb : 0) * C;
+      const uint16_t* xa = wsw + static_cast<long long>(ra) * C;
+      const uint16_t* xb = wsw + static_cast<long long>(rb) * C;
+#pragma unroll 1
+      for (int c0 = lane; c0 < ng; c0 += 64) {
+        const int c1 = c0 + 32;
+        const bool h1 = c1 < ng;
+        uint4 xa0{}, xa1{}, xb0{}, xb1{};
+        float4 ra00{}, ra01{}, ra10{}, ra11{}, rb00{}, rb01{}, rb10{}, rb11{};
+        if (ta >= 0) {
+          xa0 = *reinterpret_cast<const uint4*>(xa + c0 * 8);
+          ra00 = __ldcs(reinterpret_cast<const float4*>(resa + c0 * 8));
+          ra01 = __ldcs(reinterpret_cast<const float4*>(resa + c0 * 8 + 4));
+          if (h1) {
+            xa1 = *reinterpret_cast<const uint4*>(xa + c1 * 8);
+            ra10 = __ldcs(reinterpret_cast<const float4*>(resa + c1 * 8));
+            ra11 = __ldcs(reinterpret_cast<const float4*>(resa + c1 * 8 + 4));
+          }
+        }
+        if (tb >= 0) {
+          xb0 = *reinterpret_cast<const uint4*>(xb + c0 * 8);
+          rb00 = __ldcs(reinterpret_cast<const float4*>(resb + c0 * 8));
+          rb01 = __ldcs(reinterpret_cast<const float4*>(resb + c0 * 8 + 4));
+          if (h1) {
+            xb1 = *reinterpret_cast<const uint4*>(xb + c1 * 8);
+            rb10 = __ldcs(reinterpret_cast<const float4*>(resb + c1 * 8));
+            rb11 = __ldcs(reinterpret_cast<const float4*>(resb + c1 * 8 + 4));
+          }
+        }
+        if (ta >= 0) {
+          adaln_group(fa, scb, shb, ta, c0, ma, sa, xa0, ra00, ra01, C);
+          if (h1) adaln_group(fa, scb, shb, ta, c1, ma, sa, xa1, ra10, ra11, C);
+        }
+        if (tb >= 0) {
+          adaln_group(fa, scb, shb, tb, c0, mb, sb, xb0, rb00, rb01, C);
+          if (h1) adaln_group(fa, scb, shb, tb, c1, mb, sb, xb1, rb10, rb11, C);
+        }
+      }
+    }
+    __syncwarp();
+    mbar_arrive(win_free(wp));   // this thread has read the window's buffers of this parity
+  }
+  if (aborted) {
+    if (lane == 0) record_error(err, kStatusTimeout);
+    *abort_flag = 1;
+  }
+}
+
+template <int HD, bool OUT_F32, bool FUSED>
+__global__ void __launch_bounds__(FUSED ? kThreadsFused : kThreads, 1)
 window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__ TmaMaps maps,
-                      void* __restrict__ o, int* __restrict__ err, unsigned long long limit_ns) {
+                      void* __restrict__ o, int* __restrict__ err, unsigned long long limit_ns,
+                      const __grid_constant__ AdalnArgs fa) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(sm);
@@ -147,19 +344,26 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
   auto table_bar = [&](int s) { return bar0 + 8u * (2 * kStages + s); };  // the stage's table written
   const uint32_t s_full = bar0 + 8u * (3 * kStages + 0);
   const uint32_t s_empty = bar0 + 8u * (3 * kStages + 1);
-  auto p_full = [&](int par) { return bar0 + 8u * (3 * kStages + 2 + par); };   // main-row P of a tile
+  const uint32_t p_full = bar0 + 8u * (3 * kStages + 2);
+  const uint32_t p_empty = bar0 + 8u * (3 * kStages + 3);
   const uint32_t o_full = bar0 + 8u * (3 * kStages + 4);
   const uint32_t o_empty = bar0 + 8u * (3 * kStages + 5);
   const uint32_t drain_bar = bar0 + 8u * (3 * kStages + 6);
   // key half h of a tile of parity par wrote its row maxima
-  auto xmax_bar = [&](int par, int h) { return bar0 + 8u * (3 * kStages + 7 + 2 * par + h); };
+  auto xmax_bar = [&](int par, int h) { return bar0 + 8u * (3 * kStages + (par ? 11 : 7) + h); };
   // P of the main rows and of the tail rows are handed over separately, so the main rows'
-  // PV MMA need not wait for the tail warp.
-  auto p_full_t = [&](int par) { return bar0 + 8u * (3 * kStages + 11 + par); };
+  // next P may be written as soon as their own PV MMAs have read it.
+  const uint32_t p_full_t = bar0 + 8u * (3 * kStages + 9);
+  const uint32_t p_empty_t = bar0 + 8u * (3 * kStages + 10);
   float* xmax = reinterpret_cast<float*>(sm + OFF_XCHG);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sm + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
   volatile int* prod_stop = reinterpret_cast<volatile int*>(sm + OFF_MISC + 8);
+  float2* wstat = reinterpret_cast<float2*>(sm + OFF_WSTAT);
+  int* wtok = reinterpret_cast<int*>(sm + OFF_WTOK);
+  auto win_full = [&](int wp) { return sb + OFF_WBAR + 8u * wp; };        // window's x and statistics written
+  auto win_free = [&](int wp) { return sb + OFF_WBAR + 8u * (2 + wp); };  // window normalised: buffers free
+  const int C = g.heads * HD;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -170,18 +374,26 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(load_bar(s), 1);                        // the TMA thread's expect_tx arrival + bytes
-      mbar_init(empty_bar(s), 1 + n_soft + kEpiThreads);  // PV commit + softmax and epilogue threads (table read)
+      mbar_init(empty_bar(s), 1 + n_soft);              // PV commit + every softmax thread (table read)
       mbar_init(table_bar(s), kProducerThreads);
     }
     mbar_init(s_full, 1);
     mbar_init(s_empty, n_soft);
-    for (int par = 0; par < 2; ++par) mbar_init(p_full(par), 256);
-    for (int par = 0; par < 2; ++par) mbar_init(p_full_t(par), 32);
+    mbar_init(p_full, 256);
+    mbar_init(p_empty, 1);
+    mbar_init(p_full_t, 32);
+    mbar_init(p_empty_t, 1);
     mbar_init(o_full, 1);
-    mbar_init(o_empty, kEpiThreads);
+    mbar_init(o_empty, n_soft);
     mbar_init(drain_bar, 1);
     for (int par = 0; par < 2; ++par)
       for (int h = 0; h < 2; ++h) mbar_init(xmax_bar(par, h), 128);
+    if constexpr (FUSED) {
+      for (int wp = 0; wp < 2; ++wp) {
+        mbar_init(win_full(wp), n_soft);
+        mbar_init(win_free(wp), kAdalnThreads);
+      }
+    }
     *abort_flag = 0;
     *prod_stop = 0;
     fence_barrier_init();
@@ -189,12 +401,13 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
   }
   SlotConst* slotc = reinterpret_cast<SlotConst*>(sm + OFF_SLOTC);
   init_slot_consts(g, slotc, tid);
-  for (int i = tid; i < kOnesBytes / 16; i += kThreads)   // bf16 1.0 = 0x3f80
+  constexpr int kNT = FUSED ? kThreadsFused : kThreads;
+  for (int i = tid; i < kOnesBytes / 16; i += kNT)   // bf16 1.0 = 0x3f80
     *reinterpret_cast<uint4*>(sm + OFF_ONES + 16 * i) = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);
   fence_proxy_async_smem();
   // Slots N..143 are never loaded: keep them zero (finite) for the whole kernel.
   if (g.N < kN) {
-    for (int i = tid; i < kStages * 3 * (kN - g.N) * (kRowBytes / 16); i += kThreads) {
+    for (int i = tid; i < kStages * 3 * (kN - g.N) * (kRowBytes / 16); i += kNT) {
       const int chunk = i % (kRowBytes / 16);
       const int rest = i / (kRowBytes / 16);
       const int r = g.N + rest % (kN - g.N);
@@ -215,11 +428,10 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
 
   const Ring ring{sb + OFF_STAGE, load_bar(0), empty_bar(0), table_bar(0)};
   if (warp == kTmaWarp) {
-    // ------------------------------------------------------------------ TMA loads
-    if (lane == 0) tma_loader<1, 64, kStages, kStageBytes>(g, maps, ring, HD, num_tiles, abort_flag, err, limit_ns);
+    if (lane == 0)
+      tma_loader<1, 64, kStages, kStageBytes, FUSED>(g, maps, ring, HD, num_tiles, abort_flag, err, limit_ns);
   } else if (warp == kFirstProducerWarp) {
-    // ------------------------------------------------------------------ tile tables
-    table_writer<kStages>(g, tables, slotc, ring, num_tiles, abort_flag, prod_stop, err, limit_ns, lane);
+    table_writer<kStages, FUSED>(g, tables, slotc, ring, num_tiles, abort_flag, prod_stop, err, limit_ns, lane);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     // Issue order: S(t+1) goes out as soon as tile t+1 is loaded and S(t) has been read
@@ -236,12 +448,9 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     // V of stage 0; its second 64-column atom along N (leading byte offset) is the ones block
     const uint64_t dv0 = smem_desc(sb + OFF_STAGE + 2 * kTileBytes, OFF_ONES - (OFF_STAGE + 2 * kTileBytes), 1024,
                                    kSwizzle128B);
-    // P of the main rows over Q and K of stage 0; the tail rows' P block of stage 0
-    const uint64_t dp0 = desc_kmajor_sw128(sb + OFF_STAGE + OFF_P0B0);
-    const uint64_t dp0b = desc_kmajor_sw32(sb + OFF_STAGE + OFF_P0B2);
+    const uint64_t dp0 = desc_kmajor_sw128(sb + OFF_P0B0), dp0b = desc_kmajor_sw32(sb + OFF_P0B2);
     const uint64_t dp1 = desc_kmajor_sw128(sb + OFF_P1B0), dp1b = desc_kmajor_sw32(sb + OFF_P1B2);
     constexpr uint64_t kStageStep = kStageBytes >> 4;
-    constexpr uint64_t kTailStep = kTailPBytes >> 4;
     const uint32_t leader = lane == 0 ? 1u : 0u;
     bool issued = false;
     auto issue_s = [&](int jt) -> bool {   // S(jt) = Q K^T of the tile in stage jt % kStages
@@ -259,20 +468,20 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     };
     auto issue_pv = [&](int jt) -> bool {  // O(jt) = P V of the tile in stage jt % kStages
       const int s = jt % kStages;
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded(p_full(jt & 1), (jt >> 1) & 1, limit_ns))) return false;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(p_full, jt & 1, limit_ns))) return false;
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(o_empty, (jt & 1) ^ 1, limit_ns))) return false;
       tc_fence_after();
       // Moving V by d (bytes / 16) moves the ones block's leading offset by -d.
       const uint64_t dstage = s * kStageStep;
       const uint64_t vd = dv0 + dstage - (dstage << 16);
-      umma_chain_pv(tmem + TM_O0, dp0 + dstage, vd, idesc_o, leader, dp0b + dstage, ((OFF_P0B1 - OFF_P0B0) >> 4) - 6);
+      umma_chain_pv(tmem + TM_O0, dp0, vd, idesc_o, leader, dp0b, ((OFF_P0B1 - OFF_P0B0) >> 4) - 6);
+      umma_commit_leader(p_empty, leader);
       if (has_tail) {
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(p_full_t(jt & 1), (jt >> 1) & 1, limit_ns))) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(p_full_t, jt & 1, limit_ns))) return false;
         tc_fence_after();
-        const uint64_t dtail = s * kTailStep;
-        umma_chain_pv(tmem + TM_O1, dp1 + dtail, vd, idesc_o, leader, dp1b + dtail,
-                      ((OFF_P1B1 - OFF_P1B0) >> 4) - 6);
+        umma_chain_pv(tmem + TM_O1, dp1, vd, idesc_o, leader, dp1b, ((OFF_P1B1 - OFF_P1B0) >> 4) - 6);
       }
+      if (has_tail) umma_commit_leader(p_empty_t, leader);
       umma_commit_leader(o_full, leader);
       umma_commit_leader(empty_bar(s), leader);
       return true;
@@ -283,8 +492,10 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     // Failure injection (tests): wait on the drain barrier, which nothing signals before the
     // loop below has run, so the bounded wait expires and the CTA takes the timeout path.
     bool ok = !g.test_stall || __all_sync(0xffffffffu, mbar_wait_bounded(drain_bar, 0, limit_ns));
+    const long long my_units = FUSED ? g.windows : num_tiles;   // windows (fused) or tiles
     const long long my_tiles =
-        static_cast<long long>(blockIdx.x) < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+        (static_cast<long long>(blockIdx.x) < my_units ? (my_units - 1 - blockIdx.x) / gridDim.x + 1 : 0) *
+        (FUSED ? g.heads : 1);
     for (long long j = 0; ok && j <= my_tiles; ++j) {
       ok = !__any_sync(0xffffffffu, *abort_flag != 0);
       if (ok && j < my_tiles) ok = issue_s(static_cast<int>(j));
@@ -301,129 +512,31 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       if (!mbar_wait_bounded(drain_bar, 0, 2000000000ull)) record_error(err, kStatusTimeout);
     }
     __syncwarp();
-  } else if (warp >= kFirstEpiWarp) {
-    // ------------------------------------------------------------------ epilogue
-    // Warp 12 + q reads TMEM lane quarter q of O0 (query rows 32q .. 32q + 31, one row per
-    // thread: the head's columns and the row sum, an MMA output column), releases O, scales
-    // by 1/rowsum and stores each row to its query's original grid position; padded slots are
-    // dropped.  Warp 12 also takes the 16 tail rows of O1 (TMEM lanes 0..15), half a row per
-    // thread (16x32bx2 shape).  The grid tokens are read from the tile's table before the
-    // stage is released.
-    const int q = warp - kFirstEpiWarp;
-    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    const int row = q * 32 + lane;
-    const bool do_tail = has_tail && q == 0;
-    const int thalf = lane >> 4;
-    auto store16 = [&](int tk, int head, int col, const float* vals, float scl) {
-      // 16 consecutive outputs of one row starting at column `col`
-      if constexpr (OUT_F32) {
-        float* dst = static_cast<float*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD + col;
-#pragma unroll
-        for (int h8 = 0; h8 < 16; h8 += 8) {
-          if (g.o_rows_32b) {
-            uint32_t u[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) u[e] = __float_as_uint(vals[h8 + e] * scl);
-            st_global_v8(dst + h8, u);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; e += 4)
-              *reinterpret_cast<float4*>(dst + h8 + e) =
-                  make_float4(vals[h8 + e] * scl, vals[h8 + e + 1] * scl, vals[h8 + e + 2] * scl, vals[h8 + e + 3] * scl);
-          }
-        }
-      } else {
-        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD + col;
-        uint32_t u[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) u[e] = pack_bf16x2_rne_int(vals[2 * e] * scl, vals[2 * e + 1] * scl);
-        if (g.o_rows_32b) {
-          st_global_v8(dst, u);
-        } else {
-          *reinterpret_cast<uint4*>(dst) = make_uint4(u[0], u[1], u[2], u[3]);
-          *reinterpret_cast<uint4*>(dst + 8) = make_uint4(u[4], u[5], u[6], u[7]);
-        }
-      }
-    };
-    int it = 0;
-    bool aborted = false;
-    for (long long tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
-      const int s = it % kStages;
-      if (__any_sync(0xffffffffu, *abort_flag != 0)) {
-        aborted = true;
-        break;
-      }
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded(table_bar(s), (it / kStages) & 1, limit_ns))) {
-        aborted = true;
-        break;
-      }
-      const int tok = tables[s].tok[row];
-      const int tok_t = do_tail ? tables[s].tok[128 + (lane & 15)] : -1;
-      mbar_arrive(empty_bar(s));
-      const int head = static_cast<int>(tile) - fdiv(static_cast<int>(tile), g.div_heads) * g.heads;
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded(o_full, it & 1, limit_ns))) {
-        aborted = true;
-        break;
-      }
-      tc_fence_after();
-      float ov[HD], l;
-      float ot[HD / 2], lt = 0.f;
-#pragma unroll
-      for (int m = 0; m < HD / 16; ++m) tmem_ld16(tmem + lane_base + TM_O0 + 16 * m, ov + 16 * m);
-      tmem_ld1(tmem + lane_base + TM_O0 + kOnesCol, &l);
-      if (do_tail) {
-#pragma unroll
-        for (int m = 0; m < HD / 32; ++m) tmem_ld_16x32bx2_x16(tmem + TM_O1 + 32 * m, ot + 16 * m);
-        tmem_ld_16x32bx2_x1(tmem + TM_O1 + kOnesCol, &lt);
-      }
-      tmem_wait_ld();
-#pragma unroll
-      for (int m = 0; m < HD / 16; ++m) reg_fence16(ov + 16 * m);
-      reg_fence1(&l);
-      if (do_tail) {
-#pragma unroll
-        for (int m = 0; m < HD / 32; ++m) reg_fence16(ot + 16 * m);
-        reg_fence1(&lt);
-      }
-      tc_fence_before();
-      mbar_arrive(o_empty);
-      if (tok >= 0) {
-        const float inv = l > 0.f ? rcp_approx(l) : 0.f;
-#pragma unroll
-        for (int m = 0; m < HD / 16; ++m) store16(tok, head, 16 * m, ov + 16 * m, inv);
-      }
-      if (tok_t >= 0) {
-        const float inv = lt > 0.f ? rcp_approx(lt) : 0.f;
-#pragma unroll
-        for (int m = 0; m < HD / 32; ++m) store16(tok_t, head, 32 * m + 16 * thalf, ot + 16 * m, inv);
-      }
-    }
-    if (aborted) {
-      if (lane == 0) record_error(err, kStatusTimeout);
-      *abort_flag = 1;
-    }
+  } else if (FUSED && warp >= kFirstAdalnWarp) {
+    if constexpr (FUSED) adaln_warps(g, fa, wstat, wtok, sb + OFF_WBAR, abort_flag, err, limit_ns, warp, lane, C);
   } else if (warp < kMainWarps || (warp == kTailWarp && has_tail)) {
-    // ------------------------------------------------------------------ softmax
+    // ------------------------------------------------------------------ softmax + epilogue
     // Every softmax thread owns one (query row, key half) and runs the same code.  Half h
     // holds the key groups 2k + h (k = 0..8) of 8 keys each, 72 keys.  Main warp w: row
     // 32 (w % 4) + lane (its TMEM lane in S0 = Q[0:128] K^T), half w / 4, read with the
     // 32x32b shape at column 16k + 8h; its partner (same row, other half) is warp w ^ 4,
-    // and the two swap row maxima through shared memory.  Tail warp 8: row 128 + lane % 16
-    // (TMEM lane lane % 16 of S1 = Q[128:144] K^T), half lane / 16, read with the 16x32bx2
-    // shape (threads 16..31 see the columns 8 further on); its partner is lane ^ 16 of the
-    // same warp (a shuffle).
+    // and the two swap row max and row sum through shared memory.  Tail warp 8: row
+    // 128 + lane % 16 (TMEM lane lane % 16 of S1 = Q[128:144] K^T), half lane / 16, read
+    // with the 16x32bx2 shape (threads 16..31 see the columns 8 further on); its partner is
+    // lane ^ 16 of the same warp (a shuffle).
     const bool is_tail = warp == kTailWarp;
     const float c = g.scale_log2;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int half = is_tail ? (lane >> 4) : ((warp >> 2) & 1);
     const int row = is_tail ? 128 + (lane & 15) : (warp & 3) * 32 + lane;
     const int lrow = is_tail ? (lane & 15) : row;   // row inside its P blocks
-    // P blocks of stage 0 (main rows: over that stage's Q and K; tail rows: its tail block)
-    const uint32_t pb0 = sb + (is_tail ? OFF_P1B0 : OFF_STAGE + OFF_P0B0);
-    const uint32_t pb1 = sb + (is_tail ? OFF_P1B1 : OFF_STAGE + OFF_P0B1);
-    const uint32_t pb2 = sb + (is_tail ? OFF_P1B2 : OFF_STAGE + OFF_P0B2);
-    const uint32_t p_stage_step = is_tail ? kTailPBytes : kStageBytes;
+    const uint32_t pb0 = sb + (is_tail ? OFF_P1B0 : OFF_P0B0);
+    const uint32_t pb1 = sb + (is_tail ? OFF_P1B1 : OFF_P0B1);
+    const uint32_t pb2 = sb + (is_tail ? OFF_P1B2 : OFF_P0B2);
     const uint32_t s_base = is_tail ? tmem + TM_S1 : tmem + lane_base + TM_S0 + 8 * half;
+    // O columns of a thread: groups of 16, 32m + 16h .. +15 (m < head_dim / 32); the main
+    // rows take them with 32x32b at that column, the tail with 16x32bx2 at column 32m.
+    const uint32_t o_base = is_tail ? tmem + TM_O1 : tmem + lane_base + TM_O0 + 16 * half;
     const uint32_t my_hi = [&] {
       uint32_t h = 0;
 #pragma unroll
@@ -431,7 +544,96 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       return h;
     }();
     int it = 0;
+    // state of the previous tile, finished one iteration later
+    bool have_prev = false;
+    int prev_it = 0, prev_head = 0, prev_tok = -1;
     bool aborted = false;
+
+    auto store8 = [&](int tk, int head, int col, const float* vals, float scl) {
+      // 8 consecutive outputs of one row starting at column `col`.
+      if constexpr (OUT_F32) {
+        float* dst = static_cast<float*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD + col;
+        if (g.o_rows_32b) {
+          uint32_t u[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) u[e] = __float_as_uint(vals[e] * scl);
+          st_global_v8(dst, u);
+        } else {
+          *reinterpret_cast<float4*>(dst) = make_float4(vals[0] * scl, vals[1] * scl, vals[2] * scl, vals[3] * scl);
+          *reinterpret_cast<float4*>(dst + 4) = make_float4(vals[4] * scl, vals[5] * scl, vals[6] * scl, vals[7] * scl);
+        }
+      } else {
+        __nv_bfloat16* dst =
+            static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD + col;
+        uint4 u;
+        u.x = pack_bf16x2(vals[0] * scl, vals[1] * scl);
+        u.y = pack_bf16x2(vals[2] * scl, vals[3] * scl);
+        u.z = pack_bf16x2(vals[4] * scl, vals[5] * scl);
+        u.w = pack_bf16x2(vals[6] * scl, vals[7] * scl);
+        *reinterpret_cast<uint4*>(dst) = u;
+      }
+    };
+
+    // Epilogue of a finished tile: this thread's O columns and the row sum (column 64 of O)
+    // from TMEM, scaled by 1/rowsum, stored to the grid position of the query slot
+    // (padded slots dropped).
+    auto epilogue = [&](int pit, int head, int tok) -> bool {
+      const int k = fdiv(pit, g.div_heads);   // the CTA's window index (fused order)
+      const int wp = k & 1;
+      if constexpr (FUSED) {
+        // the window's buffers of this parity must have been normalised (window k - 2)
+        if (head == 0 && !__all_sync(0xffffffffu, mbar_wait_bounded(win_free(wp), ((k >> 1) & 1) ^ 1, limit_ns)))
+          return false;
+      }
+      bool ok = mbar_wait_bounded(o_full, pit & 1, limit_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) return false;
+      tc_fence_after();
+      float ov[HD / 2];
+      float l;
+      if (!is_tail) {
+#pragma unroll
+        for (int m = 0; m < HD / 32; ++m) tmem_ld16(o_base + 32 * m, ov + 16 * m);
+        tmem_ld1(o_base - 16 * half + kOnesCol, &l);
+      } else {
+#pragma unroll
+        for (int m = 0; m < HD / 32; ++m) tmem_ld_16x32bx2_x16(o_base + 32 * m, ov + 16 * m);
+        tmem_ld_16x32bx2_x1(o_base + kOnesCol, &l);
+      }
+      tmem_wait_ld();
+#pragma unroll
+      for (int m = 0; m < HD / 32; ++m) reg_fence16(ov + 16 * m);
+      reg_fence1(&l);
+      tc_fence_before();
+      mbar_arrive(o_empty);
+      const float inv = l > 0.f ? rcp_approx(l) : 0.f;
+      if constexpr (FUSED) {
+        fused_epilogue<HD>(g, fa, o, ov, inv, head, tok, row, half, wp, wstat, wtok, C);
+        if (head == g.heads - 1) {
+          __threadfence_block();
+          mbar_arrive(win_full(wp));   // this thread's share of the window is written
+        }
+        return true;
+      }
+      if (tok >= 0) {
+#pragma unroll
+        for (int m = 0; m < HD / 32; ++m) {
+          const int col = 32 * m + 16 * half;
+          if constexpr (!OUT_F32) {
+            if (g.o_rows_32b) {   // 16 bf16 = one 32-byte store
+              uint32_t u[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) u[e] = pack_bf16x2(ov[16 * m + 2 * e] * inv, ov[16 * m + 2 * e + 1] * inv);
+              st_global_v8(static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tok) * g.o_stride + head * HD + col, u);
+              continue;
+            }
+          }
+          store8(tok, head, col, ov + 16 * m, inv);
+          store8(tok, head, col + 8, ov + 16 * m + 8, inv);
+        }
+      }
+      return true;
+    };
 
     // The thread's 72 logits are read from TMEM once (nine 8-column loads) and stay in
     // registers.  If any thread of the warp has a masked key (near the shift seams and the
@@ -465,7 +667,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
       return fmaxf(a, b);
     };
     // exp2 and P (bf16) into the P blocks.  The row sum comes out of the PV MMA.
-    auto row_exp = [&](const float (&x)[72], float m, uint32_t pofs) {
+    auto row_exp = [&](const float (&x)[72], float m) {
       const float2 cc = make_float2(c, c), nm = make_float2(-m * c, -m * c);
       const uint32_t rsw = lrow & 7;
       const uint32_t row128 = static_cast<uint32_t>(lrow) * 128, row32 = static_cast<uint32_t>(lrow) * 32;
@@ -486,62 +688,86 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         const int g8 = 2 * k + half;   // 16-byte chunk of P along the keys
         uint32_t addr;
         if (k < 8)
-          addr = (k < 4 ? pb0 : pb1) + pofs + row128 + ((((g8 & 7) ^ rsw)) << 4);
+          addr = (k < 4 ? pb0 : pb1) + row128 + ((((g8 & 7) ^ rsw)) << 4);
         else
-          addr = pb2 + pofs + row32 + (((g8 - 16) ^ sw32) << 4);
+          addr = pb2 + row32 + (((g8 - 16) ^ sw32) << 4);
         asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(pk[0]), "r"(pk[1]), "r"(pk[2]),
                      "r"(pk[3])
                      : "memory");
       }
     };
 
+    // Iteration `it` does the softmax of tile `it` (if any) and then the epilogue of tile
+    // it-1, so the PV MMA of a tile overlaps the next tile's softmax.  One call site each.
     // S is read out of TMEM into registers in one go, so it is released (s_empty) before
     // the exponentials, and the MMA warp can compute the next tile's S underneath them.
-    for (long long tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
-      const int s = it % kStages;
-      const uint32_t ph = (it / kStages) & 1;
-      if (__any_sync(0xffffffffu, *abort_flag != 0)) {
-        aborted = true;
-        break;
-      }
-      bool ok = mbar_wait_bounded(table_bar(s), ph, limit_ns);
-      if (!__all_sync(0xffffffffu, ok)) {
-        aborted = true;
-        break;
-      }
-      const uint4 mq = tables[s].maskq[my_hi * 2 + half];
-      mbar_arrive(empty_bar(s));
-
-      ok = mbar_wait_bounded(s_full, it & 1, limit_ns);
-      if (!__all_sync(0xffffffffu, ok)) {
-        aborted = true;
-        break;
-      }
-      tc_fence_after();
-      float x[72];
-      const float mh = row_max(x, mq);
-      tc_fence_before();
-      mbar_arrive(s_empty);   // S of this thread is in registers: the next S may be written
-      const int par = it & 1;
-      float mrow;
-      if (!is_tail) {
-        xmax[(par * 2 + half) * 128 + row] = mh;
-        mbar_arrive(xmax_bar(par, half));
-        ok = mbar_wait_bounded(xmax_bar(par, half ^ 1), (it >> 1) & 1, limit_ns);
+    for (long long tile = cta_tile<FUSED>(g, 0);; tile = cta_tile<FUSED>(g, ++it)) {
+      const bool have_cur = tile >= 0;
+      int head = 0, tok = -1;
+      if (have_cur) {
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        if (__any_sync(0xffffffffu, *abort_flag != 0)) {
+          aborted = true;
+          break;
+        }
+        bool ok = mbar_wait_bounded(table_bar(s), ph, limit_ns);
         if (!__all_sync(0xffffffffu, ok)) {
           aborted = true;
           break;
         }
-        mrow = fmaxf(mh, xmax[(par * 2 + (half ^ 1)) * 128 + row]);
-      } else {
-        mrow = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 16));
+        head = static_cast<int>(tile) - fdiv(static_cast<int>(tile), g.div_heads) * g.heads;
+        const Table& tb = tables[s];
+        tok = tb.tok[row];
+        const uint4 mq = tb.maskq[my_hi * 2 + half];
+        mbar_arrive(empty_bar(s));
+
+        ok = mbar_wait_bounded(s_full, it & 1, limit_ns);
+        if (!__all_sync(0xffffffffu, ok)) {
+          aborted = true;
+          break;
+        }
+        tc_fence_after();
+        float x[72];
+        const float mh = row_max(x, mq);
+        tc_fence_before();
+        mbar_arrive(s_empty);   // S of this thread is in registers: the next S may be written
+        const int par = it & 1;
+        float mrow;
+        if (!is_tail) {
+          xmax[(par * 2 + half) * 128 + row] = mh;
+          mbar_arrive(xmax_bar(par, half));
+          ok = mbar_wait_bounded(xmax_bar(par, half ^ 1), (it >> 1) & 1, limit_ns);
+          if (!__all_sync(0xffffffffu, ok)) {
+            aborted = true;
+            break;
+          }
+          mrow = fmaxf(mh, xmax[(par * 2 + (half ^ 1)) * 128 + row]);
+        } else {
+          mrow = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 16));
+        }
+        if (mrow == -INFINITY) mrow = 0.f;
+        // P may only be overwritten once the previous tile's PV MMA has consumed it.
+        ok = mbar_wait_bounded(is_tail ? p_empty_t : p_empty, par ^ 1, limit_ns);
+        if (!__all_sync(0xffffffffu, ok)) {
+          aborted = true;
+          break;
+        }
+        row_exp(x, mrow);
+        fence_proxy_async_smem();
+        mbar_arrive(is_tail ? p_full_t : p_full);
       }
-      if (mrow == -INFINITY) mrow = 0.f;
-      // P goes to the tile's own stage (over its Q and K, consumed by S, which s_full
-      // guaranteed above): no wait for the previous tile's PV.
-      row_exp(x, mrow, static_cast<uint32_t>(s) * p_stage_step);
-      fence_proxy_async_smem();
-      mbar_arrive(is_tail ? p_full_t(par) : p_full(par));
+      if (have_prev) {
+        if (!epilogue(prev_it, prev_head, prev_tok)) {
+          aborted = true;
+          break;
+        }
+      }
+      if (!have_cur) break;
+      have_prev = true;
+      prev_it = it;
+      prev_head = head;
+      prev_tok = tok;
     }
     if (aborted) {
       if (lane == 0) record_error(err, kStatusTimeout);
@@ -555,15 +781,17 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
-template <int HD, bool OUT_F32>
+template <int HD, bool OUT_F32, bool FUSED>
 cudaError_t launch_t(const WinGeom& g, const TmaMaps& maps, void* o, int* err, long long limit_ns, int num_sms,
-                     cudaStream_t st) {
-  auto kern = window_attn_tc_kernel<HD, OUT_F32>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+                     const AdalnArgs& fa, cudaStream_t st) {
+  auto kern = window_attn_tc_kernel<HD, OUT_F32, FUSED>;
+  const int smem = FUSED ? kSmemAllocFused : kSmemAlloc;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const long long tiles = g.windows * g.heads;
-  const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-  kern<<<grid, kThreads, kSmemAlloc, st>>>(g, maps, o, err, static_cast<unsigned long long>(limit_ns < 0 ? 0 : limit_ns));
+  const long long units = FUSED ? g.windows : g.windows * g.heads;   // the fused kernel takes whole windows
+  const int grid = static_cast<int>(units < num_sms ? units : num_sms);
+  kern<<<grid, FUSED ? kThreadsFused : kThreads, smem, st>>>(
+      g, maps, o, err, static_cast<unsigned long long>(limit_ns < 0 ? 0 : limit_ns), fa);
   return cudaGetLastError();
 }
 
@@ -575,11 +803,27 @@ cudaError_t launch_window_attn_tc(const WinGeom& g, const void* q, const void* k
   const void* ptrs[3] = {q, k, v};
   cudaError_t e = make_maps(g, ptrs, false, &maps);
   if (e != cudaSuccess) return e;
+  const AdalnArgs none{};
   if (g.head_dim == 64)
-    return out_f32 ? launch_t<64, true>(g, maps, o, err, spin_limit, num_sms, stream)
-                   : launch_t<64, false>(g, maps, o, err, spin_limit, num_sms, stream);
-  return out_f32 ? launch_t<32, true>(g, maps, o, err, spin_limit, num_sms, stream)
-                 : launch_t<32, false>(g, maps, o, err, spin_limit, num_sms, stream);
+    return out_f32 ? launch_t<64, true, false>(g, maps, o, err, spin_limit, num_sms, none, stream)
+                   : launch_t<64, false, false>(g, maps, o, err, spin_limit, num_sms, none, stream);
+  return out_f32 ? launch_t<32, true, false>(g, maps, o, err, spin_limit, num_sms, none, stream)
+                 : launch_t<32, false, false>(g, maps, o, err, spin_limit, num_sms, none, stream);
+}
+
+cudaError_t launch_window_attn_adaln(const WinGeom& g, const void* q, const void* k, const void* v, void* o,
+                                     const AdalnArgs& fa, int* err, long long spin_limit, int num_sms,
+                                     cudaStream_t stream) {
+  TmaMaps maps;
+  const void* ptrs[3] = {q, k, v};
+  cudaError_t e = make_maps(g, ptrs, false, &maps);
+  if (e != cudaSuccess) return e;
+  if (g.head_dim == 64) return launch_t<64, false, true>(g, maps, o, err, spin_limit, num_sms, fa, stream);
+  return launch_t<32, false, true>(g, maps, o, err, spin_limit, num_sms, fa, stream);
+}
+
+int window_attn_adaln_grid(long long windows, int num_sms) {
+  return static_cast<int>(windows < num_sms ? windows : num_sms);
 }
 
 }  // namespace s3w

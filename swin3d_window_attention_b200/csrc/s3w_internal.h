@@ -12,6 +12,25 @@ cudaError_t launch_window_attn_tc(const WinGeom& g, const void* q, const void* k
                                   void* o, bool out_f32, int* err, long long spin_limit,
                                   int num_sms, cudaStream_t stream);
 
+// Arguments of the AdaLN half of the fused window attention + AdaLN kernel.
+struct AdalnArgs {
+  const float* residual;   // [B][L][C] fp32
+  const float* scale;      // [B][C] fp32
+  const float* shift;      // [B][C] fp32
+  void* out;               // [B][L][C], fp32 or bf16; may be residual itself
+  uint16_t* ws;            // workspace, per CTA 2 x 144 x C bf16 (window parity, slot, channel)
+  float eps;
+  int out_f32;
+};
+
+// Window attention fused with AdaLN + residual (attn_tcgen05.cu): o (bf16 attention output,
+// grid layout) is optional (nullptr: not written).
+cudaError_t launch_window_attn_adaln(const WinGeom& g, const void* q, const void* k, const void* v, void* o,
+                                     const AdalnArgs& fa, int* err, long long spin_limit, int num_sms,
+                                     cudaStream_t stream);
+// CTAs of the fused kernel (each takes whole windows); its workspace is grid x 2 x 144 x C bf16.
+int window_attn_adaln_grid(long long windows, int num_sms);
+
 // Window attention in the TF32_ACC_FP32 mode: fp32 Q/K/V, tcgen05 kind::tf32 (attn_tf32.cu).
 cudaError_t launch_window_attn_tf32(const WinGeom& g, const void* q, const void* k, const void* v,
                                     void* o, bool out_f32, int* err, long long spin_limit,

@@ -78,6 +78,12 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
 
+// Bulk prefetch of `bytes` (a multiple of 16) of global memory into L2, 16-byte aligned
+// address; no completion to wait for.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
@@ -281,15 +287,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
   const uint32_t a = __float_as_uint(lo) + 0x8000u;
   const uint32_t b = __float_as_uint(hi) + 0x8000u;
   return __byte_perm(a, b, 0x7632);
-}
-
-// Two finite fp32 values -> packed bf16x2 rounded to nearest, ties to even, on the integer
-// pipe: add 0x7fff plus the lowest kept bit to the bit pattern, keep the upper halves.
-__device__ __forceinline__ uint32_t pack_bf16x2_rne_int(float lo, float hi) {
-  const uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
-  const uint32_t ra = a + 0x7fffu + ((a >> 16) & 1u);
-  const uint32_t rb = b + 0x7fffu + ((b >> 16) & 1u);
-  return __byte_perm(ra, rb, 0x7632);
 }
 
 // 32-byte global store (one full sector per thread).

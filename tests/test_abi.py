@@ -111,6 +111,36 @@ def test_adaln_zero_tokens_is_a_no_op():
     assert _adaln(L=0, x=None, res=None, out=None) == api.S3W_OK
 
 
+def _fused(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, qs=512, res=FAKE, sc=FAKE, sh=FAKE, out=FAKE, outd=1, o=None, ws=FAKE,
+             wsb=1 << 30, B=1, T=4, H=12, W=24, wt=2, wh=6, ww=12, st=1, sh_=3, sw=6, heads=8, hd=64, scale=0.0,
+             eps=1e-5)
+    a.update(over)
+    return s3w.load_library().swin3d_window_attn_adaln_fwd(
+        a["q"], a["k"], a["v"], a["qs"], a["res"], a["sc"], a["sh"], a["out"], a["outd"], a["o"], a["ws"], a["wsb"],
+        a["B"], a["T"], a["H"], a["W"], a["wt"], a["wh"], a["ww"], a["st"], a["sh_"], a["sw"], a["heads"], a["hd"],
+        a["scale"], a["eps"], None)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(res=None), api.S3W_ERR_INVALID_ARG),
+    (dict(ws=None), api.S3W_ERR_INVALID_ARG),
+    (dict(q=None), api.S3W_ERR_INVALID_ARG),
+    (dict(eps=-1.0), api.S3W_ERR_INVALID_ARG),
+    (dict(outd=5), api.S3W_ERR_INVALID_ARG),
+    (dict(st=2), api.S3W_ERR_INVALID_ARG),                  # shift == window
+    (dict(hd=48, qs=384), api.S3W_ERR_UNSUPPORTED),
+    (dict(heads=80, qs=5120), api.S3W_ERR_UNSUPPORTED),     # C = 5120 > 4096
+    (dict(ws=FAKE + 16), api.S3W_ERR_MISALIGNED),           # workspace not 32-byte aligned
+    (dict(o=FAKE + 16), api.S3W_ERR_MISALIGNED),            # attention output not 32-byte aligned
+    (dict(out=FAKE + 16 * 512), api.S3W_ERR_INVALID_ARG),   # partial overlap of out with residual
+])
+def test_fused_rejects_bad_arguments_on_host(over, expect):
+    if "out" in over:
+        over = dict(over, res=FAKE + 64)
+    assert _fused(**over) == expect
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(api, "_lib", None)
     monkeypatch.setattr(api, "HERE", str(tmp_path))

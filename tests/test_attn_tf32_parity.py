@@ -1,10 +1,13 @@
 """GPU parity of the TF32_ACC_FP32 mode of swin3d_window_attn_fwd (fp32 Q/K/V) against the
 fp64 oracle, through the C ABI.
 
-Every operand the tensor cores read (Q, K, V and P) is TF32, whose unit roundoff 2^-11 is
-eight times finer than bf16's 2^-8, and accumulation is FP32.  The attention bar of the BF16
-path (max-abs 1e-2, relative L2 3e-3) is therefore an upper bound here; the TF32 bar below is
-derived in the design notes from the TF32 rounding of the four operands.
+Bar (fp32 output): max-abs 1e-2 and relative L2 2e-3.  Every operand the tensor cores read is
+TF32: Q, K and V as the MMA reads fp32 (relative error below 2^-10), P rounded to nearest
+(2^-11); accumulation is FP32.  A logit is scale * a sum of head_dim products: for N(0,1)
+inputs, head_dim 64 and scale 1/8 its error is about 1e-3 rms; the softmax carries it into P
+and O at about 1.4 times, so the expected relative L2 error of O is about 1e-3 (measured
+1.1e-3), and 2e-3 leaves a factor of two.  With bf16 output the output rounding (2^-9)
+dominates and the bar of the BF16 path applies (max-abs 1e-2, relative L2 3e-3).
 """
 import numpy as np
 import pytest
@@ -14,6 +17,13 @@ import oracle
 import swin3d_window_attention_b200 as s3w
 from swin3d_window_attention_b200 import inputs
 from tests.helpers import ATTN_MAX_ABS, ATTN_REL_L2, attn_errors, edge_window_ids
+
+TF32_MAX_ABS = 1e-2
+TF32_REL_L2 = 2e-3
+
+
+def bar(out_dtype):
+    return (TF32_MAX_ABS, TF32_REL_L2) if out_dtype == torch.float32 else (ATTN_MAX_ABS, ATTN_REL_L2)
 
 pytestmark = pytest.mark.gpu
 
@@ -59,7 +69,8 @@ def test_tf32_small_grids_full_compare(cuda_ok, case, out_dtype):
     ref = oracle.window_attn_grid(*host, heads, hd, window, shift)
     mx, rl2 = attn_errors(got, ref)
     print(f"tf32 {case_id(case)} {out_dtype}: max-abs {mx:.3e} rel-L2 {rl2:.3e}")
-    assert mx <= ATTN_MAX_ABS and rl2 <= ATTN_REL_L2, (mx, rl2)
+    mab, rlb = bar(out_dtype)
+    assert mx <= mab and rl2 <= rlb, (mx, rl2)
 
 
 def test_tf32_fused_qkv_buffer(cuda_ok):
@@ -74,7 +85,7 @@ def test_tf32_fused_qkv_buffer(cuda_ok):
     torch.cuda.synchronize()
     ref = oracle.window_attn_grid(*host, heads, hd, window, shift)
     mx, rl2 = attn_errors(o.cpu().numpy(), ref)
-    assert mx <= ATTN_MAX_ABS and rl2 <= ATTN_REL_L2, (mx, rl2)
+    assert mx <= TF32_MAX_ABS and rl2 <= TF32_REL_L2, (mx, rl2)
 
 
 @pytest.mark.parametrize("shift", [(1, 3, 6), (0, 0, 0)], ids=["shifted", "unshifted"])
@@ -96,7 +107,7 @@ def test_tf32_stage1_full_size_sampled(cuda_ok, shift):
     got = o.view(-1, C)[torch.from_numpy(tok[real]).cuda()].cpu().numpy()
     mx, rl2 = attn_errors(got, out[real])
     print(f"tf32 stage1 {shift}: max-abs {mx:.3e} rel-L2 {rl2:.3e}")
-    assert mx <= ATTN_MAX_ABS and rl2 <= ATTN_REL_L2, (mx, rl2)
+    assert mx <= TF32_MAX_ABS and rl2 <= TF32_REL_L2, (mx, rl2)
     assert not torch.any(o == SENTINEL)
     assert torch.isfinite(o).all()
     vmax = dev[2].abs().amax()
@@ -125,4 +136,4 @@ def test_tf32_bounded_wait_timeout(cuda_ok):
     assert s3w.poll_device_error() == 0
     ref = oracle.window_attn_grid(*host, heads, hd, window, shift)
     mx, rl2 = attn_errors(o.cpu().numpy(), ref)
-    assert mx <= ATTN_MAX_ABS and rl2 <= ATTN_REL_L2, (mx, rl2)
+    assert mx <= TF32_MAX_ABS and rl2 <= TF32_REL_L2, (mx, rl2)

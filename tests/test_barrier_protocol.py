@@ -36,7 +36,12 @@ class Bar:
             self.tile = None
 
 
-def model(ntiles, has_tail=True, variant="new", seed=0, max_steps=2_000_000):
+def model(ntiles, has_tail=True, variant="kernel", seed=0, max_steps=2_000_000):
+    """The BF16 kernel: 3 stages; one P buffer per row group (main rows, tail rows), handed to
+    the PV MMA on p_full / p_full_t and released on p_empty / p_empty_t; the softmax warps
+    finish tile t-1 (the epilogue) after handing over P(t).  variant="no_p_empty" drops the
+    release waits (P placed so that it would not need them) while keeping single hand-over
+    barriers: the combination that lets a warp lap another."""
     rng = random.Random(seed)
     n_soft_warps = 9 if has_tail else 8
     nsoft = 32 * n_soft_warps
@@ -45,20 +50,16 @@ def model(ntiles, has_tail=True, variant="new", seed=0, max_steps=2_000_000):
     def mk(name, count):
         B[name] = Bar(name, count)
 
-    nepi = 128
     for s in range(STAGES):
         mk(f"load{s}", 1)
-        mk(f"empty{s}", 1 + nsoft + nepi)
+        mk(f"empty{s}", 1 + nsoft)
         mk(f"table{s}", 32)
-    mk("s_full", 1)
-    mk("s_empty", nsoft)
-    for p in range(2):
-        mk(f"p_full{p}", 256)
-        mk(f"p_full_t{p}", 32)
+    for n, c in (("s_full", 1), ("s_empty", nsoft), ("p_full", 256), ("p_empty", 1), ("p_full_t", 32),
+                 ("p_empty_t", 1), ("o_full", 1), ("o_empty", nsoft)):
+        mk(n, c)
+    for par in range(2):
         for h in range(2):
-            mk(f"xmax{p}{h}", 128)
-    mk("o_full", 1)
-    mk("o_empty", nepi)
+            mk(f"xmax{par}{h}", 128)
 
     def tma():
         for it in range(ntiles):
@@ -82,53 +83,49 @@ def model(ntiles, has_tail=True, variant="new", seed=0, max_steps=2_000_000):
             if j > 0:
                 jt = j - 1
                 s = jt % STAGES
-                if variant == "single":
-                    yield ("wait", "p_full0", jt & 1, jt)
-                else:
-                    yield ("wait", f"p_full{jt & 1}", (jt >> 1) & 1, jt >> 1)
+                yield ("wait", "p_full", jt & 1, jt)
                 yield ("wait", "o_empty", (jt & 1) ^ 1, jt - 1)
+                yield ("commit", [("p_empty", jt)])
                 if has_tail:
-                    if variant == "single":
-                        yield ("wait", "p_full_t0", jt & 1, jt)
-                    else:
-                        yield ("wait", f"p_full_t{jt & 1}", (jt >> 1) & 1, jt >> 1)
+                    yield ("wait", "p_full_t", jt & 1, jt)
+                    yield ("commit", [("p_empty_t", jt)])
                 yield ("commit", [("o_full", jt), (f"empty{s}", jt)])
 
     def softmax(w):
         tail = w == 8
         half = 0 if tail else (w >> 2) & 1
-        for it in range(ntiles):
-            s = it % STAGES
-            yield ("wait", f"table{s}", (it // STAGES) & 1, it // STAGES)
-            yield ("arrive", f"empty{s}", it, 32)
-            yield ("wait", "s_full", it & 1, it)
-            yield ("arrive", "s_empty", it, 32)
-            par = it & 1
-            if not tail:
-                yield ("arrive", f"xmax{par}{half}", it, 32)
-                yield ("wait", f"xmax{par}{half ^ 1}", (it >> 1) & 1, it >> 1)
-            pp = 0 if variant == "single" else par
-            yield ("arrive", f"p_full_t{pp}" if tail else f"p_full{pp}", it, 32)
-
-    def epilogue():
-        # the four epilogue warps (warps 12..15): tokens from the table, then O
-        for it in range(ntiles):
-            s = it % STAGES
-            yield ("wait", f"table{s}", (it // STAGES) & 1, it // STAGES)
-            yield ("arrive", f"empty{s}", it, 32)
-            yield ("wait", "o_full", it & 1, it)
-            yield ("arrive", "o_empty", it, 32)
+        prev = None
+        for it in range(ntiles + 1):
+            if it < ntiles:
+                s = it % STAGES
+                yield ("wait", f"table{s}", (it // STAGES) & 1, it // STAGES)
+                yield ("arrive", f"empty{s}", it, 32)
+                yield ("wait", "s_full", it & 1, it)
+                yield ("arrive", "s_empty", it, 32)
+                if not tail:
+                    par = it & 1
+                    yield ("arrive", f"xmax{par}{half}", it, 32)
+                    yield ("wait", f"xmax{par}{half ^ 1}", (it >> 1) & 1, it >> 1)
+                if variant != "no_p_empty":
+                    yield ("wait", "p_empty_t" if tail else "p_empty", (it & 1) ^ 1, it - 1)
+                yield ("arrive", "p_full_t" if tail else "p_full", it, 32)
+            if prev is not None:
+                yield ("wait", "o_full", prev & 1, prev)
+                yield ("arrive", "o_empty", prev, 32)
+            if it < ntiles:
+                prev = it
 
     actors = {"tma": tma(), "table": table(), "mma": mma()}
     for w in range(n_soft_warps):
         actors[f"w{w}"] = softmax(w)
-    for e in range(4):
-        actors[f"epi{e}"] = epilogue()
+    return run(actors, B, rng, max_steps)
+
+
+def run(actors, B, rng, max_steps):
+    """Random interleaving of the actors with in-order tensor-core and TMA completion streams."""
     cur = {k: None for k in actors}
-    asyncq = []          # in-order tensor-core completions: (bar, tile)
-    tmaq = []            # TMA completions (in order among themselves)
+    asyncq, tmaq, finished = [], [], set()
     weight = {k: rng.choice([0.05, 0.3, 1.0, 1.0, 3.0]) for k in actors}
-    finished = set()
     steps = 0
     while len(finished) < len(actors) or asyncq or tmaq:
         steps += 1
@@ -146,8 +143,7 @@ def model(ntiles, has_tail=True, variant="new", seed=0, max_steps=2_000_000):
             op = cur[k]
             if op[0] == "wait":
                 b = B[op[1]]
-                ok = (b.done & 1) != op[2]
-                if ok:
+                if (b.done & 1) != op[2]:
                     assert b.done == op[3] + 1, f"{k}: wait on {op[1]} for phase {op[3]} passed with {b.done} done"
                 else:
                     assert b.done == op[3], f"{k}: wait on {op[1]} for phase {op[3]} blocked with {b.done} done"
@@ -158,7 +154,6 @@ def model(ntiles, has_tail=True, variant="new", seed=0, max_steps=2_000_000):
             break
         if not choices:
             raise AssertionError("deadlock: " + ", ".join(f"{k}:{cur[k]}" for k in actors if k not in finished))
-        # per-actor speeds drawn per seed, to provoke races
         k = rng.choices(choices, weights=[weight.get(c, 0.5) for c in choices])[0]
         if k in ("async", "tmaq"):
             q = asyncq if k == "async" else tmaq
@@ -249,52 +244,7 @@ def model_tf32(ntiles, has_tail=True, seed=0, max_steps=2_000_000):
     actors = {"tma": tma(), "table": table(), "mma": mma()}
     for w in range(nw):
         actors[f"w{w}"] = softmax(w)
-    cur = {k: None for k in actors}
-    asyncq, tmaq, finished = [], [], set()
-    weight = {k: rng.choice([0.05, 0.3, 1.0, 1.0, 3.0]) for k in actors}
-    steps = 0
-    while len(finished) < len(actors) or asyncq or tmaq:
-        steps += 1
-        assert steps < max_steps
-        runnable = []
-        for k, g in actors.items():
-            if k in finished:
-                continue
-            if cur[k] is None:
-                try:
-                    cur[k] = next(g)
-                except StopIteration:
-                    finished.add(k)
-                    continue
-            op = cur[k]
-            if op[0] == "wait":
-                b = B[op[1]]
-                if (b.done & 1) != op[2]:
-                    assert b.done == op[3] + 1, f"{k}: wait {op[1]} phase {op[3]} passed with {b.done}"
-                else:
-                    assert b.done == op[3], f"{k}: wait {op[1]} phase {op[3]} blocked with {b.done}"
-                    continue
-            runnable.append(k)
-        choices = runnable + (["async"] if asyncq else []) + (["tmaq"] if tmaq else [])
-        if not choices and len(finished) == len(actors):
-            break
-        if not choices:
-            raise AssertionError("deadlock: " + ", ".join(f"{k}:{cur[k]}" for k in actors if k not in finished))
-        k = rng.choices(choices, weights=[weight.get(c, 0.5) for c in choices])[0]
-        if k in ("async", "tmaq"):
-            q = asyncq if k == "async" else tmaq
-            bar, tile = q.pop(0)
-            B[bar].arrive(tile)
-            continue
-        op = cur[k]
-        cur[k] = None
-        if op[0] == "arrive":
-            B[op[1]].arrive(op[2], op[3])
-        elif op[0] == "commit":
-            asyncq.extend(op[1])
-        elif op[0] == "tma":
-            tmaq.append((op[1], op[2]))
-
+    return run(actors, B, rng, max_steps)
 
 
 def test_bf16_protocol_holds_under_random_schedules():
@@ -303,13 +253,14 @@ def test_bf16_protocol_holds_under_random_schedules():
             model(ntiles=1 + seed % 13, has_tail=tail, seed=seed)
 
 
-def test_single_barrier_variant_is_caught():
-    """Without per-parity hand-over barriers a warp can lap another (the protocol this
-    replaced): the model must find it."""
+def test_dropping_the_p_release_wait_is_caught():
+    """Without the p_empty waits a softmax warp can arrive for tile t+1 before another has
+    arrived for tile t, and the tail warp can complete tile t+1's P before the MMA warp has
+    waited for tile t's: the model must find it."""
     fails = 0
     for seed in range(60):
         try:
-            model(ntiles=2 + seed % 12, has_tail=True, variant="single", seed=seed)
+            model(ntiles=2 + seed % 12, has_tail=True, variant="no_p_empty", seed=seed)
         except AssertionError:
             fails += 1
     assert fails > 0
