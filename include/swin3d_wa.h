@@ -183,6 +183,41 @@ int swin3d_window_attn_adaln_fwd(const void* q, const void* k, const void* v, lo
 long long swin3d_window_attn_adaln_workspace_bytes(int B, int T, int H, int W, int win_t, int win_h, int win_w,
                                                    int heads, int head_dim);
 
+/* Size of the library's static workspace of swin3d_window_attn_adaln_fwd_static_ws: 48 MiB,
+ * the two-window workspace of 148 CTAs at C = 512 (43.6 MB) with room to spare. */
+#define S3W_ADALN_STATIC_WORKSPACE_BYTES (48ll << 20)
+
+/*
+ * swin3d_window_attn_adaln_fwd without a caller-supplied workspace, for callers that cannot
+ * allocate device memory.  The paper has no counterpart: this is a deployment variant of
+ * the fused call above, with the same arguments minus `workspace` and `workspace_bytes`, the
+ * same semantics and the same results.
+ *
+ * The workspace is a file-scope device array of S3W_ADALN_STATIC_WORKSPACE_BYTES bytes in
+ * the library (one per device, its address looked up once per device on first use).  The
+ * call allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ * Nothing in the array has to start at zero and the call clears nothing: every workspace
+ * byte the kernel reads was written earlier in the same launch.
+ *
+ * Every call on a device shares the one array.  Calls that overlap on the GPU (on different
+ * streams, or from different host threads without ordering between their streams) race on
+ * it and their outputs are undefined; calls in one stream are ordered and safe.
+ *
+ * Returns S3W_ERR_UNSUPPORTED, launching nothing, when the grid needs more workspace than
+ * the array holds (swin3d_window_attn_adaln_workspace_bytes(...) >
+ * S3W_ADALN_STATIC_WORKSPACE_BYTES; e.g. C = 1024 on 148 SMs needs 87.3 MB), S3W_ERR_CUDA if
+ * the array's address cannot be obtained, and otherwise what swin3d_window_attn_adaln_fwd
+ * returns for the same arguments.
+ */
+int swin3d_window_attn_adaln_fwd_static_ws(const void* q, const void* k, const void* v, long long qkv_token_stride,
+                                           const float* residual, const float* adaln_scale, const float* adaln_shift,
+                                           void* out, int out_dtype, void* o,
+                                           int B, int T, int H, int W,
+                                           int win_t, int win_h, int win_w,
+                                           int shift_t, int shift_h, int shift_w,
+                                           int heads, int head_dim, float attn_scale, float eps,
+                                           s3w_stream_t stream);
+
 /* Static English text for a status code (never NULL). */
 const char* s3w_status_string(int status);
 

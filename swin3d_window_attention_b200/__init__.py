@@ -14,6 +14,7 @@ from .api import (  # noqa: F401
     set_wait_limit_ns,
     status_string,
     swin3d_window_attn_adaln_fwd,
+    swin3d_window_attn_adaln_fwd_static_ws,
     swin3d_window_attn_fwd,
     swin3d_window_attn_fwd_legacy_mma,
     window_attn_adaln_workspace_bytes,

@@ -60,6 +60,8 @@ def load_library():
     lib.swin3d_window_attn_adaln_fwd.restype = I
     lib.swin3d_window_attn_adaln_workspace_bytes.argtypes = [I] * 9
     lib.swin3d_window_attn_adaln_workspace_bytes.restype = LL
+    lib.swin3d_window_attn_adaln_fwd_static_ws.argtypes = [P, P, P, LL, P, P, P, P, I, P] + [I] * 12 + [F, F, P]
+    lib.swin3d_window_attn_adaln_fwd_static_ws.restype = I
     _lib = lib
     return lib
 
@@ -174,6 +176,37 @@ def swin3d_window_attn_adaln_fwd(q, k, v, residual, scale, shift, out, heads: in
                                           float(eps), st)
     if check and rc != S3W_OK:
         raise S3WError(rc, "swin3d_window_attn_adaln_fwd")
+    return rc
+
+
+def swin3d_window_attn_adaln_fwd_static_ws(q, k, v, residual, scale, shift, out, heads: int, head_dim: int,
+                                           window=(2, 6, 12), shift_=(0, 0, 0), o=None, eps: float = 1e-5,
+                                           attn_scale: float = 0.0, stream=None, check: bool = True) -> int:
+    """The fused call on the library's static workspace: allocates nothing, here or in the
+    library.  Same arguments and results as :func:`swin3d_window_attn_adaln_fwd` without
+    ``workspace``; every call on a device shares the one workspace, so calls must not overlap
+    on the GPU."""
+    import torch
+
+    lib = load_library()
+    C = heads * head_dim
+    B, T, H, W = q.shape[:4]
+    ts = _token_stride(q, C)
+    if _token_stride(k, C) != ts or _token_stride(v, C) != ts:
+        raise ValueError("q, k and v must share one token stride")
+    for t in (residual, out):
+        if not t.is_contiguous() or t.numel() != B * T * H * W * C:
+            raise ValueError("residual and out must be contiguous [B, L, C]")
+    if o is not None and (not o.is_contiguous() or o.dtype != torch.bfloat16 or tuple(o.shape) != (B, T, H, W, C)):
+        raise ValueError("o must be a contiguous bf16 [B, T, H, W, C] tensor")
+    st = _stream_of(q) if stream is None else stream
+    rc = lib.swin3d_window_attn_adaln_fwd_static_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(), ts, residual.data_ptr(),
+                                                    scale.data_ptr(), shift.data_ptr(), out.data_ptr(),
+                                                    _dtype_code(out), None if o is None else o.data_ptr(),
+                                                    B, T, H, W, *window, *shift_, heads, head_dim, float(attn_scale),
+                                                    float(eps), st)
+    if check and rc != S3W_OK:
+        raise S3WError(rc, "swin3d_window_attn_adaln_fwd_static_ws")
     return rc
 
 
