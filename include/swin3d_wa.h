@@ -154,10 +154,10 @@ int adaln_residual_fwd(const void* x, int x_dtype, const float* residual,
  *
  * q, k, v, qkv_token_stride, the grid, window, shift, heads, head_dim (32 or 64) and
  *              attn_scale: as swin3d_window_attn_fwd; BF16 inputs only.
- * residual     device fp32 [B][T*H*W][C], C = heads * head_dim (C % 8 == 0, C <= 4096).
- * adaln_scale, adaln_shift  device fp32 [B][C].
- * out          device, out_dtype (S3W_F32 or S3W_BF16), [B][T*H*W][C]; may alias residual
- *              exactly (in-place update of the residual stream).
+ * residual     device fp32 [B][T*H*W][C], C = heads * head_dim (C <= 4096), 32-byte aligned.
+ * adaln_scale, adaln_shift  device fp32 [B][C], 32-byte aligned.
+ * out          device, out_dtype (S3W_F32 or S3W_BF16), [B][T*H*W][C], 32-byte aligned; may
+ *              alias residual exactly (in-place update of the residual stream).
  * o            optional device bf16 [B][T][H][W][C] (token stride C), 32-byte aligned: when
  *              non-NULL the attention output is written there too; NULL skips it.
  * workspace    device memory of at least swin3d_window_attn_adaln_workspace_bytes(...) bytes

@@ -222,8 +222,10 @@ int swin3d_window_attn_adaln_fwd(const void* q, const void* k, const void* v, lo
                          head_dim, qkv_token_stride, C, attn_scale, S3W_BF16, S3W_BF16, &g);
   if (rc != S3W_OK) return rc;
   if (C % 8 != 0 || C > 4096) return S3W_ERR_UNSUPPORTED;
-  if (!aligned16(residual) || !aligned16(adaln_scale) || !aligned16(adaln_shift) || !aligned16(out) ||
-      (reinterpret_cast<uintptr_t>(workspace) & 31u) != 0 || (o && (reinterpret_cast<uintptr_t>(o) & 31u) != 0))
+  // the AdaLN part moves 32-byte vectors of every one of these
+  auto aligned32 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; };
+  if (!aligned32(residual) || !aligned32(adaln_scale) || !aligned32(adaln_shift) || !aligned32(out) ||
+      !aligned32(workspace) || (o && !aligned32(o)))
     return S3W_ERR_MISALIGNED;
   // out may alias residual exactly; any other overlap with residual is rejected
   const long long n = static_cast<long long>(B) * T * H * W * C;

@@ -58,7 +58,10 @@ namespace {
 using namespace sm100;
 using namespace attn;
 
-constexpr int kStages = 3;
+// Stages of the Q/K/V ring: three for the attention kernel; two in the fused kernel, whose
+// AdaLN warps stream their rows through the shared memory the third stage would take.
+constexpr int kStagesPlain = 3;
+constexpr int kStagesFused = 2;
 constexpr int kTileBytes = kChunkTileBytes;         // 18432: one of Q / K / V
 constexpr int kStageBytes = 3 * kTileBytes;         // 55296
 
@@ -72,37 +75,40 @@ constexpr int OFF_P0B0 = 5120;     // P rows 0..127, keys 0..63
 constexpr int OFF_P0B1 = OFF_P0B0 + 16384;
 constexpr int OFF_P0B2 = OFF_P0B1 + 16384;   // keys 128..143, 32B swizzle, 4 KB
 constexpr int OFF_STAGE = OFF_P0B2 + 4096;   // 41984 (1024-aligned)
-// 16 key rows of bf16 ones in the V operand's layout: the PV MMA reads them as 16 more
-// output columns (through the descriptor's leading byte offset), so every such column of O
-// is the row sum of P as rounded to bf16, the exact normaliser of the P the MMA used.
-constexpr int OFF_ONES = OFF_STAGE + kStages * kStageBytes;
 constexpr int kOnesBytes = 16 * kRowBytes;
-constexpr int OFF_TABLE = OFF_ONES + kOnesBytes;
-
-constexpr int OFF_SLOTC = OFF_TABLE + kStages * kTableBytes;
-constexpr int OFF_BARS = OFF_SLOTC + kSlotConstBytes;
-// barriers: load[3] (TMA bytes), empty[3], table[3], s_full, s_empty, p_full, p_empty,
-// o_full, o_empty, drain, row max written[0][2], tail p_full, tail p_empty, row max
-// written[1][2] (row max barriers: [tile parity][key half]).  A softmax thread releases S (s_empty) before it waits for the other half's row
-// maximum, so the warps of one half can reach tile t+2 before a warp of the other half has
-// waited for tile t; one row-max barrier per tile parity keeps that wait on its own phase.
-constexpr int kNumBars = 3 * kStages + 13;
-// Row max of each key half of the main rows, exchanged between the two warps that share a
-// row: [tile parity][key half][row].
-constexpr int OFF_XCHG = OFF_BARS + kNumBars * 8;
 constexpr int kXchgFloats = 2 * 2 * 128;
-constexpr int OFF_MISC = OFF_XCHG + kXchgFloats * 4;   // tmem address, abort flag, producer stop
-constexpr int kSmemBytes = OFF_MISC + 16;
-constexpr int kSmemAlloc = kSmemBytes + 1024;       // slack for the 1024-byte alignment
-static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
-// Fused attention + AdaLN only: per window parity, the running statistics of every row's two
-// column halves, the rows' grid tokens, and the window-ready / window-free barriers.
-constexpr int OFF_WSTAT = kSmemBytes;                         // float2 [2 parity][2 half][kN]
-constexpr int OFF_WTOK = OFF_WSTAT + 2 * 2 * kN * 8;          // int [2 parity][kN]
-constexpr int OFF_WBAR = OFF_WTOK + 2 * kN * 4;               // win_full[2], win_free[2]
-constexpr int kSmemBytesFused = OFF_WBAR + 4 * 8;
-constexpr int kSmemAllocFused = kSmemBytesFused + 1024;
-static_assert(kSmemAllocFused <= 232448, "shared memory per CTA (fused)");
+
+template <bool FUSED>
+struct SmemLayout {
+  static constexpr int kStages = FUSED ? kStagesFused : kStagesPlain;
+  // 16 key rows of bf16 ones in the V operand's layout: the PV MMA reads them as 16 more
+  // output columns (through the descriptor's leading byte offset), so every such column of
+  // O is the row sum of P as rounded to bf16, the exact normaliser of the P the MMA used.
+  static constexpr int OFF_ONES = OFF_STAGE + kStages * kStageBytes;
+  static constexpr int OFF_TABLE = OFF_ONES + kOnesBytes;
+  static constexpr int OFF_SLOTC = OFF_TABLE + kStages * kTableBytes;
+  static constexpr int OFF_BARS = OFF_SLOTC + kSlotConstBytes;
+  // barriers: load[S] (TMA bytes), empty[S], table[S], s_full, s_empty, p_full, p_empty,
+  // o_full, o_empty, drain, row max written[0][2], tail p_full, tail p_empty, row max
+  // written[1][2] (row max barriers: [tile parity][key half]).  A softmax thread releases S
+  // (s_empty) before it waits for the other half's row maximum, so the warps of one half
+  // can reach tile t+2 before a warp of the other half has waited for tile t; one row-max
+  // barrier per tile parity keeps that wait on its own phase.
+  static constexpr int kNumBars = 3 * kStages + 13;
+  // Row max of each key half of the main rows, exchanged between the two warps that share
+  // a row: [tile parity][key half][row].
+  static constexpr int OFF_XCHG = OFF_BARS + kNumBars * 8;
+  static constexpr int OFF_MISC = OFF_XCHG + kXchgFloats * 4;   // tmem address, abort flag, producer stop
+  static constexpr int kPlainBytes = OFF_MISC + 16;
+  // Fused attention + AdaLN only: per window parity, the running statistics of every row's
+  // two column halves, the rows' grid tokens, and the window-ready / window-free barriers.
+  static constexpr int OFF_WSTAT = kPlainBytes;                  // float2 [2 parity][2 half][kN]
+  static constexpr int OFF_WTOK = OFF_WSTAT + 2 * 2 * kN * 8;     // int [2 parity][kN]
+  static constexpr int OFF_WBAR = OFF_WTOK + 2 * kN * 4;          // win_full[2], win_free[2]
+  static constexpr int kBytes = FUSED ? OFF_WBAR + 4 * 8 : kPlainBytes;
+  static constexpr int kAlloc = kBytes + 1024;                    // slack for the 1024-byte alignment
+  static_assert(kAlloc <= 232448, "shared memory per CTA");
+};
 
 // TMEM columns (fp32 accumulators, lane = row).  Every MMA destination is 32-aligned.  O
 // has 80 columns: the head's outputs (the first head_dim of 64), then from column 64 on 16
@@ -188,44 +194,77 @@ __device__ __forceinline__ void fused_epilogue(const WinGeom& g, const AdalnArgs
 }
 
 // The AdaLN warps (warps 12..15): per finished window, warp q normalises rows q, q + 4, ...,
-// two rows per pass; lane l takes the 8-channel groups l and l + 32 of each pass (then
-// l + 64, l + 96, ... for wider rows).  Every load of a pass is issued before its first
-// store (the output may be the residual itself, so the compiler could not reorder them),
-// and the residual rows kPrefetchPasses passes ahead are prefetched into L2, so a pass
-// costs about one L2 round trip.  The two column halves' running statistics of a row
-// combine into the row's mean and variance (biased, over C).
+// two rows per pass; lane l owns the 16-channel blocks l, l + 32, ... of each row.  A block
+// moves with one 32-byte load of x (bf16, from the workspace), two of the residual and one
+// or two 32-byte stores, and the per-channel factors 1 + scale and shift of a lane's block
+// stay in registers for the whole window when each lane has at most one block (C <= 512):
+// the warps' global loads and stores share the SM's memory-instruction queue with the
+// softmax warps' shared- and tensor-memory traffic, so the fewer of them the better.  Every
+// load of a pass is issued before its first store (the output may be the residual itself,
+// so the compiler could not reorder them).  The two column halves' running statistics of a
+// row combine into the row's mean and variance (biased, over C); then, per element,
+//   y = x * g + (r + shift - mean * g),   g = rstd * (1 + scale),
+// in packed two-lane fp32 arithmetic.
 // wbar0: the window barriers, win_full[2] then win_free[2].
-constexpr int kPrefetchPasses = 3;
+struct AdalnBlockIn {
+  uint32_t x[8];    // 16 bf16 of x
+  uint32_t r[16];   // 16 fp32 of the residual (bit patterns)
+};
 
-__device__ __forceinline__ void adaln_group(const AdalnArgs& fa, const float* scb, const float* shb, int tok, int cg,
-                                            float mean, float rstd, const uint4 xv, const float4 r0, const float4 r1,
-                                            int C) {
-  const float4 a0 = __ldg(reinterpret_cast<const float4*>(scb + cg * 8));
-  const float4 a1 = __ldg(reinterpret_cast<const float4*>(scb + cg * 8 + 4));
-  const float4 c0 = __ldg(reinterpret_cast<const float4*>(shb + cg * 8));
-  const float4 c1 = __ldg(reinterpret_cast<const float4*>(shb + cg * 8 + 4));
-  const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-  const float rr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-  const float sc[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-  const float sh[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-  float y[8];
+__device__ __forceinline__ void adaln_block_load(const uint16_t* xrow, const float* rrow, int cb, AdalnBlockIn& in) {
+  ld_global_v8(xrow + cb * 16, in.x);
+  uint32_t (&r0)[8] = *reinterpret_cast<uint32_t(*)[8]>(&in.r[0]);
+  uint32_t (&r1)[8] = *reinterpret_cast<uint32_t(*)[8]>(&in.r[8]);
+  ld_global_cs_v8(rrow + cb * 16, r0);
+  ld_global_cs_v8(rrow + cb * 16 + 8, r1);
+}
+
+__device__ __forceinline__ void adaln_block_store(const AdalnArgs& fa, int tok, int cb, int C, float mean, float rstd,
+                                                  const AdalnBlockIn& in, const float (&sc1)[16],
+                                                  const float (&sh)[16]) {
+  const float2 rs = make_float2(rstd, rstd), nm = make_float2(-mean, -mean);
+  float y[16];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const float x = (e & 1) ? __uint_as_float(xw[e >> 1] & 0xffff0000u) : __uint_as_float(xw[e >> 1] << 16);
-    y[e] = rr[e] + (x - mean) * rstd * (1.0f + sc[e]) + sh[e];
+  for (int e = 0; e < 16; e += 2) {
+    const uint32_t u = in.x[e >> 1];
+    const float2 x = make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+    const float2 gg = mul2(rs, make_float2(sc1[e], sc1[e + 1]));
+    const float2 bb = fma2(nm, gg, make_float2(sh[e], sh[e + 1]));
+    const float2 t = add2(make_float2(__uint_as_float(in.r[e]), __uint_as_float(in.r[e + 1])), bb);
+    const float2 yy = fma2(x, gg, t);
+    y[e] = yy.x;
+    y[e + 1] = yy.y;
   }
   if (fa.out_f32) {
-    float* op = static_cast<float*>(fa.out) + static_cast<long long>(tok) * C + cg * 8;
-    __stcs(reinterpret_cast<float4*>(op), make_float4(y[0], y[1], y[2], y[3]));
-    __stcs(reinterpret_cast<float4*>(op + 4), make_float4(y[4], y[5], y[6], y[7]));
+    float* op = static_cast<float*>(fa.out) + static_cast<long long>(tok) * C + cb * 16;
+    uint32_t v0[8], v1[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      v0[e] = __float_as_uint(y[e]);
+      v1[e] = __float_as_uint(y[8 + e]);
+    }
+    st_global_cs_v8(op, v0);
+    st_global_cs_v8(op + 8, v1);
   } else {
-    uint4 uo;
-    uo.x = pack_bf16x2(y[0], y[1]);
-    uo.y = pack_bf16x2(y[2], y[3]);
-    uo.z = pack_bf16x2(y[4], y[5]);
-    uo.w = pack_bf16x2(y[6], y[7]);
-    __stcs(reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(fa.out) + static_cast<long long>(tok) * C + cg * 8),
-           uo);
+    uint32_t v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = pack_bf16x2(y[2 * e], y[2 * e + 1]);
+    st_global_cs_v8(static_cast<__nv_bfloat16*>(fa.out) + static_cast<long long>(tok) * C + cb * 16, v);
+  }
+}
+
+__device__ __forceinline__ void adaln_factors(const float* scb, const float* shb, int cb, float (&sc1)[16],
+                                              float (&sh)[16]) {
+  uint32_t a[8], b[8];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    ld_global_v8(scb + cb * 16 + 8 * h, a);
+    ld_global_v8(shb + cb * 16 + 8 * h, b);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      sc1[8 * h + e] = 1.0f + __uint_as_float(a[e]);
+      sh[8 * h + e] = __uint_as_float(b[e]);
+    }
   }
 }
 
@@ -236,7 +275,8 @@ __device__ __forceinline__ void adaln_warps(const WinGeom& g, const AdalnArgs& f
   auto win_free = [&](int wp) { return wbar0 + 8u * (2 + wp); };
   const int q = warp - kFirstAdalnWarp;
   const float nh = 0.5f * static_cast<float>(C);   // values per column half of a row
-  const int ng = C >> 3;                            // 8-channel groups per row
+  const int nb = C >> 4;                            // 16-channel blocks per row
+  const bool hoisted = nb <= 32;                    // at most one block per lane
   bool aborted = false;
   for (int k = 0;; ++k) {
     const long long win = blockIdx.x + static_cast<long long>(k) * gridDim.x;
@@ -246,37 +286,31 @@ __device__ __forceinline__ void adaln_warps(const WinGeom& g, const AdalnArgs& f
       aborted = true;
       break;
     }
+    const long long b = fdiv(static_cast<int>(win), g.div_per_sample);
+    const float* scb = fa.scale + b * C;
+    const float* shb = fa.shift + b * C;
+    float sc1[16], sh[16];
+    if (hoisted && lane < nb) adaln_factors(scb, shb, lane, sc1, sh);
     if (!__all_sync(0xffffffffu, mbar_wait_bounded(win_full(wp), (k >> 1) & 1, limit_ns))) {
       aborted = true;
       break;
     }
-    const long long b = fdiv(static_cast<int>(win), g.div_per_sample);
-    const float* scb = fa.scale + b * C;
-    const float* shb = fa.shift + b * C;
     const uint16_t* wsw = fa.ws + (static_cast<long long>(blockIdx.x) * 2 + wp) * kN * C;
     const int* tokw = wtok + wp * kN;
     // this warp's rows: j-th row q + 4j; rows at or beyond the window size are padding
     // slots (rows 128.. exist only with a tail warp)
     const int nrows = g.N > q ? (g.N - q + 3) / 4 : 0;
-    auto prefetch_row = [&](int j) {
-      if (j < nrows) {
-        const int tok = tokw[q + 4 * j];
-        if (tok >= 0) bulk_prefetch_l2(fa.residual + static_cast<long long>(tok) * C, static_cast<uint32_t>(C) * 4u);
-      }
+    auto stats = [&](int r, float& mean, float& rstd) {
+      const float2 s0 = wstat[(wp * 2 + 0) * kN + r], s1 = wstat[(wp * 2 + 1) * kN + r];
+      const float d = s1.x - s0.x;
+      mean = 0.5f * (s0.x + s1.x);
+      const float var = (s0.y + s1.y + d * d * (0.5f * nh)) / static_cast<float>(C);
+      rstd = 1.0f / sqrtf(var + fa.eps);
     };
-    if (lane < 2 * kPrefetchPasses) prefetch_row(lane);
     for (int j = 0; j < nrows; j += 2) {
-      if (lane < 2) prefetch_row(j + 2 * kPrefetchPasses + lane);
       const int ra = q + 4 * j, rb = ra + 4;
       const int ta = tokw[ra];
       const int tb = j + 1 < nrows ? tokw[rb] : -1;
-      auto stats = [&](int r, float& mean, float& rstd) {
-        const float2 s0 = wstat[(wp * 2 + 0) * kN + r], s1 = wstat[(wp * 2 + 1) * kN + r];
-        const float d = s1.x - s0.x;
-        mean = 0.5f * (s0.x + s1.x);
-        const float var = (s0.y + s1.y + d * d * (0.5f * nh)) / static_cast<float>(C);
-        rstd = 1.0f / sqrtf(var + fa.eps);
-      };
       float ma = 0.f, sa = 0.f, mb = 0.f, sb = 0.f;
       if (ta >= 0) stats(ra, ma, sa);
       if (tb >= 0) stats(rb, mb, sb);
@@ -285,39 +319,13 @@ __device__ __forceinline__ void adaln_warps(const WinGeom& g, const AdalnArgs& f
       const uint16_t* xa = wsw + static_cast<long long>(ra) * C;
       const uint16_t* xb = wsw + static_cast<long long>(rb) * C;
 #pragma unroll 1
-      for (int c0 = lane; c0 < ng; c0 += 64) {
-        const int c1 = c0 + 32;
-        const bool h1 = c1 < ng;
-        uint4 xa0{}, xa1{}, xb0{}, xb1{};
-        float4 ra00{}, ra01{}, ra10{}, ra11{}, rb00{}, rb01{}, rb10{}, rb11{};
-        if (ta >= 0) {
-          xa0 = *reinterpret_cast<const uint4*>(xa + c0 * 8);
-          ra00 = __ldcs(reinterpret_cast<const float4*>(resa + c0 * 8));
-          ra01 = __ldcs(reinterpret_cast<const float4*>(resa + c0 * 8 + 4));
-          if (h1) {
-            xa1 = *reinterpret_cast<const uint4*>(xa + c1 * 8);
-            ra10 = __ldcs(reinterpret_cast<const float4*>(resa + c1 * 8));
-            ra11 = __ldcs(reinterpret_cast<const float4*>(resa + c1 * 8 + 4));
-          }
-        }
-        if (tb >= 0) {
-          xb0 = *reinterpret_cast<const uint4*>(xb + c0 * 8);
-          rb00 = __ldcs(reinterpret_cast<const float4*>(resb + c0 * 8));
-          rb01 = __ldcs(reinterpret_cast<const float4*>(resb + c0 * 8 + 4));
-          if (h1) {
-            xb1 = *reinterpret_cast<const uint4*>(xb + c1 * 8);
-            rb10 = __ldcs(reinterpret_cast<const float4*>(resb + c1 * 8));
-            rb11 = __ldcs(reinterpret_cast<const float4*>(resb + c1 * 8 + 4));
-          }
-        }
-        if (ta >= 0) {
-          adaln_group(fa, scb, shb, ta, c0, ma, sa, xa0, ra00, ra01, C);
-          if (h1) adaln_group(fa, scb, shb, ta, c1, ma, sa, xa1, ra10, ra11, C);
-        }
-        if (tb >= 0) {
-          adaln_group(fa, scb, shb, tb, c0, mb, sb, xb0, rb00, rb01, C);
-          if (h1) adaln_group(fa, scb, shb, tb, c1, mb, sb, xb1, rb10, rb11, C);
-        }
+      for (int cb = lane; cb < nb; cb += 32) {
+        AdalnBlockIn ina, inb;
+        if (ta >= 0) adaln_block_load(xa, resa, cb, ina);
+        if (tb >= 0) adaln_block_load(xb, resb, cb, inb);
+        if (!hoisted) adaln_factors(scb, shb, cb, sc1, sh);
+        if (ta >= 0) adaln_block_store(fa, ta, cb, C, ma, sa, ina, sc1, sh);
+        if (tb >= 0) adaln_block_store(fa, tb, cb, C, mb, sb, inb, sc1, sh);
       }
     }
     __syncwarp();
@@ -334,6 +342,11 @@ __global__ void __launch_bounds__(FUSED ? kThreadsFused : kThreads, 1)
 window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__ TmaMaps maps,
                       void* __restrict__ o, int* __restrict__ err, unsigned long long limit_ns,
                       const __grid_constant__ AdalnArgs fa) {
+  using L = SmemLayout<FUSED>;
+  constexpr int kStages = L::kStages;
+  constexpr int OFF_ONES = L::OFF_ONES, OFF_TABLE = L::OFF_TABLE, OFF_SLOTC = L::OFF_SLOTC, OFF_BARS = L::OFF_BARS;
+  constexpr int OFF_XCHG = L::OFF_XCHG, OFF_MISC = L::OFF_MISC;
+  constexpr int OFF_WSTAT = L::OFF_WSTAT, OFF_WTOK = L::OFF_WTOK, OFF_WBAR = L::OFF_WBAR;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(sm);
@@ -785,7 +798,7 @@ template <int HD, bool OUT_F32, bool FUSED>
 cudaError_t launch_t(const WinGeom& g, const TmaMaps& maps, void* o, int* err, long long limit_ns, int num_sms,
                      const AdalnArgs& fa, cudaStream_t st) {
   auto kern = window_attn_tc_kernel<HD, OUT_F32, FUSED>;
-  const int smem = FUSED ? kSmemAllocFused : kSmemAlloc;
+  const int smem = SmemLayout<FUSED>::kAlloc;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const long long units = FUSED ? g.windows : g.windows * g.heads;   // the fused kernel takes whole windows

@@ -78,12 +78,6 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
 
-// Bulk prefetch of `bytes` (a multiple of 16) of global memory into L2, 16-byte aligned
-// address; no completion to wait for.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
@@ -287,6 +281,44 @@ __device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
   const uint32_t a = __float_as_uint(lo) + 0x8000u;
   const uint32_t b = __float_as_uint(hi) + 0x8000u;
   return __byte_perm(a, b, 0x7632);
+}
+
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  uint64_t d;
+  asm("{\n\t.reg .b64 a, b;\n\tmov.b64 a, {%1,%2};\n\tmov.b64 b, {%3,%4};\n\tmul.rn.f32x2 %0, a, b;\n\t}"
+      : "=l"(d) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  float2 r;
+  asm("mov.b64 {%0,%1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
+  return r;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t d;
+  asm("{\n\t.reg .b64 a, b;\n\tmov.b64 a, {%1,%2};\n\tmov.b64 b, {%3,%4};\n\tadd.rn.f32x2 %0, a, b;\n\t}"
+      : "=l"(d) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  float2 r;
+  asm("mov.b64 {%0,%1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
+  return r;
+}
+
+// 32-byte global loads (one full sector per thread): plain, and evict-first for data read
+// once.
+__device__ __forceinline__ void ld_global_v8(const void* p, uint32_t (&v)[8]) {
+  asm volatile("ld.global.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+               : "l"(p)
+               : "memory");
+}
+__device__ __forceinline__ void ld_global_cs_v8(const void* p, uint32_t (&v)[8]) {
+  asm volatile("ld.global.cs.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+               : "l"(p)
+               : "memory");
+}
+// 32-byte evict-first global store (output written once).
+__device__ __forceinline__ void st_global_cs_v8(void* p, const uint32_t (&v)[8]) {
+  asm volatile("st.global.cs.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v[0]), "r"(v[1]), "r"(v[2]),
+               "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
 }
 
 // 32-byte global store (one full sector per thread).

@@ -133,10 +133,13 @@ def _fused(**over):
     (dict(heads=80, qs=5120), api.S3W_ERR_UNSUPPORTED),     # C = 5120 > 4096
     (dict(ws=FAKE + 16), api.S3W_ERR_MISALIGNED),           # workspace not 32-byte aligned
     (dict(o=FAKE + 16), api.S3W_ERR_MISALIGNED),            # attention output not 32-byte aligned
+    (dict(res=FAKE + 16, out=FAKE + 16), api.S3W_ERR_MISALIGNED),   # residual / out (in place) not 32-byte aligned
+    (dict(sc=FAKE + 16), api.S3W_ERR_MISALIGNED),           # FiLM scale not 32-byte aligned
+    (dict(sh=FAKE + 48), api.S3W_ERR_MISALIGNED),           # FiLM shift not 32-byte aligned
     (dict(out=FAKE + 16 * 512), api.S3W_ERR_INVALID_ARG),   # partial overlap of out with residual
 ])
 def test_fused_rejects_bad_arguments_on_host(over, expect):
-    if "out" in over:
+    if "out" in over and "res" not in over:
         over = dict(over, res=FAKE + 64)
     assert _fused(**over) == expect
 
