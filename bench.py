@@ -191,8 +191,11 @@ def launch_stats(ms):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples taken while the timed region runs."""
+    """SM clock and clock-event (throttle) reasons sampled while the timed region runs: NVML
+    read every 5 ms from a thread (nvidia-smi at 50 ms if NVML is unavailable).  Read-only."""
 
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40}
     QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -201,32 +204,63 @@ class ClockSampler:
         self.dev = device_index
         self.proc = None
         self.path = None
+        self.thread = None
+        self.rows = []
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+
+        pynvml.nvmlInit()
+        p = torch.cuda.get_device_properties(self.dev)
+        bus = getattr(p, "pci_bus_id", None)
+        if bus is not None:
+            dom = getattr(p, "pci_domain_id", 0)
+            devid = getattr(p, "pci_device_id", 0)
+            return pynvml.nvmlDeviceGetHandleByPciBusId(f"{dom:08x}:{bus:02x}:{devid:02x}.0")
+        return pynvml.nvmlDeviceGetHandleByIndex(self.dev)
 
     def start(self):
+        import threading
+
+        try:
+            import pynvml
+
+            h = self._nvml_handle()
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.stop_evt = threading.Event()
+
+            def run():
+                while not self.stop_evt.is_set():
+                    try:
+                        self.rows.append((time.time(), float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)),
+                                          float(mx), int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))))
+                    except Exception:
+                        pass
+                    self.stop_evt.wait(0.005)
+
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+            self.source = "nvml 5 ms"
+            return
+        except Exception:
+            self.thread = None
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
                  "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi 50 ms"
         except (OSError, FileNotFoundError):
             self.proc = None
 
-    def stop(self, window=None):
-        """Median SM clock and the throttle reasons seen; with window = (t0, t1) in epoch
-        seconds only the samples taken inside it count (all of them if none is)."""
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    def _smi_rows(self):
         import datetime
 
         rows = []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             f = [x.strip() for x in line.split(",")]
             if len(f) < 10:
@@ -236,19 +270,37 @@ class ClockSampler:
             except ValueError:
                 ts = None
             try:
-                rows.append((ts, float(f[2]), float(f[3]), f[6:10]))
+                bits = sum(self.REASON_BITS[nm] for nm, val in zip(names, f[6:10]) if val.lower() == "active")
+                rows.append((ts, float(f[2]), float(f[3]), bits))
             except ValueError:
                 continue
         os.unlink(self.path)
+        return rows
+
+    def stop(self, window=None):
+        """Median SM clock and the throttle reasons seen; with window = (t0, t1) in epoch
+        seconds only the samples taken inside it count (all of them if none is)."""
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=5)
+            rows = list(self.rows)
+        elif self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            rows = self._smi_rows()
+        else:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source"]}
         inside = [r for r in rows if window and (r[0] is None or window[0] <= r[0] <= window[1])]
-        for _, s_mhz, m_mhz, flags in (inside or rows):
-            sm.append(s_mhz)
-            mx.append(m_mhz)
-            for nm, val in zip(names, flags):
-                if val.lower() == "active":
-                    reasons.add(nm)
+        use = inside or rows
+        reasons = sorted({nm for _, _, _, bits in use for nm, bit in self.REASON_BITS.items() if bits & bit})
+        sm = [r[1] for r in use]
+        mx = [r[2] for r in use]
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "samples": len(sm), "reasons": sorted(reasons)}
+                "samples": len(sm), "samples_in_timed_region": len(inside), "source": self.source,
+                "reasons": reasons}
 
 
 # ----------------------------------------------------------------------------- GPU arm
