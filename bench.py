@@ -69,11 +69,11 @@ KERNEL_SOURCES = [os.path.join("swin3d_window_attention_b200", "csrc", f)
                   for f in ("attn_tcgen05.cu", "attn_common.cuh", "sm100_ptx.cuh", "s3w_common.cuh")]
 
 
-def geometry(w):
+def geometry(w, window=WINDOW):
     """Derived sizes of a workload: channels, tokens, windows (all samples)."""
     C = w["heads"] * w["hd"]
     tokens = w["B"] * w["T"] * w["H"] * w["W"]
-    windows = w["B"] * math.prod(-(-d // a) for d, a in zip((w["T"], w["H"], w["W"]), WINDOW))
+    windows = w["B"] * math.prod(-(-d // a) for d, a in zip((w["T"], w["H"], w["W"]), window))
     return C, tokens, windows
 
 
@@ -83,10 +83,11 @@ def attn_bytes(w, o_bytes=2, in_bytes=2):
     return (3 * in_bytes + o_bytes) * tokens * C
 
 
-def attn_flops(w):
+def attn_flops(w, window=WINDOW):
     """4 N^2 d per (window, head): QK^T and PV, dense inside each window."""
-    _, _, windows = geometry(w)
-    return windows * w["heads"] * 4 * N_TOK * N_TOK * w["hd"]
+    _, _, windows = geometry(w, window)
+    n = math.prod(window)
+    return windows * w["heads"] * 4 * n * n * w["hd"]
 
 
 def fused_bytes(w, out_bytes=4):
@@ -412,6 +413,25 @@ def bench_configs(torch, s3w, dev, stream, peaks, reps):
         "attn": {**launch_stats(ms_a), "bytes": nbytes, "flops": attn_flops(w), "windows_per_s": windows / (a_med * 1e-3),
                  "roofline": roofline(nbytes, attn_flops(w), a_med,
                                       {**peaks, "bf16_tflops": peaks["bf16_tflops"] / 2})}}
+    del q, k, v, o
+
+    # windows larger than one tile: the streaming path on the stage-1 grid with (2,12,12)
+    # windows (N = 288), shift (1,6,6)
+    w = WORKLOADS["stage1"]
+    big = (2, 12, 12)
+    C, tokens, windows = geometry(w, big)
+    q, k, v = device_qkv(torch, w, dev, 945)
+    o = torch.empty_like(q)
+    ms_a = timed(torch, stream, lambda: s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], big, (1, 6, 6)),
+                 reps)
+    launches += len(ms_a)
+    a_med = statistics.median(ms_a)
+    out["stage1_window_2x12x12"] = {
+        "grid": "B=1 T4xH180xW360, 8 heads x 64, window (2,12,12) N=288, shift (1,6,6), 900 windows; streaming "
+                "path (K/V blocks of 72 slots, online softmax)",
+        "attn": {**launch_stats(ms_a), "bytes": attn_bytes(w), "flops": attn_flops(w, big),
+                 "windows_per_s": windows / (a_med * 1e-3),
+                 "roofline": roofline(attn_bytes(w), attn_flops(w, big), a_med, peaks)}}
     del q, k, v, o
 
     # fused attention + AdaLN (one kernel per block) on the stage-1 grid: one launch, and the

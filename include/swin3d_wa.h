@@ -83,7 +83,11 @@ typedef enum { S3W_BF16 = 0, S3W_F32 = 1 } s3w_dtype;
  *           o_token_stride elements between tokens (>= heads*head_dim, 16-byte rows).
  *           Must not overlap q, k or v.  Channels beyond heads*head_dim are not written.
  * B,T,H,W   batch and unpadded grid sizes, each >= 1.
- * win_*     window extents, each >= 1; N = win_t*win_h*win_w must satisfy 1 <= N <= 144.
+ * win_*     window extents, each >= 1, N = win_t*win_h*win_w.  1 <= N <= 144: one tile per
+ *           (window, head).  144 < N <= 65536 (BF16 inputs, win_w <= 128): the streaming
+ *           path of the same section (K/V blocks of whole (t, h) rows, <= 128 slots each,
+ *           streamed past each query block with online-softmax rescaling).  Anything else
+ *           returns S3W_ERR_UNSUPPORTED.
  * shift_*   0 <= shift < window on each axis.
  * heads     >= 1.  head_dim: 32 or 64.
  * scale     logit scale; a value <= 0 selects 1/sqrt(head_dim).

@@ -16,6 +16,7 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr long long kMaxStreamN = 1 << 16;   // window slots on the streaming path
 
 // One error word per device; kernels get its device address.
 __device__ int g_s3w_error_word;
@@ -105,8 +106,11 @@ int make_geometry(const void* q, const void* k, const void* v, void* o, int B, i
     return S3W_ERR_INVALID_ARG;
   const long long C = static_cast<long long>(heads) * head_dim;
   if (qkv_token_stride < C || o_token_stride < C) return S3W_ERR_INVALID_ARG;
+  if (win_t > 65536 || win_h > 65536 || win_w > 65536) return S3W_ERR_UNSUPPORTED;   // keeps N in range
   const long long N = static_cast<long long>(win_t) * win_h * win_w;
-  if (N > 144) return S3W_ERR_UNSUPPORTED;
+  // N <= 144: one tile per (window, head); above, the streaming kernel, whose blocks hold
+  // whole rows of win_w tokens (<= 128), and only for BF16 inputs
+  if (N > 144 && (win_w > 128 || in_dtype != S3W_BF16 || N > kMaxStreamN)) return S3W_ERR_UNSUPPORTED;
   if (head_dim != 32 && head_dim != 64) return S3W_ERR_UNSUPPORTED;
   const int ib = in_dtype == S3W_F32 ? 4 : 2;
   const int ob = out_dtype == S3W_F32 ? 4 : 2;
@@ -121,6 +125,8 @@ int make_geometry(const void* q, const void* k, const void* v, void* o, int B, i
   const long long per_sample = (Pt / win_t) * (Ph / win_h) * (Pw / win_w);
   if (per_sample > INT32_MAX) return S3W_ERR_UNSUPPORTED;
   if (per_sample * B * heads > INT32_MAX) return S3W_ERR_UNSUPPORTED;  // tile index is 32-bit
+  // streaming path: units = tiles x blocks (at most win_t x win_h blocks per window)
+  if (N > 144 && per_sample * B * heads * win_t * win_h > INT32_MAX) return S3W_ERR_UNSUPPORTED;
 
   s3w::WinGeom& g = *out;
   g = s3w::WinGeom{};
@@ -169,9 +175,11 @@ int swin3d_window_attn_fwd(const void* q, const void* k, const void* v, void* o,
   g.test_stall = g_test_stall.load(std::memory_order_relaxed);
   const long long limit = g_wait_limit_ns.load(std::memory_order_relaxed);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = in_dtype == S3W_F32
-                      ? s3w::launch_window_attn_tf32(g, q, k, v, o, out_dtype == S3W_F32, ds->err, limit, ds->num_sms, st)
-                      : s3w::launch_window_attn_tc(g, q, k, v, o, out_dtype == S3W_F32, ds->err, limit, ds->num_sms, st);
+  cudaError_t e =
+      g.N > 144 ? s3w::launch_window_attn_stream(g, q, k, v, o, out_dtype == S3W_F32, ds->err, limit, ds->num_sms, st)
+      : in_dtype == S3W_F32
+          ? s3w::launch_window_attn_tf32(g, q, k, v, o, out_dtype == S3W_F32, ds->err, limit, ds->num_sms, st)
+          : s3w::launch_window_attn_tc(g, q, k, v, o, out_dtype == S3W_F32, ds->err, limit, ds->num_sms, st);
   return e == cudaSuccess ? S3W_OK : S3W_ERR_CUDA;
 }
 
@@ -184,6 +192,7 @@ int swin3d_window_attn_fwd_legacy_mma(const void* q, const void* k, const void* 
                          qkv_token_stride, o_token_stride, scale, in_dtype, out_dtype, &g);
   if (rc != S3W_OK) return rc;
   if (in_dtype != S3W_BF16) return S3W_ERR_UNSUPPORTED;   // the baseline path is BF16 only
+  if (g.N > 144) return S3W_ERR_UNSUPPORTED;               // and single-tile windows only
   if (g.windows * heads > (1ll << 31) - 1) return S3W_ERR_UNSUPPORTED;
   DeviceState* ds = nullptr;
   rc = device_state(&ds);
@@ -221,6 +230,7 @@ int swin3d_window_attn_adaln_fwd(const void* q, const void* k, const void* v, lo
   int rc = make_geometry(q, k, v, o ? o : out, B, T, H, W, win_t, win_h, win_w, shift_t, shift_h, shift_w, heads,
                          head_dim, qkv_token_stride, C, attn_scale, S3W_BF16, S3W_BF16, &g);
   if (rc != S3W_OK) return rc;
+  if (g.N > 144) return S3W_ERR_UNSUPPORTED;   // the fused kernel takes single-tile windows
   if (C % 8 != 0 || C > 4096) return S3W_ERR_UNSUPPORTED;
   // the AdaLN part moves 32-byte vectors of every one of these
   auto aligned32 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; };

@@ -36,6 +36,14 @@ cudaError_t launch_window_attn_tf32(const WinGeom& g, const void* q, const void*
                                     void* o, bool out_f32, int* err, long long spin_limit,
                                     int num_sms, cudaStream_t stream);
 
+// Window attention for windows of more than 144 slots (attn_stream.cu): BF16 Q/K/V, the
+// window cut into blocks of whole (t, h) rows (<= 128 slots; win_w <= 128), K/V blocks
+// streamed with online-softmax rescaling.  Units of work: windows x heads x blocks.
+cudaError_t launch_window_attn_stream(const WinGeom& g, const void* q, const void* k, const void* v, void* o,
+                                      bool out_f32, int* err, long long spin_limit, int num_sms,
+                                      cudaStream_t stream);
+long long window_attn_stream_units(const WinGeom& g);
+
 // Window attention on the legacy warp-level mma.sync path (attn_mma.cu); kept as the
 // measured baseline the tcgen05 kernel is compared with.
 cudaError_t launch_window_attn_mma(const WinGeom& g, const void* q, const void* k, const void* v,

@@ -60,7 +60,10 @@ def _attn(**over):
     (dict(os_=511), api.S3W_ERR_INVALID_ARG),
     (dict(outd=7), api.S3W_ERR_INVALID_ARG),
     (dict(scale=float("nan")), api.S3W_ERR_INVALID_ARG),
-    (dict(ww=13, sw=6), api.S3W_ERR_UNSUPPORTED),   # N = 156 > 144
+    (dict(ww=130, sw=6), api.S3W_ERR_UNSUPPORTED),  # N > 144 with win_w > 128: no streaming blocks of whole rows
+    (dict(wh=300, ww=120, sh=3, sw=6), api.S3W_ERR_UNSUPPORTED),   # N = 72,000 > 65,536
+    (dict(wt=70000, st=1), api.S3W_ERR_UNSUPPORTED),                # a window extent above 65,536
+    (dict(ww=13, sw=6, ind=1, qs=512, os_=512), api.S3W_ERR_UNSUPPORTED),   # N = 156: streaming is BF16 only
     (dict(hd=48, qs=384, os_=384), api.S3W_ERR_UNSUPPORTED),
     (dict(ind=1, qs=514), api.S3W_ERR_MISALIGNED),  # fp32 token rows not on 16-byte boundaries
     (dict(q=FAKE + 8), api.S3W_ERR_MISALIGNED),

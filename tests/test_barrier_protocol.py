@@ -8,9 +8,11 @@ has completed (so it can neither pass on, nor miss, another phase); every arriva
 belongs to one tile.  mbarrier semantics modelled: a phase completes when its count of
 arrivals is reached; try_wait.parity(p) passes iff the current phase parity differs from p.
 
-The BF16 kernel (3 stages, P over the stage's Q/K, P and row-max hand-over barriers per tile
-parity, O read out by four epilogue warps) and the TF32 kernel (2 stages, P over S in TMEM, S(t+1) after PV(t) completes) are
-modelled; the single-barrier variant of the BF16 protocol must be caught.
+Modelled: the BF16 kernel (3 stages, P and row-max hand-over barriers per tile parity), the
+TF32 kernel (2 stages, P over S in TMEM, S(t+1) after PV(t) completes) and the streaming kernel
+for windows of more than 144 slots (Q by unit parity, K/V ring, S double-buffered in TMEM, P
+hand-over per block parity).  The single-barrier variants of the BF16 and streaming protocols
+must be caught.
 """
 import random
 
@@ -270,3 +272,110 @@ def test_tf32_protocol_holds_under_random_schedules():
     for seed in range(120):
         for tail in (True, False):
             model_tf32(ntiles=1 + seed % 11, has_tail=tail, seed=seed)
+
+
+def model_stream(nunits, nblk, seed=0, variant="kernel", max_steps=2_000_000):
+    """The streaming kernel (windows of more than 144 slots): Q blocks by unit parity, K/V
+    blocks through a 3-stage ring, S double-buffered by block parity in TMEM with P written
+    back over it (S(j + 2) waits for PV(j)), P handed over on a barrier per block parity, one
+    O accumulator read out by every softmax thread before the next PV.  variant="single_p_full"
+    hands P over on one barrier, which a fast row can lap."""
+    rng = random.Random(seed)
+    S = 3
+    B = {}
+
+    def mk(name, count):
+        B[name] = Bar(name, count)
+
+    for b in range(2):
+        mk(f"q_full{b}", 1); mk(f"q_free{b}", 1); mk(f"s_full{b}", 1); mk(f"s_free{b}", 1)
+        mk(f"p_full{b}", 256)
+    for s in range(S):
+        mk(f"kv_full{s}", 1); mk(f"kv_empty{s}", 1 + 256); mk(f"tab_full{s}", 32)
+    mk("o_full", 1); mk("o_empty", 256)
+    for par in range(2):
+        for h in range(2):
+            mk(f"xmax{par}{h}", 128)
+    nblocks = nunits * nblk
+
+    def pfull(j):   # barrier name, parity, phase index of block j's P hand-over
+        if variant == "single_p_full":
+            return "p_full0", j & 1, j
+        return f"p_full{j & 1}", (j >> 1) & 1, j >> 1
+
+    def tma():
+        j = 0
+        for ui in range(nunits):
+            qp = ui & 1
+            yield ("wait", f"q_free{qp}", ((ui >> 1) & 1) ^ 1, (ui >> 1) - 1)
+            yield ("tma", f"q_full{qp}", ui)
+            for _ in range(nblk):
+                s = j % S
+                yield ("wait", f"kv_empty{s}", ((j // S) & 1) ^ 1, j // S - 1)
+                yield ("tma", f"kv_full{s}", j)
+                j += 1
+
+    def table():
+        for j in range(nblocks):
+            s = j % S
+            yield ("wait", f"kv_empty{s}", ((j // S) & 1) ^ 1, j // S - 1)
+            yield ("arrive", f"tab_full{s}", j, 32)
+
+    def mma():
+        for jj in range(nblocks + 1):
+            if jj < nblocks:
+                ui, kb = divmod(jj, nblk)
+                s, buf, qp = jj % S, jj & 1, ui & 1
+                if kb == 0:
+                    yield ("wait", f"q_full{qp}", (ui >> 1) & 1, ui >> 1)
+                yield ("wait", f"kv_full{s}", (jj // S) & 1, jj // S)
+                yield ("wait", f"s_free{buf}", ((jj >> 1) & 1) ^ 1, (jj >> 1) - 1)
+                yield ("commit", [(f"s_full{buf}", jj)] + ([(f"q_free{qp}", ui)] if kb == nblk - 1 else []))
+            if jj > 0:
+                t = jj - 1
+                name, par, ph = pfull(t)
+                yield ("wait", name, par, ph)
+                yield ("wait", "o_empty", (t & 1) ^ 1, t - 1)
+                yield ("commit", [("o_full", t), (f"kv_empty{t % S}", t), (f"s_free{t & 1}", t)])
+
+    def softmax(w):
+        half = w >> 2
+        j = 0
+        for _ in range(nunits):
+            for kb in range(nblk):
+                s, buf = j % S, j & 1
+                yield ("wait", f"tab_full{s}", (j // S) & 1, j // S)
+                yield ("arrive", f"kv_empty{s}", j, 32)
+                yield ("wait", f"s_full{buf}", (j >> 1) & 1, j >> 1)
+                yield ("arrive", f"xmax{buf}{half}", j, 32)
+                yield ("wait", f"xmax{buf}{half ^ 1}", (j >> 1) & 1, j >> 1)
+                name, _, _ = pfull(j)
+                yield ("arrive", name, j, 32)
+                if kb > 0:
+                    yield ("wait", "o_full", (j - 1) & 1, j - 1)
+                    yield ("arrive", "o_empty", j - 1, 32)
+                j += 1
+            yield ("wait", "o_full", (j - 1) & 1, j - 1)
+            yield ("arrive", "o_empty", j - 1, 32)
+
+    actors = {"tma": tma(), "table": table(), "mma": mma()}
+    for w in range(8):
+        actors[f"w{w}"] = softmax(w)
+    return run(actors, B, rng, max_steps)
+
+
+def test_stream_protocol_holds_under_random_schedules():
+    for seed in range(100):
+        model_stream(nunits=1 + seed % 5, nblk=1 + seed % 4, seed=seed)
+
+
+def test_stream_single_p_full_is_caught():
+    """With one P hand-over barrier a softmax warp can arrive for block j + 1 before a warp of
+    another row has arrived for block j (nothing between the two needs PV(j)): caught."""
+    fails = 0
+    for seed in range(60):
+        try:
+            model_stream(nunits=2 + seed % 3, nblk=2 + seed % 3, seed=seed, variant="single_p_full")
+        except AssertionError:
+            fails += 1
+    assert fails > 0
