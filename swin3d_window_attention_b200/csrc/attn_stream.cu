@@ -1,6 +1,7 @@
 // Shifted-window attention for windows larger than one 144-slot tile (N > 144): the
-// multi-block streaming path.  Each window is cut into blocks of whole (t, h) rows of one
-// T-slab, at most 128 slots each.  A unit of work is one (window, head, query block); the
+// multi-block streaming path.  Each window is cut into blocks of consecutive whole (t, h)
+// rows (a block may span T-slabs), at most 128 slots each.  A unit of work is one (window,
+// head, query block); the
 // window's K/V blocks stream past it through a TMA ring, and the softmax is carried across
 // key blocks online (running row max, rescaled row sum and output), so any N fits.
 //
@@ -24,8 +25,9 @@
 //                       TMEM (the A operand of the TS form) and V plus a block of ones from
 //                       shared memory: O's columns 64.. are the row sums of the bf16 P.
 //   TMA warp 9          the unit's Q block (two buffers) and every K/V block through a
-//                       three-stage ring: one box per block, or one per (t, h) row where a
-//                       block crosses a seam.  Padded coordinates read as zero.
+//                       three-stage ring: per run of rows inside one T-slab and one side of
+//                       the H seam, boxes of 2^k rows; one row at a time (cut in two) where
+//                       the window wraps around the W seam.  Padded coordinates read as zero.
 //   table warp 10       per K/V block, the visible keys for each of the 8 combinations of a
 //                       query's wrapped-around sides.
 // Every wait is bounded; a timeout unwinds the CTA (error word set, copies drained, TMEM
@@ -55,14 +57,20 @@ constexpr int kMmaWarpS = 8, kTmaWarpS = 9, kTableWarpS = 10;
 // of the row sum) after them.
 constexpr uint32_t TS_S = 0, TS_O = 256, kSumCol = 64;
 
-// Box shapes of the tensor maps: a block of nh rows, the shorter last block of a slab, one
-// (t, h) row, and a row cut at the W seam (win_w - shift_w tokens, then shift_w).
-enum : int { kBoxGroup = 0, kBoxGroupRem = 1, kBoxRun = 2, kBoxW1 = 3, kBoxW2 = 4 };
+// Box shapes of the tensor maps: 2^k (t, h) rows of win_w tokens (k = 0..7; a run of rows
+// is loaded as its binary decomposition), and a row cut at the W seam (win_w - shift_w
+// tokens, then shift_w).
+constexpr int kRowShapes = 8;
+enum : int { kBoxW1 = kRowShapes, kBoxW2 = kRowShapes + 1, kBoxShapesS = kRowShapes + 2 };
+struct StreamMaps {
+  CUtensorMap m[3][kBoxShapesS];   // [tensor q/k/v][box shape]
+};
 
-// How a window is cut into blocks.
+// How a window is cut into blocks: its (t, h) rows, numbered R = t win_h + h, in runs of
+// `nr` consecutive rows (the last may be shorter), at most 128 slots each; a block may span
+// two or more T-slabs.
 struct StreamPlan {
-  int nh;        // (t, h) rows per block (the last block of a slab may have fewer)
-  int groups;    // blocks per T-slab
+  int nr;        // rows per block
   int nblk;      // blocks per window (= query blocks = key blocks)
   long long units;   // windows * heads * nblk
 };
@@ -90,47 +98,61 @@ struct SmemS {
   static_assert(OFF_BARS % 8 == 0, "mbarrier alignment");
 };
 
-// Rows of block b: T-slab rt, (t, h) rows [r0, r0 + nr).
+// Rows of block b: window rows [r0, r0 + nr) (row R = t win_h + h).
 struct BlockRows {
-  int rt, r0, nr;
+  int r0, nr;
 };
 __device__ __forceinline__ BlockRows block_rows(const WinGeom& g, const StreamPlan& sp, int b) {
   BlockRows br;
-  br.rt = b / sp.groups;
-  br.r0 = (b - br.rt * sp.groups) * sp.nh;
-  br.nr = min(sp.nh, g.wh - br.r0);
+  br.r0 = b * sp.nr;
+  br.nr = min(sp.nr, g.wt * g.wh - br.r0);
   return br;
 }
 
 // Loads block b of tensor `tsr` of the tile into `dst` (slot i of the block at row i) and
-// completes its bytes on `bar`.
-__device__ __forceinline__ void load_block(const WinGeom& g, const StreamPlan& sp, const TmaMaps& maps, int tsr,
+// completes its bytes on `bar`.  Rows of one T-slab on one side of the H seam form a run,
+// loaded as boxes of 2^k rows (its binary decomposition); where the window wraps around the
+// W seam, every row is two boxes.
+__device__ __forceinline__ void load_block(const WinGeom& g, const StreamPlan& sp, const StreamMaps& maps, int tsr,
                                            const TileCoord& tc, int b, uint32_t dst, uint32_t bar) {
   const BlockRows br = block_rows(g, sp, b);
-  int t = tc.bt + br.rt;
-  t -= t >= g.Pt ? g.Pt : 0;
   const int c0 = tc.head * g.head_dim;
   const bool wrap_w = tc.bw + g.ww > g.Pw;
-  const int n1h = g.Ph - tc.bh;   // window rows before the H seam
+  const int n1h = g.Ph - tc.bh;   // window rows (h) before the H seam
   const int n1w = g.Pw - tc.bw;   // window columns before the W seam
-  auto hrow = [&](int r) {
-    const int h = tc.bh + r;
-    return h - (h >= g.Ph ? g.Ph : 0);
-  };
-  if (!wrap_w && !(br.r0 < n1h && br.r0 + br.nr > n1h)) {
-    tma_load_5d(dst, &maps.m[tsr][br.nr == sp.nh ? kBoxGroup : kBoxGroupRem], c0, tc.bw, hrow(br.r0), t, tc.bsmp,
-                bar);
-    return;
-  }
+  const uint32_t row_bytes = static_cast<uint32_t>(g.ww * kRowBytes);
+  int rt = br.r0 / g.wh, rh = br.r0 - rt * g.wh;
+  int done = 0;
 #pragma unroll 1
-  for (int r = 0; r < br.nr; ++r) {
-    const uint32_t d = dst + static_cast<uint32_t>(r * g.ww * kRowBytes);
-    const int h = hrow(br.r0 + r);
+  while (done < br.nr) {
+    int t = tc.bt + rt;
+    t -= t >= g.Pt ? g.Pt : 0;
+    // the run: rows of this slab, up to the H seam or the slab's end
+    const int lim = rh < n1h ? min(g.wh, n1h) : g.wh;
+    const int n = min(br.nr - done, lim - rh);
+    int h = tc.bh + rh;
+    h -= h >= g.Ph ? g.Ph : 0;
+    uint32_t d = dst + static_cast<uint32_t>(done) * row_bytes;
     if (!wrap_w) {
-      tma_load_5d(d, &maps.m[tsr][kBoxRun], c0, tc.bw, h, t, tc.bsmp, bar);
+#pragma unroll 1
+      for (int k = kRowShapes - 1; k >= 0; --k) {
+        if (!((n >> k) & 1)) continue;
+        tma_load_5d(d, &maps.m[tsr][k], c0, tc.bw, h, t, tc.bsmp, bar);
+        d += static_cast<uint32_t>(1 << k) * row_bytes;
+        h += 1 << k;
+      }
     } else {
-      tma_load_5d(d, &maps.m[tsr][kBoxW1], c0, tc.bw, h, t, tc.bsmp, bar);
-      tma_load_5d(d + static_cast<uint32_t>(n1w * kRowBytes), &maps.m[tsr][kBoxW2], c0, 0, h, t, tc.bsmp, bar);
+#pragma unroll 1
+      for (int r = 0; r < n; ++r, d += row_bytes, ++h) {
+        tma_load_5d(d, &maps.m[tsr][kBoxW1], c0, tc.bw, h, t, tc.bsmp, bar);
+        tma_load_5d(d + static_cast<uint32_t>(n1w * kRowBytes), &maps.m[tsr][kBoxW2], c0, 0, h, t, tc.bsmp, bar);
+      }
+    }
+    done += n;
+    rh += n;
+    if (rh == g.wh) {
+      rh = 0;
+      ++rt;
     }
   }
 }
@@ -138,9 +160,10 @@ __device__ __forceinline__ void load_block(const WinGeom& g, const StreamPlan& s
 // The grid token of slot i of block b (-1 if padded) and its wrapped-around sides.
 __device__ __forceinline__ int block_slot(const WinGeom& g, const TileCoord& tc, const BlockRows& br, int i,
                                           uint32_t* sides) {
-  const int rh = br.r0 + i / g.ww, rw = i - (i / g.ww) * g.ww;
-  *sides = (br.rt >= g.wt - g.st ? 1u : 0u) | (rh >= g.wh - g.sh ? 2u : 0u) | (rw >= g.ww - g.sw ? 4u : 0u);
-  int t = tc.bt + br.rt, h = tc.bh + rh, w = tc.bw + rw;
+  const int row = br.r0 + i / g.ww, rw = i - (i / g.ww) * g.ww;
+  const int rt = row / g.wh, rh = row - rt * g.wh;
+  *sides = (rt >= g.wt - g.st ? 1u : 0u) | (rh >= g.wh - g.sh ? 2u : 0u) | (rw >= g.ww - g.sw ? 4u : 0u);
+  int t = tc.bt + rt, h = tc.bh + rh, w = tc.bw + rw;
   t -= t >= g.Pt ? g.Pt : 0;
   h -= h >= g.Ph ? g.Ph : 0;
   w -= w >= g.Pw ? g.Pw : 0;
@@ -148,24 +171,61 @@ __device__ __forceinline__ int block_slot(const WinGeom& g, const TileCoord& tc,
   return ((tc.bsmp * g.T + t) * g.H + h) * g.W + w;
 }
 
-// O (+)= P [V | 1] over `ksteps` K steps of 16 keys: A (P, bf16) from TMEM at column
-// 64 (k / 4) + 8 (k % 4) of the S buffer, B (V, MN-major) from shared memory moving 2048
-// bytes per step while its leading byte offset (the ones block behind it) moves back as much.
+// Word w (bits 32 w .. 32 w + 31) of the 128-bit set of indices in [lo, hi).
+__device__ __forceinline__ uint32_t range_word(int lo, int hi, int w) {
+  const int a = max(lo - 32 * w, 0), b = min(hi - 32 * w, 32);
+  if (b <= a) return 0u;
+  return (b - a == 32) ? 0xffffffffu : (((1u << (b - a)) - 1u) << a);
+}
+
+// 32 bits of the 128-bit set (c0, c1, c2, c3) starting at bit a (0 <= a < 128; zeros past
+// the end), with register selects instead of an indexed array.
+__device__ __forceinline__ uint32_t bits_at(const uint32_t (&c)[4], int a) {
+  const int w = a >> 5;
+  const uint32_t x = w == 0 ? c[0] : (w == 1 ? c[1] : (w == 2 ? c[2] : c[3]));
+  const uint32_t y = w == 0 ? c[1] : (w == 1 ? c[2] : (w == 2 ? c[3] : 0u));
+  return __funnelshift_r(x, y, static_cast<uint32_t>(a & 31));
+}
+
+// Offsets r in [0, w) of a window axis whose coordinate (base + r, wrapped at P) lies inside
+// the unpadded extent D: [0, min(P - base, D - base)) and, past the seam, [P - base,
+// min(w, P - base + D)).
+struct RealRange {
+  int a1, b1, a2, b2;
+};
+__device__ __forceinline__ RealRange real_range(int base, int w, int P, int D) {
+  RealRange r;
+  const int n1 = P - base;
+  r.a1 = 0;
+  r.b1 = min(min(n1, w), D - base);
+  r.a2 = n1;
+  r.b2 = min(w, n1 + D);
+  return r;
+}
+__device__ __forceinline__ bool in_real(const RealRange& r, int x) {
+  return (x >= r.a1 && x < r.b1) || (x >= r.a2 && x < r.b2);
+}
+
+// O (+)= P [V | 1] over `ksteps` (1..8) K steps of 16 keys, one asm block: A (P, bf16) from
+// TMEM at column 64 (k / 4) + 8 (k % 4) of the S buffer, B (V, MN-major) from shared memory
+// moving 2048 bytes per step while its leading byte offset (the ones block behind it) moves
+// back as much (-8388480 = 2048 / 16 - (2048 / 16 << 16) in descriptor units).  Steps past
+// `ksteps` are predicated off.  Executed by the whole warp; only `leader` issues.
+#define S3W_PV_STEP_(K, AOFF)                                                                     \
+  "add.s64 b, b, -8388480;\n\tadd.u32 a, %1, " AOFF ";\n\tsetp.gt.and.s32 p, %5, " K ", q;\n\t" \
+  "@p tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, t;\n\t"
 __device__ __forceinline__ void umma_pv_ts(uint32_t d_tmem, uint32_t p_tmem, uint64_t v0, int ksteps, uint32_t idesc,
                                            uint32_t leader) {
-#pragma unroll 1
-  for (int k = 0; k < ksteps; ++k) {
-    const uint32_t a = p_tmem + 64u * static_cast<uint32_t>(k >> 2) + 8u * static_cast<uint32_t>(k & 3);
-    const uint64_t d = static_cast<uint64_t>(k) * (2048 >> 4);
-    const uint64_t b = v0 + d - (d << 16);
-    const uint32_t acc = k ? 1u : 0u;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 q, %5, 0;\n\t"
-        "@q tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a), "l"(b), "r"(idesc), "r"(acc), "r"(leader)
-        : "memory");
-  }
+  asm volatile(
+      "{\n\t.reg .pred q, p, f, t;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
+      "setp.ne.b32 q, %4, 0;\n\tsetp.ne.b32 f, %4, %4;\n\tsetp.eq.b32 t, %4, %4;\n\t"
+      "mov.b64 b, %2;\n\t@q tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b, %3, f;\n\t"
+      S3W_PV_STEP_("1", "8") S3W_PV_STEP_("2", "16") S3W_PV_STEP_("3", "24") S3W_PV_STEP_("4", "64")
+      S3W_PV_STEP_("5", "72") S3W_PV_STEP_("6", "80") S3W_PV_STEP_("7", "88") "}" ::"r"(d_tmem),
+      "r"(p_tmem), "l"(v0), "r"(idesc), "r"(leader), "r"(ksteps)
+      : "memory");
 }
+#undef S3W_PV_STEP_
 
 __device__ __forceinline__ void tmem_wait_st_s() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -178,7 +238,7 @@ __device__ __forceinline__ void tmem_st8_s(uint32_t taddr, const uint32_t (&v)[8
 
 template <int HD, bool OUT_F32>
 __global__ void __launch_bounds__(kThreadsS, 1)
-window_attn_stream_kernel(const __grid_constant__ WinGeom g, const __grid_constant__ TmaMaps maps,
+window_attn_stream_kernel(const __grid_constant__ WinGeom g, const __grid_constant__ StreamMaps maps,
                           const StreamPlan sp, void* __restrict__ o, int* __restrict__ err,
                           unsigned long long limit_ns) {
   extern __shared__ uint8_t smem_raw[];
@@ -255,7 +315,7 @@ window_attn_stream_kernel(const __grid_constant__ WinGeom g, const __grid_consta
 #pragma unroll
       for (int a = 0; a < 3; ++a)
 #pragma unroll
-        for (int b = 0; b < kBoxShapes; ++b) prefetch_tmap(&maps.m[a][b]);
+        for (int b = 0; b < kBoxShapesS; ++b) prefetch_tmap(&maps.m[a][b]);
       long long j = 0, nq = 0;   // K/V blocks and Q blocks issued
       bool ok = true;
       for (long long ui = 0; ok && ui < my_units; ++ui) {
@@ -300,7 +360,10 @@ window_attn_stream_kernel(const __grid_constant__ WinGeom g, const __grid_consta
     }
   } else if (warp == kTableWarpS) {
     // ------------------------------------------------------------------ key tables
-    // Lane L fills word L % 4 (keys 32 (L % 4) ..) of combination L / 4.
+    // Lane L fills word L % 4 (keys 32 (L % 4) ..) of combination L / 4.  The visibility of
+    // a key factors by axis: its T-slab (per block), its (t, h) row and its column.  Per
+    // window the visible columns of the lane's combination are a 128-bit set built from index
+    // intervals; a block's word then walks its keys row by row without divisions.
     const uint32_t combo = static_cast<uint32_t>(lane) >> 2;
     const int word = lane & 3;
     long long j = 0;
@@ -311,8 +374,21 @@ window_attn_stream_kernel(const __grid_constant__ WinGeom g, const __grid_consta
       const TileCoord tc = tile_coord(g, tile);
       // sides that split the window's regions: axes along which it is the last window of
       // a shifted axis
-      const uint32_t last = ((tc.itw == g.nwt - 1 && g.st > 0) ? 1u : 0u) | ((tc.ih == g.nwh - 1 && g.sh > 0) ? 2u : 0u) |
-                            ((tc.iw == g.nww - 1 && g.sw > 0) ? 4u : 0u);
+      const bool last_t = tc.itw == g.nwt - 1 && g.st > 0, last_h = tc.ih == g.nwh - 1 && g.sh > 0,
+                 last_w = tc.iw == g.nww - 1 && g.sw > 0;
+      const RealRange rt_r = real_range(tc.bt, g.wt, g.Pt, g.T);
+      const RealRange rh_r = real_range(tc.bh, g.wh, g.Ph, g.H);
+      const RealRange rw_r = real_range(tc.bw, g.ww, g.Pw, g.W);
+      uint32_t colok[4];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t real = range_word(rw_r.a1, rw_r.b1, q4) | range_word(rw_r.a2, rw_r.b2, q4);
+        if (last_w) {
+          const uint32_t side = range_word(g.ww - g.sw, g.ww, q4);
+          real &= (combo & 4u) ? side : ~side;
+        }
+        colok[q4] = real;
+      }
       for (int kb = 0; kb < sp.nblk; ++kb, ++j) {
         const int s = static_cast<int>(j % kStagesS);
         if (__any_sync(0xffffffffu, *abort_flag != 0) ||
@@ -323,14 +399,26 @@ window_attn_stream_kernel(const __grid_constant__ WinGeom g, const __grid_consta
         }
         const BlockRows br = block_rows(g, sp, kb);
         const int nb = br.nr * g.ww;
+        auto row_ok = [&](int row) {   // row of the block -> its (t, h) visible for the combination
+          const int rr = br.r0 + row;
+          const int rt = rr / g.wh, rh = rr - rt * g.wh;
+          return row < br.nr && in_real(rt_r, rt) && (!last_t || (rt >= g.wt - g.st) == ((combo & 1u) != 0)) &&
+                 in_real(rh_r, rh) && (!last_h || (rh >= g.wh - g.sh) == ((combo & 2u) != 0));
+        };
+        // the word's keys [i0, i1) are key = row * win_w + col: per (t, h) row overlapping
+        // them, that row's visible columns shifted into place
         uint32_t bits = 0;
+        const int i0 = 32 * word, i1 = min(i0 + 32, nb);
+        if (i0 < i1) {
+          int row = i0 / g.ww;
 #pragma unroll 1
-        for (int b = 0; b < 32; ++b) {
-          const int i = 32 * word + b;
-          if (i >= nb) break;
-          uint32_t sides;
-          const int tok = block_slot(g, tc, br, i, &sides);
-          if (tok >= 0 && ((sides ^ combo) & last) == 0) bits |= 1u << b;
+          for (int base = row * g.ww; base < i1; base += g.ww, ++row) {
+            if (!row_ok(row)) continue;
+            const int lo = max(base, i0), hi = min(base + g.ww, i1);
+            const int len = hi - lo;
+            const uint32_t seg = bits_at(colok, lo - base) & (len >= 32 ? 0xffffffffu : ((1u << len) - 1u));
+            bits |= seg << (lo - i0);
+          }
         }
         tabs[s].mask[combo][word] = bits;
         __syncwarp();
@@ -464,16 +552,22 @@ window_attn_stream_kernel(const __grid_constant__ WinGeom g, const __grid_consta
         }
         tc_fence_after();
         const uint32_t sbase = tmem + lane_base + TS_S + 128u * buf + 64u * half;
+        // the block's key columns (slots rounded up to 16) of this thread's half, in groups
+        // of 8; the rest are never computed by the S MMA nor read by the PV MMA
+        const int ng = min(max((((block_rows(g, sp, kb).nr * g.ww + 15) & ~15) - 64 * half) >> 3, 0), 8);
+        // columns past the block hold stale values: their mask bits are 0
         float x[64];
 #pragma unroll
         for (int k = 0; k < 8; ++k) tmem_ld8(sbase + 8 * k, x + 8 * k);
         tmem_wait_ld();
 #pragma unroll
         for (int k = 0; k < 8; ++k) reg_fence8(x + 8 * k);
+        if (__any_sync(0xffffffffu, (mw0 & mw1) != 0xffffffffu)) {   // some key of the warp hidden
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          x[e] = selb(mw0, e, x[e]);
-          x[32 + e] = selb(mw1, e, x[32 + e]);
+          for (int e = 0; e < 32; ++e) {
+            x[e] = selb(mw0, e, x[e]);
+            x[32 + e] = selb(mw1, e, x[32 + e]);
+          }
         }
         float a = -INFINITY, b = -INFINITY;
 #pragma unroll
@@ -505,6 +599,7 @@ window_attn_stream_kernel(const __grid_constant__ WinGeom g, const __grid_consta
         const float2 cc = make_float2(c, c), nm = make_float2(-mu * c, -mu * c);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
+          if (2 * k >= ng) break;   // keys 16k .. of the half are past the block's columns
           uint32_t pk[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -567,20 +662,19 @@ window_attn_stream_kernel(const __grid_constant__ WinGeom g, const __grid_consta
   if (warp == kMmaWarpS) tmem_dealloc(tmem, 512);
 }
 
-// Block plan: as few blocks per T-slab as fit 128 slots each, rows spread evenly.
+// Block plan: as few blocks as fit 128 slots each, the window's rows spread evenly.
 StreamPlan make_plan(const WinGeom& g) {
   StreamPlan sp;
-  const int per_slab = g.wh * g.ww;
-  int groups = (per_slab + kBlk - 1) / kBlk;
-  sp.nh = (g.wh + groups - 1) / groups;
-  if (sp.nh * g.ww > kBlk) sp.nh = kBlk / g.ww;
-  sp.groups = (g.wh + sp.nh - 1) / sp.nh;
-  sp.nblk = g.wt * sp.groups;
+  const int rows = g.wt * g.wh;
+  const int per_block = kBlk / g.ww;                  // rows that fit one block (win_w <= 128)
+  sp.nblk = (rows + per_block - 1) / per_block;
+  sp.nr = (rows + sp.nblk - 1) / sp.nblk;
+  sp.nblk = (rows + sp.nr - 1) / sp.nr;
   sp.units = g.windows * g.heads * sp.nblk;
   return sp;
 }
 
-cudaError_t make_stream_maps(const WinGeom& g, const StreamPlan& sp, const void* const ptrs[3], TmaMaps* maps) {
+cudaError_t make_stream_maps(const WinGeom& g, const void* const ptrs[3], StreamMaps* maps) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
   const cuuint64_t C = static_cast<cuuint64_t>(g.heads) * g.head_dim;
@@ -589,15 +683,20 @@ cudaError_t make_stream_maps(const WinGeom& g, const StreamPlan& sp, const void*
   const cuuint64_t row = static_cast<cuuint64_t>(g.qkv_stride) * 2;
   const cuuint64_t strides[4] = {row, row * g.W, row * g.W * g.H, row * g.W * g.H * g.T};
   const cuuint32_t ww = static_cast<cuuint32_t>(g.ww), sw = static_cast<cuuint32_t>(g.sw);
-  const cuuint32_t nh = static_cast<cuuint32_t>(sp.nh);
-  const cuuint32_t nh_rem = static_cast<cuuint32_t>(g.wh - (sp.groups - 1) * sp.nh);
-  // a seam shape of an unshifted axis is never used and gets a whole row instead
-  const cuuint32_t boxwh[kBoxShapes][2] = {{ww, nh}, {ww, nh_rem}, {ww, 1}, {sw > 0 ? ww - sw : ww, 1},
-                                           {sw > 0 ? sw : ww, 1}};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   for (int t = 0; t < 3; ++t)
-    for (int b = 0; b < kBoxShapes; ++b) {
-      const cuuint32_t box[5] = {static_cast<cuuint32_t>(kRowBytes / 2), boxwh[b][0], boxwh[b][1], 1, 1};
+    for (int b = 0; b < kBoxShapesS; ++b) {
+      // 2^b rows of win_w tokens (a shape taller than any run of 128 slots is never used and
+      // is encoded one row high); a seam shape of an unshifted axis is never used either
+      cuuint32_t bw = ww, bh = 1;
+      if (b < kRowShapes) {
+        if ((static_cast<cuuint32_t>(1) << b) * ww <= static_cast<cuuint32_t>(kBlk)) bh = 1u << b;
+      } else if (b == kBoxW1) {
+        bw = sw > 0 ? ww - sw : ww;
+      } else {
+        bw = sw > 0 ? sw : ww;
+      }
+      const cuuint32_t box[5] = {static_cast<cuuint32_t>(kRowBytes / 2), bw, bh, 1, 1};
       CUresult r = enc(&maps->m[t][b], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptrs[t]), dims, strides,
                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -607,7 +706,7 @@ cudaError_t make_stream_maps(const WinGeom& g, const StreamPlan& sp, const void*
 }
 
 template <int HD, bool OUT_F32>
-cudaError_t launch_s(const WinGeom& g, const TmaMaps& maps, const StreamPlan& sp, void* o, int* err,
+cudaError_t launch_s(const WinGeom& g, const StreamMaps& maps, const StreamPlan& sp, void* o, int* err,
                      long long limit_ns, int num_sms, cudaStream_t st) {
   auto kern = window_attn_stream_kernel<HD, OUT_F32>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SmemS::kAlloc);
@@ -625,9 +724,9 @@ long long window_attn_stream_units(const WinGeom& g) { return make_plan(g).units
 cudaError_t launch_window_attn_stream(const WinGeom& g, const void* q, const void* k, const void* v, void* o,
                                       bool out_f32, int* err, long long spin_limit, int num_sms, cudaStream_t stream) {
   const StreamPlan sp = make_plan(g);
-  TmaMaps maps;
+  StreamMaps maps;
   const void* ptrs[3] = {q, k, v};
-  cudaError_t e = make_stream_maps(g, sp, ptrs, &maps);
+  cudaError_t e = make_stream_maps(g, ptrs, &maps);
   if (e != cudaSuccess) return e;
   if (g.head_dim == 64)
     return out_f32 ? launch_s<64, true>(g, maps, sp, o, err, spin_limit, num_sms, stream)
