@@ -434,6 +434,32 @@ def bench_configs(torch, s3w, dev, stream, peaks, reps):
                  "roofline": roofline(attn_bytes(w), attn_flops(w, big), a_med, peaks)}}
     del q, k, v, o
 
+    # QKV projection (the attention's prologue) on the stage-1 grid: 259,200 tokens x 512 ->
+    # 1536 (bf16, fp32 accumulate), then the attention on its grid-layout output
+    w = WORKLOADS["stage1"]
+    C, tokens, windows = geometry(w)
+    from swin3d_window_attention_b200 import inputs as _inp
+    x = _inp.normal_bf16_torch((w["B"], w["T"], w["H"], w["W"], C), dev, tensor_index=960)
+    wq = _inp.normal_bf16_torch((3 * C, C), dev, tensor_index=961, sigma=C ** -0.5)
+    bq = _inp.normal_f32_torch(3 * C, dev, tensor_index=962, sigma=0.1)
+    qkv = torch.empty((w["B"], w["T"], w["H"], w["W"], 3 * C), dtype=torch.bfloat16, device=dev)
+    o = torch.empty_like(x)
+    ms_p = timed(torch, stream, lambda: s3w.swin3d_qkv_proj_fwd(x, wq, bq, qkv), reps)
+    ms_c = timed(torch, stream, lambda: s3w.swin3d_qkv_window_attn_fwd(x, wq, bq, qkv, o, w["heads"], w["hd"], WINDOW,
+                                                                       SHIFTED), reps)
+    launches += len(ms_p) + 2 * len(ms_c)
+    p_med, c_med = statistics.median(ms_p), statistics.median(ms_c)
+    p_flops = 2 * tokens * C * 3 * C
+    p_bytes = tokens * C * 2 + 3 * C * C * 2 + tokens * 3 * C * 2
+    out["stage1_qkv_proj"] = {
+        "grid": "B=1 T4xH180xW360: 259,200 tokens x C=512 -> 3C=1536 (bf16 in/out, fp32 accumulate, bias), then "
+                "the shifted-window attention on the projection's [tokens][3C] output",
+        "proj": {**launch_stats(ms_p), "bytes": p_bytes, "flops": p_flops, "tflops": p_flops / (p_med * 1e-3) / 1e12,
+                 "roofline": roofline(p_bytes, p_flops, p_med, peaks)},
+        "proj_then_attn_ms": launch_stats(ms_c),
+        "windows_per_s": windows / (c_med * 1e-3)}
+    del x, wq, bq, qkv, o
+
     # fused attention + AdaLN (one kernel per block) on the stage-1 grid: one launch, and the
     # headline step (two blocks) made of fused calls against the two-call step
     w = WORKLOADS["stage1"]

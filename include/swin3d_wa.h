@@ -222,6 +222,53 @@ int swin3d_window_attn_adaln_fwd_static_ws(const void* q, const void* k, const v
                                            int heads, int head_dim, float attn_scale, float eps,
                                            s3w_stream_t stream);
 
+/*
+ * QKV projection of grid-layout tokens, the prologue of the window attention:
+ *   qkv[l][n] = sum_c x[l][c] * w_qkv[n][c] (+ b_qkv[n]),   n < 3C,
+ * bf16 operands, fp32 accumulation on the tensor cores, bf16 output rounded to nearest even.
+ * Features n = 0..C-1 are q, C..2C-1 are k, 2C..3C-1 are v, each in head-major order
+ * (channel head * head_dim + d), the layout swin3d_window_attn_fwd reads with token stride 3C.
+ *
+ * Defines: "Flash-Aurora: Toward Efficient Inference for Geospatial Foundation Models",
+ * section "Mixed-precision inference" (bf16_mixed backbone: BF16 QKV projection feeding the
+ * BF16 attention).
+ *
+ * x       device bf16 [tokens][C] (grid layout, contiguous), 16-byte aligned.
+ * w_qkv   device bf16 [3C][C] (the Linear weight: output features x input channels), 16-byte
+ *         aligned.
+ * b_qkv   device fp32 [3C] or NULL (no bias), 16-byte aligned.
+ * qkv     device bf16 [tokens][3C], 32-byte aligned, owned by the caller; must not overlap x,
+ *         w_qkv or b_qkv.
+ * tokens  1 .. 2^31 - 1.   C: a multiple of 32, <= 16384.
+ * Returns S3W_OK or an s3w_status; on error nothing is launched.
+ */
+int swin3d_qkv_proj_fwd(const void* x, const void* w_qkv, const float* b_qkv, void* qkv, long long tokens, int C,
+                        s3w_stream_t stream);
+
+/*
+ * The QKV projection followed by the shifted-window attention on its output: the attention
+ * gathers its windows straight from the projection's grid-layout [tokens][3C] buffer (shift,
+ * pad and partition folded into its loads), so no layout pass sits between the two launches.
+ *
+ * Defines: the two calls above ("Flash-Aurora: Toward Efficient Inference for Geospatial
+ * Foundation Models", sections "Mixed-precision inference" and "Kernel fusion for backbone
+ * memory traffic": no eager shift / pad / partition copies between projection and attention).
+ *
+ * x, w_qkv, b_qkv  as swin3d_qkv_proj_fwd, with C = heads * head_dim and tokens = B T H W.
+ * qkv     device bf16 [B][T][H][W][3C] workspace (also an output: the projected q, k, v),
+ *         32-byte aligned, owned by the caller.
+ * o       device out_dtype (S3W_BF16 or S3W_F32) [B][T][H][W][C], token stride C; must not
+ *         overlap qkv.
+ * Grid, window, shift, heads, head_dim (32 or 64) and attn_scale: as swin3d_window_attn_fwd.
+ * Every argument of both launches is checked before the first; on error nothing is launched.
+ */
+int swin3d_qkv_window_attn_fwd(const void* x, const void* w_qkv, const float* b_qkv, void* qkv, void* o,
+                               int out_dtype, int B, int T, int H, int W,
+                               int win_t, int win_h, int win_w,
+                               int shift_t, int shift_h, int shift_w,
+                               int heads, int head_dim, float attn_scale,
+                               s3w_stream_t stream);
+
 /* Static English text for a status code (never NULL). */
 const char* s3w_status_string(int status);
 

@@ -16,6 +16,9 @@ Parity status of each function (what pins it, in ``tests/test_oracle.py``):
   * ``dense_masked_attn`` pinned against the same PyTorch route and the group sizes.
   * ``adaln``             pinned: ``torch.nn.functional.layer_norm`` in fp64, a
     constant row, zero-input closed form.
+  * ``qkv_proj``          pinned: a permutation weight returns the permuted channels
+    (a transposed weight or swapped q/k/v thirds fails it), a zero input returns the
+    bias, additivity in x, and the q/k/v thirds equal three separate projections.
 """
 from __future__ import annotations
 
@@ -175,3 +178,25 @@ def adaln(x, residual, scale, shift, eps=1e-5, film_form=0):
     if rc != 0:
         raise ValueError("oracle rejected the AdaLN arguments")
     return out
+
+
+def _as_f64(a):
+    """bf16 bits (uint16) widened exactly, or a float array as doubles."""
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def qkv_proj(x, w, b=None):
+    """QKV projection of grid-layout tokens ("Flash-Aurora: Toward Efficient Inference for
+    Geospatial Foundation Models", section "Mixed-precision inference": the BF16 QKV
+    projection ahead of the window attention): ``x`` ``[..., C]`` and ``w`` ``[3C, C]``
+    (bf16 bits or floats), ``b`` ``[3C]`` or None.  Returns ``x w^T + b`` in doubles,
+    ``[..., 3C]``; one fp64 matrix product (a library primitive) and the bias add."""
+    xf, wf = _as_f64(x), _as_f64(w)
+    assert wf.ndim == 2 and wf.shape[1] == xf.shape[-1] and wf.shape[0] == 3 * wf.shape[1]
+    y = xf.reshape(-1, xf.shape[-1]) @ wf.T
+    if b is not None:
+        y = y + np.asarray(b, dtype=np.float64)[None, :]
+    return y.reshape(*xf.shape[:-1], wf.shape[0])

@@ -17,5 +17,7 @@ from .api import (  # noqa: F401
     swin3d_window_attn_adaln_fwd_static_ws,
     swin3d_window_attn_fwd,
     swin3d_window_attn_fwd_legacy_mma,
+    swin3d_qkv_proj_fwd,
+    swin3d_qkv_window_attn_fwd,
     window_attn_adaln_workspace_bytes,
 )

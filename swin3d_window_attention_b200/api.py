@@ -62,6 +62,10 @@ def load_library():
     lib.swin3d_window_attn_adaln_workspace_bytes.restype = LL
     lib.swin3d_window_attn_adaln_fwd_static_ws.argtypes = [P, P, P, LL, P, P, P, P, I, P] + [I] * 12 + [F, F, P]
     lib.swin3d_window_attn_adaln_fwd_static_ws.restype = I
+    lib.swin3d_qkv_proj_fwd.argtypes = [P, P, P, P, LL, I, P]
+    lib.swin3d_qkv_proj_fwd.restype = I
+    lib.swin3d_qkv_window_attn_fwd.argtypes = [P, P, P, P, P, I] + [I] * 12 + [F, P]
+    lib.swin3d_qkv_window_attn_fwd.restype = I
     _lib = lib
     return lib
 
@@ -207,6 +211,48 @@ def swin3d_window_attn_adaln_fwd_static_ws(q, k, v, residual, scale, shift, out,
                                                     float(eps), st)
     if check and rc != S3W_OK:
         raise S3WError(rc, "swin3d_window_attn_adaln_fwd_static_ws")
+    return rc
+
+
+def swin3d_qkv_proj_fwd(x, w, b, qkv, stream=None, check: bool = True) -> int:
+    """QKV projection on the tensor cores.  x: contiguous bf16 [..., C]; w: contiguous bf16
+    [3C, C]; b: fp32 [3C] or None; qkv: contiguous bf16 [..., 3C] (the same leading shape)."""
+    lib = load_library()
+    C = x.shape[-1]
+    tokens = x.numel() // C
+    for t in (x, w, qkv):
+        if not t.is_contiguous():
+            raise ValueError("x, w and qkv must be contiguous")
+    if tuple(w.shape) != (3 * C, C) or qkv.numel() != tokens * 3 * C or qkv.shape[-1] != 3 * C:
+        raise ValueError("w must be [3C, C] and qkv [..., 3C]")
+    st = _stream_of(x) if stream is None else stream
+    rc = lib.swin3d_qkv_proj_fwd(x.data_ptr(), w.data_ptr(), None if b is None else b.data_ptr(), qkv.data_ptr(),
+                                 tokens, C, st)
+    if check and rc != S3W_OK:
+        raise S3WError(rc, "swin3d_qkv_proj_fwd")
+    return rc
+
+
+def swin3d_qkv_window_attn_fwd(x, w, b, qkv, o, heads: int, head_dim: int, window=(2, 6, 12), shift=(0, 0, 0),
+                               scale: float = 0.0, stream=None, check: bool = True) -> int:
+    """QKV projection followed by the shifted-window attention on its output.  x: contiguous bf16
+    [B, T, H, W, C]; w: bf16 [3C, C]; b: fp32 [3C] or None; qkv: bf16 [B, T, H, W, 3C]
+    workspace (holds the projected q, k, v afterwards); o: bf16 or fp32 [B, T, H, W, C]."""
+    lib = load_library()
+    B, T, H, W, C = x.shape
+    if C != heads * head_dim:
+        raise ValueError("x must have heads * head_dim channels")
+    for t in (x, w, qkv, o):
+        if not t.is_contiguous():
+            raise ValueError("x, w, qkv and o must be contiguous")
+    if tuple(qkv.shape) != (B, T, H, W, 3 * C) or tuple(o.shape) != (B, T, H, W, C) or tuple(w.shape) != (3 * C, C):
+        raise ValueError("qkv must be [B, T, H, W, 3C], o [B, T, H, W, C] and w [3C, C]")
+    st = _stream_of(x) if stream is None else stream
+    rc = lib.swin3d_qkv_window_attn_fwd(x.data_ptr(), w.data_ptr(), None if b is None else b.data_ptr(),
+                                        qkv.data_ptr(), o.data_ptr(), _dtype_code(o), B, T, H, W, *window, *shift,
+                                        heads, head_dim, float(scale), st)
+    if check and rc != S3W_OK:
+        raise S3WError(rc, "swin3d_qkv_window_attn_fwd")
     return rc
 
 

@@ -257,6 +257,60 @@ int swin3d_window_attn_adaln_fwd(const void* q, const void* k, const void* v, lo
   return e == cudaSuccess ? S3W_OK : S3W_ERR_CUDA;
 }
 
+int swin3d_qkv_proj_fwd(const void* x, const void* w_qkv, const float* b_qkv, void* qkv, long long tokens, int C,
+                        s3w_stream_t stream) {
+  if (!x || !w_qkv || !qkv) return S3W_ERR_INVALID_ARG;
+  if (tokens < 1 || C < 1) return S3W_ERR_INVALID_ARG;
+  if (C % 32 != 0 || C > 16384) return S3W_ERR_UNSUPPORTED;
+  if (tokens > INT32_MAX) return S3W_ERR_UNSUPPORTED;   // TMA row coordinates are 32-bit
+  if (!aligned16(x) || !aligned16(w_qkv) || (b_qkv && !aligned16(b_qkv)) ||
+      (reinterpret_cast<uintptr_t>(qkv) & 31u) != 0)
+    return S3W_ERR_MISALIGNED;
+  // qkv must not overlap x, w or the bias
+  const char* q0 = static_cast<const char*>(qkv);
+  const long long qbytes = tokens * 3 * C * 2;
+  auto overlaps = [&](const void* p, long long bytes) {
+    const char* a = static_cast<const char*>(p);
+    return a < q0 + qbytes && q0 < a + bytes;
+  };
+  if (overlaps(x, tokens * C * 2) || overlaps(w_qkv, 3ll * C * C * 2) || (b_qkv && overlaps(b_qkv, 3ll * C * 4)))
+    return S3W_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != S3W_OK) return rc;
+  cudaError_t e = s3w::launch_qkv_gemm(x, w_qkv, b_qkv, qkv, tokens, C, ds->err,
+                                       g_wait_limit_ns.load(std::memory_order_relaxed), ds->num_sms,
+                                       g_test_stall.load(std::memory_order_relaxed),
+                                       reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? S3W_OK : S3W_ERR_CUDA;
+}
+
+int swin3d_qkv_window_attn_fwd(const void* x, const void* w_qkv, const float* b_qkv, void* qkv, void* o,
+                               int out_dtype, int B, int T, int H, int W, int win_t, int win_h, int win_w,
+                               int shift_t, int shift_h, int shift_w, int heads, int head_dim, float attn_scale,
+                               s3w_stream_t stream) {
+  if (!x || !w_qkv || !qkv || !o) return S3W_ERR_INVALID_ARG;
+  if (B < 1 || T < 1 || H < 1 || W < 1 || heads < 1 || head_dim < 1) return S3W_ERR_INVALID_ARG;
+  const long long C = static_cast<long long>(heads) * head_dim;
+  if (C > 16384) return S3W_ERR_UNSUPPORTED;
+  // every check of the attention call first (geometry, dtypes, sizes: B T H W <= 2^31 - 1),
+  // so that nothing is launched unless both launches are valid; the projection's follow
+  s3w::WinGeom g;
+  const char* qkvc = static_cast<const char*>(qkv);
+  int rc = make_geometry(qkvc, qkvc + C * 2, qkvc + 2 * C * 2, o, B, T, H, W, win_t, win_h, win_w, shift_t, shift_h,
+                         shift_w, heads, head_dim, 3 * C, C, attn_scale, S3W_BF16, out_dtype, &g);
+  if (rc != S3W_OK) return rc;
+  const long long tokens = static_cast<long long>(B) * T * H * W;
+  // o must not overlap the projection's output, which the attention reads
+  const char* o0 = static_cast<const char*>(o);
+  const long long ob = out_dtype == S3W_F32 ? 4 : 2;
+  if (o0 < qkvc + tokens * 3 * C * 2 && qkvc < o0 + tokens * C * ob) return S3W_ERR_INVALID_ARG;
+  rc = swin3d_qkv_proj_fwd(x, w_qkv, b_qkv, qkv, tokens, static_cast<int>(C), stream);
+  if (rc != S3W_OK) return rc;
+  return swin3d_window_attn_fwd(qkvc, qkvc + C * 2, qkvc + 2 * C * 2, o, B, T, H, W, win_t, win_h, win_w, shift_t,
+                                shift_h, shift_w, heads, head_dim, 3 * C, C, attn_scale, S3W_BF16, out_dtype, stream);
+}
+
 int adaln_residual_fwd(const void* x, int x_dtype, const float* residual, const float* scale, const float* shift,
                        void* out, int out_dtype, int B, long long tokens_per_sample, int C, float eps,
                        s3w_stream_t stream) {

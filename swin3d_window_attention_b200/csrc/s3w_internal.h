@@ -44,6 +44,12 @@ cudaError_t launch_window_attn_stream(const WinGeom& g, const void* q, const voi
                                       cudaStream_t stream);
 long long window_attn_stream_units(const WinGeom& g);
 
+// QKV projection (qkv_gemm.cu): qkv[l][n] = sum_c x[l][c] w[n][c] (+ bias[n]) for n < 3C, bf16
+// in and out, fp32 accumulation, on the tensor cores.  x: [tokens][C], w: [3C][C], qkv:
+// [tokens][3C]; C a multiple of 32.
+cudaError_t launch_qkv_gemm(const void* x, const void* w, const float* bias, void* qkv, long long tokens, int C,
+                            int* err, long long spin_limit, int num_sms, int test_stall, cudaStream_t stream);
+
 // Window attention on the legacy warp-level mma.sync path (attn_mma.cu); kept as the
 // measured baseline the tcgen05 kernel is compared with.
 cudaError_t launch_window_attn_mma(const WinGeom& g, const void* q, const void* k, const void* v,

@@ -297,3 +297,46 @@ def test_adaln_zero_film_closed_form():
     var = x.var(axis=-1)
     np.testing.assert_allclose(got.mean(axis=-1), 0.0, atol=1e-14)
     np.testing.assert_allclose(got.var(axis=-1), var / (var + eps), rtol=1e-12)
+
+
+# ---------------------------------------------------------------------------- QKV projection
+def test_qkv_proj_permutation_weight_returns_permuted_channels():
+    """w[n][c] = 1 iff c = perm(n): the output is x at the permuted channels.  A transposed
+    weight (x w instead of x w^T) or swapped q/k/v thirds give other channels."""
+    rng = np.random.default_rng(1)
+    C = 8
+    x = rng.standard_normal((5, C))
+    perm = rng.integers(0, C, size=3 * C)
+    w = np.zeros((3 * C, C))
+    w[np.arange(3 * C), perm] = 1.0
+    y = oracle.qkv_proj(x, w)
+    assert y.shape == (5, 3 * C)
+    np.testing.assert_array_equal(y, x[:, perm])
+
+
+def test_qkv_proj_zero_input_gives_bias_and_is_additive():
+    rng = np.random.default_rng(2)
+    C = 16
+    w = rng.standard_normal((3 * C, C))
+    b = rng.standard_normal(3 * C)
+    np.testing.assert_array_equal(oracle.qkv_proj(np.zeros((4, C)), w, b), np.broadcast_to(b, (4, 3 * C)))
+    x1, x2 = rng.standard_normal((6, C)), rng.standard_normal((6, C))
+    lhs = oracle.qkv_proj(x1 + x2, w, b)
+    rhs = oracle.qkv_proj(x1, w, b) + oracle.qkv_proj(x2, w, b) - b
+    np.testing.assert_allclose(lhs, rhs, rtol=0, atol=1e-12)
+
+
+def test_qkv_proj_thirds_are_the_q_k_v_projections_and_bf16_bits_widen_exactly():
+    """The three thirds of the output are the projections by the three row blocks of w (grid
+    shape kept), and bf16 bit patterns enter as their exact values."""
+    from swin3d_window_attention_b200 import inputs
+
+    C = 32
+    xb = inputs.normal_bf16_bits((2, 3, 4, C), tensor_index=91)
+    wb = inputs.normal_bf16_bits((3 * C, C), tensor_index=92)
+    y = oracle.qkv_proj(xb, wb)
+    assert y.shape == (2, 3, 4, 3 * C)
+    xf, wf = inputs.bf16_bits_to_f32(xb).astype(np.float64), inputs.bf16_bits_to_f32(wb).astype(np.float64)
+    for j in range(3):
+        part = oracle.qkv_proj(xf, np.concatenate([wf[j * C:(j + 1) * C]] * 3))[..., :C]
+        np.testing.assert_allclose(y[..., j * C:(j + 1) * C], part, rtol=0, atol=1e-12)
