@@ -347,201 +347,236 @@ def timed(torch, stream, fn, reps, warmup=3):
     return [a.elapsed_time(b) for a, b in ev]
 
 
-def bench_configs(torch, s3w, dev, stream, peaks, reps):
-    """Every workload of the set besides the headline, each timed on its own."""
+def bench_configs(torch, s3w, dev, stream, peaks, reps, only=None):
+    """Every workload of the set besides the headline, each timed on its own (or only the one
+    named by ``only``)."""
+
+    def want(name):
+        return only is None or only == name
+
     out = {}
     launches = 0
-    # tiny grid: launch-bound, latency reported
-    w = WORKLOADS["tiny"]
-    q, k, v = device_qkv(torch, w, dev, 900)
-    o = torch.empty_like(q)
-    ms = timed(torch, stream, lambda: s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTED),
-               reps)
-    launches += len(ms)
-    out["tiny"] = {"grid": "B=1 T2xH15xW30 (padded 2x18x36), 2 heads x 32, shift (1,3,6), 9 windows",
-                   "attn": launch_stats(ms), "latency_us_median": 1e3 * statistics.median(ms)}
-    del q, k, v, o
+    if want("tiny"):
+        # tiny grid: launch-bound, latency reported
+        w = WORKLOADS["tiny"]
+        q, k, v = device_qkv(torch, w, dev, 900)
+        o = torch.empty_like(q)
+        ms = timed(torch, stream, lambda: s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTED),
+                   reps)
+        launches += len(ms)
+        out["tiny"] = {"grid": "B=1 T2xH15xW30 (padded 2x18x36), 2 heads x 32, shift (1,3,6), 9 windows",
+                       "attn": launch_stats(ms), "latency_us_median": 1e3 * statistics.median(ms)}
+        del q, k, v, o
 
-    # stage 2: shifted attention + AdaLN at C = 1024
-    w = WORKLOADS["stage2"]
-    C, tokens, windows = geometry(w)
-    q, k, v = device_qkv(torch, w, dev, 910)
-    sc, sh, res = device_film(torch, w, dev, 920, 0.1)
-    o = torch.empty_like(q)
-    ms_a = timed(torch, stream, lambda: s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTED),
-                 reps)
-    x = o.view(w["B"], tokens // w["B"], C)
-    ms_n = timed(torch, stream, lambda: s3w.adaln_residual_fwd(x, res, sc, sh, res, eps=1e-5), reps)
-    launches += len(ms_a) + len(ms_n)
-    a_med, n_med = statistics.median(ms_a), statistics.median(ms_n)
-    out["stage2"] = {"grid": "B=1 T4xH90xW180, 16 heads x 64, shift (1,3,6), 450 windows; AdaLN C=1024 fp32 out",
-                     "attn": {**launch_stats(ms_a), "bytes": attn_bytes(w), "flops": attn_flops(w),
-                              "windows_per_s": windows / (a_med * 1e-3),
-                              "roofline": roofline(attn_bytes(w), attn_flops(w), a_med, peaks)},
-                     "adaln": {**launch_stats(ms_n), "bytes": adaln_bytes(w),
-                               "roofline": roofline(adaln_bytes(w), 0, n_med, peaks)}}
-    del q, k, v, o, x, sc, sh, res
+    if want("stage2"):
+        # stage 2: shifted attention + AdaLN at C = 1024
+        w = WORKLOADS["stage2"]
+        C, tokens, windows = geometry(w)
+        q, k, v = device_qkv(torch, w, dev, 910)
+        sc, sh, res = device_film(torch, w, dev, 920, 0.1)
+        o = torch.empty_like(q)
+        ms_a = timed(torch, stream, lambda: s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTED),
+                     reps)
+        x = o.view(w["B"], tokens // w["B"], C)
+        ms_n = timed(torch, stream, lambda: s3w.adaln_residual_fwd(x, res, sc, sh, res, eps=1e-5), reps)
+        launches += len(ms_a) + len(ms_n)
+        a_med, n_med = statistics.median(ms_a), statistics.median(ms_n)
+        out["stage2"] = {"grid": "B=1 T4xH90xW180, 16 heads x 64, shift (1,3,6), 450 windows; AdaLN C=1024 fp32 out",
+                         "attn": {**launch_stats(ms_a), "bytes": attn_bytes(w), "flops": attn_flops(w),
+                                  "windows_per_s": windows / (a_med * 1e-3),
+                                  "roofline": roofline(attn_bytes(w), attn_flops(w), a_med, peaks)},
+                         "adaln": {**launch_stats(ms_n), "bytes": adaln_bytes(w),
+                                   "roofline": roofline(adaln_bytes(w), 0, n_med, peaks)}}
+        del q, k, v, o, x, sc, sh, res
 
-    # stage 3: padded grid (45 -> 48, 90 -> 96), padded keys masked, padded outputs dropped
-    w = WORKLOADS["stage3_padded"]
-    _, _, windows = geometry(w)
-    q, k, v = device_qkv(torch, w, dev, 930)
-    o = torch.empty_like(q)
-    ms_a = timed(torch, stream, lambda: s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTED),
-                 reps)
-    launches += len(ms_a)
-    a_med = statistics.median(ms_a)
-    out["stage3_padded"] = {
-        "grid": "B=2 T4xH45xW90 (padded 4x48x96), 32 heads x 64, shift (1,3,6), 256 windows",
-        "attn": {**launch_stats(ms_a), "bytes": attn_bytes(w), "flops": attn_flops(w),
-                 "windows_per_s": windows / (a_med * 1e-3),
-                 "roofline": roofline(attn_bytes(w), attn_flops(w), a_med, peaks)}}
-    del q, k, v, o
+    if want("stage3_padded"):
+        # stage 3: padded grid (45 -> 48, 90 -> 96), padded keys masked, padded outputs dropped
+        w = WORKLOADS["stage3_padded"]
+        _, _, windows = geometry(w)
+        q, k, v = device_qkv(torch, w, dev, 930)
+        o = torch.empty_like(q)
+        ms_a = timed(torch, stream, lambda: s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTED),
+                     reps)
+        launches += len(ms_a)
+        a_med = statistics.median(ms_a)
+        out["stage3_padded"] = {
+            "grid": "B=2 T4xH45xW90 (padded 4x48x96), 32 heads x 64, shift (1,3,6), 256 windows",
+            "attn": {**launch_stats(ms_a), "bytes": attn_bytes(w), "flops": attn_flops(w),
+                     "windows_per_s": windows / (a_med * 1e-3),
+                     "roofline": roofline(attn_bytes(w), attn_flops(w), a_med, peaks)}}
+        del q, k, v, o
 
-    # TF32_ACC_FP32 mode on the stage-1 grid: fp32 Q/K/V in, fp32 O out
-    w = WORKLOADS["stage1"]
-    C, tokens, windows = geometry(w)
-    q, k, v = (inputs_f32(torch, w, dev, 940 + j) for j in range(3))
-    o = torch.empty_like(q)
-    ms_a = timed(torch, stream, lambda: s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTED),
-                 reps)
-    launches += len(ms_a)
-    a_med = statistics.median(ms_a)
-    nbytes = attn_bytes(w, o_bytes=4, in_bytes=4)
-    out["stage1_tf32"] = {
-        "grid": "B=1 T4xH180xW360, 8 heads x 64, shift (1,3,6), 1800 windows; fp32 Q/K/V/O, TF32 MMAs (TF32_ACC_FP32)",
-        "attn": {**launch_stats(ms_a), "bytes": nbytes, "flops": attn_flops(w), "windows_per_s": windows / (a_med * 1e-3),
-                 "roofline": roofline(nbytes, attn_flops(w), a_med,
-                                      {**peaks, "bf16_tflops": peaks["bf16_tflops"] / 2})}}
-    del q, k, v, o
+    if want("stage1_tf32"):
+        # TF32_ACC_FP32 mode on the stage-1 grid: fp32 Q/K/V in, fp32 O out
+        w = WORKLOADS["stage1"]
+        C, tokens, windows = geometry(w)
+        q, k, v = (inputs_f32(torch, w, dev, 940 + j) for j in range(3))
+        o = torch.empty_like(q)
+        ms_a = timed(torch, stream, lambda: s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTED),
+                     reps)
+        launches += len(ms_a)
+        a_med = statistics.median(ms_a)
+        nbytes = attn_bytes(w, o_bytes=4, in_bytes=4)
+        out["stage1_tf32"] = {
+            "grid": "B=1 T4xH180xW360, 8 heads x 64, shift (1,3,6), 1800 windows; fp32 Q/K/V/O, TF32 MMAs (TF32_ACC_FP32)",
+            "attn": {**launch_stats(ms_a), "bytes": nbytes, "flops": attn_flops(w), "windows_per_s": windows / (a_med * 1e-3),
+                     "roofline": roofline(nbytes, attn_flops(w), a_med,
+                                          {**peaks, "bf16_tflops": peaks["bf16_tflops"] / 2})}}
+        del q, k, v, o
 
-    # windows larger than one tile: the streaming path on the stage-1 grid with (2,12,12)
-    # windows (N = 288), shift (1,6,6)
-    w = WORKLOADS["stage1"]
-    big = (2, 12, 12)
-    C, tokens, windows = geometry(w, big)
-    q, k, v = device_qkv(torch, w, dev, 945)
-    o = torch.empty_like(q)
-    ms_a = timed(torch, stream, lambda: s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], big, (1, 6, 6)),
-                 reps)
-    launches += len(ms_a)
-    a_med = statistics.median(ms_a)
-    out["stage1_window_2x12x12"] = {
-        "grid": "B=1 T4xH180xW360, 8 heads x 64, window (2,12,12) N=288, shift (1,6,6), 900 windows; streaming "
-                "path (K/V blocks of 72 slots, online softmax)",
-        "attn": {**launch_stats(ms_a), "bytes": attn_bytes(w), "flops": attn_flops(w, big),
-                 "windows_per_s": windows / (a_med * 1e-3),
-                 "roofline": roofline(attn_bytes(w), attn_flops(w, big), a_med, peaks)}}
-    del q, k, v, o
+    if want("stage1_window_2x12x12"):
+        # windows larger than one tile: the streaming path on the stage-1 grid with (2,12,12)
+        # windows (N = 288), shift (1,6,6)
+        w = WORKLOADS["stage1"]
+        big = (2, 12, 12)
+        C, tokens, windows = geometry(w, big)
+        q, k, v = device_qkv(torch, w, dev, 945)
+        o = torch.empty_like(q)
+        ms_a = timed(torch, stream, lambda: s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], big, (1, 6, 6)),
+                     reps)
+        launches += len(ms_a)
+        a_med = statistics.median(ms_a)
+        out["stage1_window_2x12x12"] = {
+            "grid": "B=1 T4xH180xW360, 8 heads x 64, window (2,12,12) N=288, shift (1,6,6), 900 windows; streaming "
+                    "path (K/V blocks of 72 slots, online softmax)",
+            "attn": {**launch_stats(ms_a), "bytes": attn_bytes(w), "flops": attn_flops(w, big),
+                     "windows_per_s": windows / (a_med * 1e-3),
+                     "roofline": roofline(attn_bytes(w), attn_flops(w, big), a_med, peaks)}}
+        del q, k, v, o
 
-    # QKV projection (the attention's prologue) on the stage-1 grid: 259,200 tokens x 512 ->
-    # 1536 (bf16, fp32 accumulate), then the attention on its grid-layout output
-    w = WORKLOADS["stage1"]
-    C, tokens, windows = geometry(w)
-    from swin3d_window_attention_b200 import inputs as _inp
-    x = _inp.normal_bf16_torch((w["B"], w["T"], w["H"], w["W"], C), dev, tensor_index=960)
-    wq = _inp.normal_bf16_torch((3 * C, C), dev, tensor_index=961, sigma=C ** -0.5)
-    bq = _inp.normal_f32_torch(3 * C, dev, tensor_index=962, sigma=0.1)
-    qkv = torch.empty((w["B"], w["T"], w["H"], w["W"], 3 * C), dtype=torch.bfloat16, device=dev)
-    o = torch.empty_like(x)
-    ms_p = timed(torch, stream, lambda: s3w.swin3d_qkv_proj_fwd(x, wq, bq, qkv), reps)
-    ms_c = timed(torch, stream, lambda: s3w.swin3d_qkv_window_attn_fwd(x, wq, bq, qkv, o, w["heads"], w["hd"], WINDOW,
-                                                                       SHIFTED), reps)
-    launches += len(ms_p) + 2 * len(ms_c)
-    p_med, c_med = statistics.median(ms_p), statistics.median(ms_c)
-    p_flops = 2 * tokens * C * 3 * C
-    p_bytes = tokens * C * 2 + 3 * C * C * 2 + tokens * 3 * C * 2
-    out["stage1_qkv_proj"] = {
-        "grid": "B=1 T4xH180xW360: 259,200 tokens x C=512 -> 3C=1536 (bf16 in/out, fp32 accumulate, bias), then "
-                "the shifted-window attention on the projection's [tokens][3C] output",
-        "proj": {**launch_stats(ms_p), "bytes": p_bytes, "flops": p_flops, "tflops": p_flops / (p_med * 1e-3) / 1e12,
-                 "roofline": roofline(p_bytes, p_flops, p_med, peaks)},
-        "proj_then_attn_ms": launch_stats(ms_c),
-        "windows_per_s": windows / (c_med * 1e-3)}
-    del x, wq, bq, qkv, o
+    if want("stage1_qkv_proj"):
+        # QKV projection (the attention's prologue) on the stage-1 grid: 259,200 tokens x 512 ->
+        # 1536 (bf16, fp32 accumulate), then the attention on its grid-layout output
+        w = WORKLOADS["stage1"]
+        C, tokens, windows = geometry(w)
+        from swin3d_window_attention_b200 import inputs as _inp
+        x = _inp.normal_bf16_torch((w["B"], w["T"], w["H"], w["W"], C), dev, tensor_index=960)
+        wq = _inp.normal_bf16_torch((3 * C, C), dev, tensor_index=961, sigma=C ** -0.5)
+        bq = _inp.normal_f32_torch(3 * C, dev, tensor_index=962, sigma=0.1)
+        qkv = torch.empty((w["B"], w["T"], w["H"], w["W"], 3 * C), dtype=torch.bfloat16, device=dev)
+        o = torch.empty_like(x)
+        ms_p = timed(torch, stream, lambda: s3w.swin3d_qkv_proj_fwd(x, wq, bq, qkv), reps)
+        ms_c = timed(torch, stream, lambda: s3w.swin3d_qkv_window_attn_fwd(x, wq, bq, qkv, o, w["heads"], w["hd"], WINDOW,
+                                                                           SHIFTED), reps)
+        launches += len(ms_p) + 2 * len(ms_c)
+        p_med, c_med = statistics.median(ms_p), statistics.median(ms_c)
+        p_flops = 2 * tokens * C * 3 * C
+        p_bytes = tokens * C * 2 + 3 * C * C * 2 + tokens * 3 * C * 2
+        out["stage1_qkv_proj"] = {
+            "grid": "B=1 T4xH180xW360: 259,200 tokens x C=512 -> 3C=1536 (bf16 in/out, fp32 accumulate, bias), then "
+                    "the shifted-window attention on the projection's [tokens][3C] output",
+            "proj": {**launch_stats(ms_p), "bytes": p_bytes, "flops": p_flops, "tflops": p_flops / (p_med * 1e-3) / 1e12,
+                     "roofline": roofline(p_bytes, p_flops, p_med, peaks)},
+            "proj_then_attn_ms": launch_stats(ms_c),
+            "windows_per_s": windows / (c_med * 1e-3)}
+        del x, wq, bq, qkv, o
 
-    # fused attention + AdaLN (one kernel per block) on the stage-1 grid: one launch, and the
-    # headline step (two blocks) made of fused calls against the two-call step
-    w = WORKLOADS["stage1"]
-    C, tokens, windows = geometry(w)
-    qkv = [device_qkv(torch, w, dev, 950 + 10 * b) for b in range(2)]
-    films = [device_film(torch, w, dev, 970 + 10 * b, 0.1)[:2] for b in range(2)]
-    res = device_film(torch, w, dev, 990, 1.0)[2]
-    o = torch.empty_like(qkv[0][0])
-    x = o.view(w["B"], tokens // w["B"], C)
-    ws = torch.empty(s3w.window_attn_adaln_workspace_bytes(w["B"], w["T"], w["H"], w["W"], w["heads"], w["hd"],
-                                                           WINDOW), dtype=torch.uint8, device=dev)
+    if want("stage1_fused"):
+        # fused attention + AdaLN (one kernel per block) on the stage-1 grid: one launch, and the
+        # headline step (two blocks) made of fused calls against the two-call step
+        w = WORKLOADS["stage1"]
+        C, tokens, windows = geometry(w)
+        qkv = [device_qkv(torch, w, dev, 950 + 10 * b) for b in range(2)]
+        films = [device_film(torch, w, dev, 970 + 10 * b, 0.1)[:2] for b in range(2)]
+        res = device_film(torch, w, dev, 990, 1.0)[2]
+        o = torch.empty_like(qkv[0][0])
+        x = o.view(w["B"], tokens // w["B"], C)
+        ws = torch.empty(s3w.window_attn_adaln_workspace_bytes(w["B"], w["T"], w["H"], w["W"], w["heads"], w["hd"],
+                                                               WINDOW), dtype=torch.uint8, device=dev)
 
-    def fused_call(b):
-        q, k, v = qkv[b]
-        s3w.swin3d_window_attn_adaln_fwd(q, k, v, res, films[b][0], films[b][1], res, w["heads"], w["hd"], WINDOW,
-                                         SHIFTS[b], workspace=ws, eps=1e-5)
-
-    def two_call_block(b):
-        q, k, v = qkv[b]
-        s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTS[b])
-        s3w.adaln_residual_fwd(x, res, films[b][0], films[b][1], res, eps=1e-5)
-
-    ms_f = timed(torch, stream, lambda: fused_call(1), reps)
-    ms_fs = timed(torch, stream, lambda: [fused_call(b) for b in range(2)], reps)
-    ms_ts = timed(torch, stream, lambda: [two_call_block(b) for b in range(2)], reps)
-    launches += len(ms_f) + 2 * len(ms_fs) + 4 * len(ms_ts)
-    f_med = statistics.median(ms_f)
-    nbytes = fused_bytes(w)
-    out["stage1_fused"] = {
-        "grid": "B=1 T4xH180xW360, 8 heads x 64, shift (1,3,6), 1800 windows; attention + AdaLN in one kernel, "
-                "fp32 residual in place",
-        "fused": {**launch_stats(ms_f), "bytes": nbytes, "flops": attn_flops(w), "windows_per_s": windows / (f_med * 1e-3),
-                  "roofline": roofline(nbytes, attn_flops(w), f_med, peaks)},
-        "step_fused_ms": launch_stats(ms_fs), "step_two_call_ms": launch_stats(ms_ts),
-        "step_bytes_fused": 2 * nbytes, "step_bytes_two_call": 2 * (attn_bytes(w) + adaln_bytes(w)),
-        "step_windows_per_s_fused": 2 * windows / (statistics.median(ms_fs) * 1e-3),
-        "step_windows_per_s_two_call": 2 * windows / (statistics.median(ms_ts) * 1e-3)}
-    del qkv, films, res, o, x, ws
-
-    # six-block stage-1 stack at B = 4: fresh Q/K/V per block, fp32 residual chained
-    w = WORKLOADS["stack_b4"]
-    C, tokens, windows = geometry(w)
-    qkv = [device_qkv(torch, w, dev, 1000 + 10 * b) for b in range(STACK_BLOCKS)]
-    films = [device_film(torch, w, dev, 1100 + 10 * b, 1.0)[:2] for b in range(STACK_BLOCKS)]
-    res = device_film(torch, w, dev, 1190, 1.0)[2]
-    o = torch.empty_like(qkv[0][0])
-    x = o.view(w["B"], tokens // w["B"], C)
-
-    def stack():
-        for b in range(STACK_BLOCKS):
-            q, k, v = qkv[b]
-            s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTS[b % 2])
-            s3w.adaln_residual_fwd(x, res, films[b][0], films[b][1], res, eps=1e-5)
-
-    ws = torch.empty(s3w.window_attn_adaln_workspace_bytes(w["B"], w["T"], w["H"], w["W"], w["heads"], w["hd"],
-                                                           WINDOW), dtype=torch.uint8, device=dev)
-
-    def stack_fused():
-        for b in range(STACK_BLOCKS):
+        def fused_call(b):
             q, k, v = qkv[b]
             s3w.swin3d_window_attn_adaln_fwd(q, k, v, res, films[b][0], films[b][1], res, w["heads"], w["hd"], WINDOW,
-                                             SHIFTS[b % 2], workspace=ws, eps=1e-5)
+                                             SHIFTS[b], workspace=ws, eps=1e-5)
 
-    stack_reps = max(3, reps // 4)
-    ms_s = timed(torch, stream, stack, stack_reps, warmup=2)
-    ms_sf = timed(torch, stream, stack_fused, stack_reps, warmup=2)
-    launches += 3 * STACK_BLOCKS * stack_reps
-    s_med = statistics.median(ms_s)
-    nbytes = STACK_BLOCKS * (attn_bytes(w) + adaln_bytes(w))
-    flops = STACK_BLOCKS * attn_flops(w)
-    out["stack_b4"] = {
-        "grid": "B=4 T4xH180xW360, 8 heads x 64, 6 x (attn alternating shift + AdaLN fp32 out), 7200 windows per call",
-        "ms_per_stack": launch_stats(ms_s), "bytes": nbytes, "flops": flops,
-        "floor_ms_at_measured_hbm": nbytes / (peaks["hbm_gbs"] * 1e9) * 1e3,
-        "windows_per_s": STACK_BLOCKS * windows / (s_med * 1e-3),
-        "roofline": roofline(nbytes, flops, s_med, peaks),
-        "fused": {"ms_per_stack": launch_stats(ms_sf), "bytes": STACK_BLOCKS * fused_bytes(w),
-                  "windows_per_s": STACK_BLOCKS * windows / (statistics.median(ms_sf) * 1e-3),
-                  "roofline": roofline(STACK_BLOCKS * fused_bytes(w), flops, statistics.median(ms_sf), peaks)}}
-    del qkv, films, res, o, x, ws
-    torch.cuda.empty_cache()
+        def two_call_block(b):
+            q, k, v = qkv[b]
+            s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTS[b])
+            s3w.adaln_residual_fwd(x, res, films[b][0], films[b][1], res, eps=1e-5)
+
+        ms_f = timed(torch, stream, lambda: fused_call(1), reps)
+        ms_fs = timed(torch, stream, lambda: [fused_call(b) for b in range(2)], reps)
+        ms_ts = timed(torch, stream, lambda: [two_call_block(b) for b in range(2)], reps)
+        launches += len(ms_f) + 2 * len(ms_fs) + 4 * len(ms_ts)
+        f_med = statistics.median(ms_f)
+        nbytes = fused_bytes(w)
+        out["stage1_fused"] = {
+            "grid": "B=1 T4xH180xW360, 8 heads x 64, shift (1,3,6), 1800 windows; attention + AdaLN in one kernel, "
+                    "fp32 residual in place",
+            "fused": {**launch_stats(ms_f), "bytes": nbytes, "flops": attn_flops(w), "windows_per_s": windows / (f_med * 1e-3),
+                      "roofline": roofline(nbytes, attn_flops(w), f_med, peaks)},
+            "step_fused_ms": launch_stats(ms_fs), "step_two_call_ms": launch_stats(ms_ts),
+            "step_bytes_fused": 2 * nbytes, "step_bytes_two_call": 2 * (attn_bytes(w) + adaln_bytes(w)),
+            "step_windows_per_s_fused": 2 * windows / (statistics.median(ms_fs) * 1e-3),
+            "step_windows_per_s_two_call": 2 * windows / (statistics.median(ms_ts) * 1e-3)}
+        del qkv, films, res, o, x, ws
+
+    if want("stack_b4"):
+        # six-block stage-1 stack at B = 4: fresh Q/K/V per block, fp32 residual chained
+        w = WORKLOADS["stack_b4"]
+        C, tokens, windows = geometry(w)
+        qkv = [device_qkv(torch, w, dev, 1000 + 10 * b) for b in range(STACK_BLOCKS)]
+        films = [device_film(torch, w, dev, 1100 + 10 * b, 1.0)[:2] for b in range(STACK_BLOCKS)]
+        res = device_film(torch, w, dev, 1190, 1.0)[2]
+        o = torch.empty_like(qkv[0][0])
+        x = o.view(w["B"], tokens // w["B"], C)
+
+        def stack():
+            for b in range(STACK_BLOCKS):
+                q, k, v = qkv[b]
+                s3w.swin3d_window_attn_fwd(q, k, v, o, w["heads"], w["hd"], WINDOW, SHIFTS[b % 2])
+                s3w.adaln_residual_fwd(x, res, films[b][0], films[b][1], res, eps=1e-5)
+
+        ws = torch.empty(s3w.window_attn_adaln_workspace_bytes(w["B"], w["T"], w["H"], w["W"], w["heads"], w["hd"],
+                                                               WINDOW), dtype=torch.uint8, device=dev)
+
+        def stack_fused():
+            for b in range(STACK_BLOCKS):
+                q, k, v = qkv[b]
+                s3w.swin3d_window_attn_adaln_fwd(q, k, v, res, films[b][0], films[b][1], res, w["heads"], w["hd"], WINDOW,
+                                                 SHIFTS[b % 2], workspace=ws, eps=1e-5)
+
+        stack_reps = max(3, reps // 4)
+        ms_s = timed(torch, stream, stack, stack_reps, warmup=2)
+        ms_sf = timed(torch, stream, stack_fused, stack_reps, warmup=2)
+        launches += 3 * STACK_BLOCKS * stack_reps
+        s_med = statistics.median(ms_s)
+        nbytes = STACK_BLOCKS * (attn_bytes(w) + adaln_bytes(w))
+        flops = STACK_BLOCKS * attn_flops(w)
+        out["stack_b4"] = {
+            "grid": "B=4 T4xH180xW360, 8 heads x 64, 6 x (attn alternating shift + AdaLN fp32 out), 7200 windows per call",
+            "ms_per_stack": launch_stats(ms_s), "bytes": nbytes, "flops": flops,
+            "floor_ms_at_measured_hbm": nbytes / (peaks["hbm_gbs"] * 1e9) * 1e3,
+            "windows_per_s": STACK_BLOCKS * windows / (s_med * 1e-3),
+            "roofline": roofline(nbytes, flops, s_med, peaks),
+            "fused": {"ms_per_stack": launch_stats(ms_sf), "bytes": STACK_BLOCKS * fused_bytes(w),
+                      "windows_per_s": STACK_BLOCKS * windows / (statistics.median(ms_sf) * 1e-3),
+                      "roofline": roofline(STACK_BLOCKS * fused_bytes(w), flops, statistics.median(ms_sf), peaks)}}
+        del qkv, films, res, o, x, ws
+        torch.cuda.empty_cache()
     return out, launches
+
+
+CONFIG_NAMES = ("tiny", "stage2", "stage3_padded", "stage1_tf32", "stage1_window_2x12x12", "stage1_qkv_proj",
+                "stage1_fused", "stack_b4")
+
+
+def bench_one_config(args):
+    """One workload of the set on its own (``--config NAME``): its entry of ``configs``."""
+    import torch
+
+    import swin3d_window_attention_b200 as s3w
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    s3w.load_library()
+    out, launches = bench_configs(torch, s3w, dev, torch.cuda.current_stream(dev), load_peaks(), args.config_reps,
+                                  only=args.config)
+    if s3w.poll_device_error() != 0:
+        raise SystemExit("device error word set")
+    print(json.dumps({"config": args.config, "gpu_launches": launches, **out[args.config]}), flush=True)
 
 
 def bench_cuda(args):
@@ -856,11 +891,15 @@ def main():
     ap.add_argument("--config-reps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true")
+    ap.add_argument("--config", choices=CONFIG_NAMES, default=None,
+                    help="time only this workload of the set (no headline step)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         bench_reference(args)
+    elif args.config is not None:
+        bench_one_config(args)
     else:
         bench_cuda(args)
 
