@@ -120,6 +120,17 @@ def config_for(world):
     return c
 
 
+def reduce_max_over_ranks(torch, dist, values, device):
+    """Element-wise max over the ranks of a list of floats: the slowest rank's time, and any
+    rank's error flag.  Every rank calls it at the same points, error or not, so that no rank
+    is left waiting in a collective; without a process group it returns the values."""
+    if dist is None:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 def load_peaks():
     """Measured peaks of this machine's B200s if the driver wrote them, else the fallback."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -654,14 +665,12 @@ def bench_cuda(args):
     wall1 = time.time()
     if dist:
         dist.barrier()
-    ms = t0.elapsed_time(t1)
     clk = clocks.stop((wall0, wall1))
-    if s3w.poll_device_error() != 0:
-        raise SystemExit("device error word set during the timed region")
-    if dist:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms, bad = reduce_max_over_ranks(torch, dist, [t0.elapsed_time(t1), s3w.poll_device_error() != 0], dev)
+    if bad:
+        if dist:
+            dist.destroy_process_group()
+        raise SystemExit("device error word set during the timed region (on at least one rank)")
     attn_ms = [a.elapsed_time(b) for a, b in attn_ev]
     adaln_ms = [a.elapsed_time(b) for a, b in adaln_ev]
     attn = launch_stats(attn_ms)
@@ -695,11 +704,7 @@ def bench_cuda(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
-    if dist:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms, = reduce_max_over_ranks(torch, dist, [e0.elapsed_time(e1) / args.steps], dev)
     del pinned, res_out
 
     configs, extra_launches = None, 0
