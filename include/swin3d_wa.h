@@ -199,7 +199,10 @@ long long swin3d_window_attn_adaln_workspace_bytes(int B, int T, int H, int W, i
  *
  * The workspace is a file-scope device array of S3W_ADALN_STATIC_WORKSPACE_BYTES bytes in
  * the library (one per device, its address looked up once per device on first use).  The
- * call allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ * array lives in a device-code module of its own, holding no kernels, so under CUDA's lazy
+ * module loading (the default) it occupies device memory only on devices where this call
+ * has run; with eager loading, on every device the process uses.  The call allocates nothing:
+ * no cudaMalloc, no cudaFree, no allocating library routine.
  * Nothing in the array has to start at zero and the call clears nothing: every workspace
  * byte the kernel reads was written earlier in the same launch.
  *
