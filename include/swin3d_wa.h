@@ -59,7 +59,7 @@ typedef enum {
   S3W_OK = 0,
   S3W_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, shift >= window, ...     */
   S3W_ERR_UNSUPPORTED = 2,   /* valid but not built: head_dim, window size, dtype combo   */
-  S3W_ERR_MISALIGNED = 3,    /* pointer or stride not 16-byte aligned                     */
+  S3W_ERR_MISALIGNED = 3,    /* pointer or stride not aligned as the call requires        */
   S3W_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed                      */
   S3W_ERR_DEVICE_TIMEOUT = 5 /* a bounded wait inside a kernel expired                    */
 } s3w_status;
@@ -161,9 +161,11 @@ int adaln_residual_fwd(const void* x, int x_dtype, const float* residual,
  * residual     device fp32 [B][T*H*W][C], C = heads * head_dim (C <= 4096), 32-byte aligned.
  * adaln_scale, adaln_shift  device fp32 [B][C], 32-byte aligned.
  * out          device, out_dtype (S3W_F32 or S3W_BF16), [B][T*H*W][C], 32-byte aligned; may
- *              alias residual exactly (in-place update of the residual stream).
+ *              alias residual exactly (in-place update of the residual stream); must not
+ *              overlap q, k or v.
  * o            optional device bf16 [B][T][H][W][C] (token stride C), 32-byte aligned: when
- *              non-NULL the attention output is written there too; NULL skips it.
+ *              non-NULL the attention output is written there too; NULL skips it.  Must not
+ *              overlap q, k or v.
  * workspace    device memory of at least swin3d_window_attn_adaln_workspace_bytes(...) bytes
  *              for the current device, 32-byte aligned, owned by the caller; its contents on
  *              entry do not matter.  Calls that overlap on the GPU must not share it.

@@ -63,7 +63,7 @@ const char* s3w_status_string(int status) {
     case S3W_OK: return "ok";
     case S3W_ERR_INVALID_ARG: return "invalid argument";
     case S3W_ERR_UNSUPPORTED: return "unsupported configuration";
-    case S3W_ERR_MISALIGNED: return "pointer or stride not 16-byte aligned";
+    case S3W_ERR_MISALIGNED: return "pointer or stride not aligned as the call requires";
     case S3W_ERR_CUDA: return "CUDA runtime error";
     case S3W_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel expired";
     default: return "unknown status";
@@ -90,6 +90,20 @@ int s3w_poll_device_error(s3w_stream_t stream) {
 }  // extern "C"
 
 namespace {
+
+// True when the byte range [p, p + bytes) meets any of the q, k, v token ranges (tokens rows of
+// row_bytes at a stride of stride_bytes).  The callers bound every size below 2^62.
+bool overlaps_qkv(const void* q, const void* k, const void* v, long long stride_bytes, long long row_bytes,
+                  long long tokens, const void* p, long long bytes) {
+  const char* p0 = static_cast<const char*>(p);
+  const char* p1 = p0 + bytes;
+  for (const void* t : {q, k, v}) {
+    const char* t0 = static_cast<const char*>(t);
+    const char* t1 = t0 + (tokens - 1) * stride_bytes + row_bytes;
+    if (p0 < t1 && t0 < p1) return true;
+  }
+  return false;
+}
 
 // Host-side checks shared by both attention entry points; fills the kernel geometry.
 int make_geometry(const void* q, const void* k, const void* v, void* o, int B, int T, int H, int W, int win_t,
@@ -127,6 +141,15 @@ int make_geometry(const void* q, const void* k, const void* v, void* o, int B, i
   if (per_sample * B * heads > INT32_MAX) return S3W_ERR_UNSUPPORTED;  // tile index is 32-bit
   // streaming path: units = tiles x blocks (at most win_t x win_h blocks per window)
   if (N > 144 && per_sample * B * heads * win_t * win_h > INT32_MAX) return S3W_ERR_UNSUPPORTED;
+  // o must not overlap q, k or v (which may overlap one another: slices of one buffer).  The
+  // sizes are bounded above (tokens < 2^31, strides checked against C), so no product overflows
+  // once the strides are below 2^31.
+  if (qkv_token_stride > INT32_MAX || o_token_stride > INT32_MAX) return S3W_ERR_UNSUPPORTED;
+  {
+    const long long tokens = static_cast<long long>(B) * T * H * W;
+    if (overlaps_qkv(q, k, v, qkv_token_stride * ib, C * ib, tokens, o, ((tokens - 1) * o_token_stride + C) * ob))
+      return S3W_ERR_INVALID_ARG;
+  }
 
   s3w::WinGeom& g = *out;
   g = s3w::WinGeom{};
@@ -243,6 +266,8 @@ int swin3d_window_attn_adaln_fwd(const void* q, const void* k, const void* v, lo
   const char* o0 = reinterpret_cast<const char*>(out);
   const long long ob = out_dtype == S3W_F32 ? 4 : 2;
   if (o0 != r0 && o0 < r0 + n * 4 && r0 < o0 + n * ob) return S3W_ERR_INVALID_ARG;
+  // out is written while other windows still read q, k and v
+  if (overlaps_qkv(q, k, v, qkv_token_stride * 2, C * 2, n / C, out, n * ob)) return S3W_ERR_INVALID_ARG;
   DeviceState* ds = nullptr;
   rc = device_state(&ds);
   if (rc != S3W_OK) return rc;

@@ -11,6 +11,7 @@ from swin3d_window_attention_b200 import api
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 FAKE = 0x10000  # 16-byte aligned dummy address; only used with arguments that are rejected first
+FAKE_QKV = 0x40000000   # a second dummy region, far from FAKE
 
 
 def declared_functions():
@@ -69,6 +70,12 @@ def _attn(**over):
     (dict(q=FAKE + 8), api.S3W_ERR_MISALIGNED),
     (dict(o=FAKE + 2), api.S3W_ERR_MISALIGNED),
     (dict(qs=516), api.S3W_ERR_MISALIGNED),         # token rows not on 16-byte boundaries
+    # o overlapping q, k, v (1,152 tokens x 512 channels x 2 bytes = 1,179,648 bytes each)
+    (dict(), api.S3W_ERR_INVALID_ARG),                                  # o == q == k == v
+    (dict(o=FAKE + 1179648 - 1024), api.S3W_ERR_INVALID_ARG),           # o starts inside the last row
+    (dict(o=FAKE - 1024), api.S3W_ERR_INVALID_ARG),                     # o ends inside the first rows
+    (dict(q=FAKE_QKV, k=FAKE_QKV + 1024, v=FAKE_QKV + 2048, qs=1536, o=FAKE_QKV + 1536 * 2 * 1151 + 2048),
+     api.S3W_ERR_INVALID_ARG),                                          # o on the last token row of v
 ])
 def test_attn_rejects_bad_arguments_on_host(over, expect):
     assert _attn(**over) == expect
@@ -76,8 +83,8 @@ def test_attn_rejects_bad_arguments_on_host(over, expect):
 
 def test_legacy_baseline_is_bf16_only():
     lib = s3w.load_library()
-    rc = lib.swin3d_window_attn_fwd_legacy_mma(FAKE, FAKE, FAKE, FAKE, 1, 4, 12, 24, 2, 6, 12, 1, 3, 6, 8, 64, 512,
-                                               512, 0.0, api.S3W_F32, 0, None)
+    rc = lib.swin3d_window_attn_fwd_legacy_mma(FAKE, FAKE, FAKE, FAKE_QKV, 1, 4, 12, 24, 2, 6, 12, 1, 3, 6, 8, 64,
+                                               512, 512, 0.0, api.S3W_F32, 0, None)
     assert rc == api.S3W_ERR_UNSUPPORTED
 
 
@@ -115,8 +122,10 @@ def test_adaln_zero_tokens_is_a_no_op():
 
 
 def _fused(**over):
-    a = dict(q=FAKE, k=FAKE, v=FAKE, qs=512, res=FAKE, sc=FAKE, sh=FAKE, out=FAKE, outd=1, o=None, ws=FAKE,
-             wsb=1 << 30, B=1, T=4, H=12, W=24, wt=2, wh=6, ww=12, st=1, sh_=3, sw=6, heads=8, hd=64, scale=0.0,
+    # every default is valid except the workspace size, which is checked last (a call with these
+    # defaults returns on the host on every machine)
+    a = dict(q=FAKE_QKV, k=FAKE_QKV, v=FAKE_QKV, qs=512, res=FAKE, sc=FAKE, sh=FAKE, out=FAKE, outd=1, o=None,
+             ws=FAKE, wsb=0, B=1, T=4, H=12, W=24, wt=2, wh=6, ww=12, st=1, sh_=3, sw=6, heads=8, hd=64, scale=0.0,
              eps=1e-5)
     a.update(over)
     return s3w.load_library().swin3d_window_attn_adaln_fwd(
@@ -140,6 +149,8 @@ def _fused(**over):
     (dict(sc=FAKE + 16), api.S3W_ERR_MISALIGNED),           # FiLM scale not 32-byte aligned
     (dict(sh=FAKE + 48), api.S3W_ERR_MISALIGNED),           # FiLM shift not 32-byte aligned
     (dict(out=FAKE + 16 * 512), api.S3W_ERR_INVALID_ARG),   # partial overlap of out with residual
+    (dict(out=FAKE_QKV + 4096, res=FAKE_QKV + 4096), api.S3W_ERR_INVALID_ARG),   # out over q, k, v
+    (dict(o=FAKE_QKV + 1024), api.S3W_ERR_INVALID_ARG),     # attention output over q, k, v
 ])
 def test_fused_rejects_bad_arguments_on_host(over, expect):
     if "out" in over and "res" not in over:
