@@ -127,7 +127,8 @@ int swin3d_window_attn_fwd(const void* q, const void* k, const void* v, void* o,
  * residual  device fp32 [B][L][C], 16-byte aligned.  out may alias residual exactly
  *           (in-place update of the residual stream); no other overlap is allowed.
  * scale, shift  device fp32 [B][C] per-sample FiLM vectors, 16-byte aligned.
- * out       device, out_dtype, [B][L][C], 16-byte aligned.
+ * out       device, out_dtype, [B][L][C], 16-byte aligned; must not overlap x, scale or
+ *           shift (S3W_ERR_INVALID_ARG).
  * B >= 1, tokens_per_sample >= 0, C a multiple of 8 with 8 <= C <= 4096; eps >= 0.
  * With tokens_per_sample == 0 nothing is launched and the pointers are not used (they
  * may be NULL).  B * tokens_per_sample above (2^31 - 1) * 8 returns S3W_ERR_UNSUPPORTED.

@@ -357,6 +357,14 @@ int adaln_residual_fwd(const void* x, int x_dtype, const float* residual, const 
   const char* o0 = reinterpret_cast<const char*>(out);
   const long long ob = out_dtype == S3W_F32 ? 4 : 2;
   if (o0 != r0 && o0 < r0 + n * 4 && r0 < o0 + n * ob) return S3W_ERR_INVALID_ARG;
+  // and out overlaps none of x, scale, shift
+  auto meets_out = [&](const void* p, long long bytes) {
+    const char* a = static_cast<const char*>(p);
+    return a < o0 + n * ob && o0 < a + bytes;
+  };
+  if (meets_out(x, n * (x_dtype == S3W_F32 ? 4 : 2)) || meets_out(scale, B * 4ll * C) ||
+      meets_out(shift, B * 4ll * C))
+    return S3W_ERR_INVALID_ARG;
   DeviceState* ds = nullptr;
   int rc = device_state(&ds);
   if (rc != S3W_OK) return rc;

@@ -106,12 +106,16 @@ def _adaln(**over):
     (dict(C=8192), api.S3W_ERR_UNSUPPORTED),
     (dict(sc=FAKE + 4), api.S3W_ERR_MISALIGNED),
     (dict(out=FAKE + 16 * 512), api.S3W_ERR_INVALID_ARG),   # partial overlap with residual
+    (dict(x=FAKE_QKV, sc=FAKE_QKV, sh=FAKE_QKV, res=FAKE_QKV + 8192, out=FAKE_QKV + 8192),
+     api.S3W_ERR_INVALID_ARG),                               # out in place on residual, but over x
+    (dict(x=FAKE_QKV, sc=FAKE + 4096, sh=FAKE_QKV + 65536, res=FAKE, out=FAKE, xd=1, L=4),
+     api.S3W_ERR_INVALID_ARG),                               # out over scale (x, shift elsewhere)
     (dict(L=(2 ** 31 - 1) * 8 + 1), api.S3W_ERR_UNSUPPORTED),   # more row blocks than a grid holds
     (dict(B=4, L=2 ** 62), api.S3W_ERR_UNSUPPORTED),             # B * L * C would overflow int64
 ])
 def test_adaln_rejects_bad_arguments_on_host(over, expect):
     # the overlap case keeps out != residual while the two ranges intersect
-    if "out" in over:
+    if "out" in over and "res" not in over:
         over = dict(over, res=FAKE + 64)
     assert _adaln(**over) == expect
 
