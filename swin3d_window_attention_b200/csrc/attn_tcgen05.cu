@@ -628,6 +628,31 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         }
         return true;
       }
+      if constexpr (HD == 64 && !OUT_F32) {
+        if (g.o_rows_32b && !is_tail) {
+          // The thread holds two 32-byte pieces of its row, 64 bytes apart in the same 128-byte
+          // line (columns 16 half .. +15 and 32 + 16 half .. +15).  Lanes 2i and 2i+1 swap one
+          // piece each, so that every store instruction writes both pieces of one row per lane
+          // pair: 16 lines per warp instruction instead of 32 (the store path's cost is per line).
+          uint32_t u0[8], u1[8], x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            u0[e] = pack_bf16x2(ov[2 * e] * inv, ov[2 * e + 1] * inv);
+            u1[e] = pack_bf16x2(ov[16 + 2 * e] * inv, ov[16 + 2 * e + 1] * inv);
+          }
+          const bool odd = lane & 1;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = __shfl_xor_sync(0xffffffffu, odd ? u0[e] : u1[e], 1);
+          const int ptok = __shfl_xor_sync(0xffffffffu, tok, 1);
+          // first store: the even lane's row (even lane: piece 0, odd lane: piece 1); second:
+          // the odd lane's row
+          const int t1 = odd ? ptok : tok, t2 = odd ? tok : ptok;
+          __nv_bfloat16* base = static_cast<__nv_bfloat16*>(o) + head * HD + (odd ? 32 : 0) + 16 * half;
+          if (t1 >= 0) st_global_v8(base + static_cast<long long>(t1) * g.o_stride, odd ? x : u0);
+          if (t2 >= 0) st_global_v8(base + static_cast<long long>(t2) * g.o_stride, odd ? u1 : x);
+          return true;
+        }
+      }
       if (tok >= 0) {
 #pragma unroll
         for (int m = 0; m < HD / 32; ++m) {
