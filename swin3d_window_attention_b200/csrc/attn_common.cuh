@@ -356,5 +356,82 @@ __device__ __forceinline__ void table_writer(const WinGeom& g, Table* tables, co
   }
 }
 
+// Epilogue store of the softmax threads: a thread holds HD / 2 outputs of one query row, the
+// column groups 32 m + 16 half .. +15 (m < HD / 32), in v[16 m + j], scaled here by inv and
+// written to token `tok` (-1: a padded slot, nothing written) of grid tensor o.  Every lane of
+// the warp calls it; the lanes of a pair (2i, 2i+1) hold rows of the same key half.
+//  * bf16, HD = 64, 32-byte rows: the thread's two 32-byte pieces sit 64 bytes apart in one
+//    128-byte line.  The lanes of a pair swap one piece each, so the first store instruction
+//    writes both pieces of the even lane's row and the second those of the odd lane's row: 16
+//    lines per warp instruction instead of 32 (the store path's cost is per line).
+//  * otherwise, 32-byte rows: one 32-byte store per 16 bf16 or 8 fp32 values.
+//  * rows not 32-byte aligned: 16-byte stores.
+template <int HD, bool OUT_F32>
+__device__ __forceinline__ void store_o_row(void* o, long long o_stride, bool rows_32b, int tok, int head, int half,
+                                            int lane, const float* v, float inv) {
+  constexpr int kGroups = HD / 32 > 0 ? HD / 32 : 1;
+  constexpr int kPer = HD >= 32 ? 16 : HD / 2;   // values per column group
+  if constexpr (!OUT_F32 && HD == 64) {
+    if (rows_32b) {
+      uint32_t u0[8], u1[8], x[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        u0[e] = pack_bf16x2(v[2 * e] * inv, v[2 * e + 1] * inv);
+        u1[e] = pack_bf16x2(v[16 + 2 * e] * inv, v[16 + 2 * e + 1] * inv);
+      }
+      const bool odd = lane & 1;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = __shfl_xor_sync(0xffffffffu, odd ? u0[e] : u1[e], 1);
+      const int ptok = __shfl_xor_sync(0xffffffffu, tok, 1);
+      const int t1 = odd ? ptok : tok, t2 = odd ? tok : ptok;
+      __nv_bfloat16* base = static_cast<__nv_bfloat16*>(o) + head * HD + (odd ? 32 : 0) + 16 * half;
+      if (t1 >= 0) sm100::st_global_v8(base + static_cast<long long>(t1) * o_stride, odd ? x : u0);
+      if (t2 >= 0) sm100::st_global_v8(base + static_cast<long long>(t2) * o_stride, odd ? u1 : x);
+      return;
+    }
+  }
+  if (tok < 0) return;
+#pragma unroll
+  for (int m = 0; m < kGroups; ++m) {
+    const int col = 32 * m + 16 * half;
+    const float* w = v + 16 * m;
+    if constexpr (OUT_F32) {
+      float* dst = static_cast<float*>(o) + static_cast<long long>(tok) * o_stride + head * HD + col;
+#pragma unroll
+      for (int q = 0; q < kPer; q += 8) {
+        if (rows_32b && kPer % 8 == 0) {
+          uint32_t u[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) u[e] = __float_as_uint(w[q + e] * inv);
+          sm100::st_global_v8(dst + q, u);
+        } else {
+#pragma unroll
+          for (int r = 0; r < 8 && q + r < kPer; r += 4)
+            *reinterpret_cast<float4*>(dst + q + r) =
+                make_float4(w[q + r] * inv, w[q + r + 1] * inv, w[q + r + 2] * inv, w[q + r + 3] * inv);
+        }
+      }
+    } else {
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tok) * o_stride + head * HD + col;
+      if (rows_32b && kPer == 16) {
+        uint32_t u[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) u[e] = pack_bf16x2(w[2 * e] * inv, w[2 * e + 1] * inv);
+        sm100::st_global_v8(dst, u);
+      } else {
+#pragma unroll
+        for (int q = 0; q < kPer; q += 8) {
+          uint4 u;
+          u.x = pack_bf16x2(w[q] * inv, w[q + 1] * inv);
+          u.y = pack_bf16x2(w[q + 2] * inv, w[q + 3] * inv);
+          u.z = pack_bf16x2(w[q + 4] * inv, w[q + 5] * inv);
+          u.w = pack_bf16x2(w[q + 6] * inv, w[q + 7] * inv);
+          *reinterpret_cast<uint4*>(dst + q) = u;
+        }
+      }
+    }
+  }
+}
+
 }  // namespace attn
 }  // namespace s3w

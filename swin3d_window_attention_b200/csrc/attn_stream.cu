@@ -622,33 +622,8 @@ window_attn_stream_kernel(const __grid_constant__ WinGeom g, const __grid_consta
         aborted = true;
         break;
       }
-      if (tok >= 0) {
-        const float inv = l > 0.f ? 1.0f / l : 0.f;
-#pragma unroll
-        for (int mm = 0; mm < HD / 32; ++mm) {
-          const int col = 32 * mm + 16 * half;
-          if constexpr (OUT_F32) {
-            float* dst = static_cast<float*>(o) + static_cast<long long>(tok) * g.o_stride + tc.head * HD + col;
-#pragma unroll
-            for (int q4 = 0; q4 < 16; q4 += 4)
-              *reinterpret_cast<float4*>(dst + q4) =
-                  make_float4(acc[16 * mm + q4] * inv, acc[16 * mm + q4 + 1] * inv, acc[16 * mm + q4 + 2] * inv,
-                              acc[16 * mm + q4 + 3] * inv);
-          } else {
-            __nv_bfloat16* dst =
-                static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tok) * g.o_stride + tc.head * HD + col;
-#pragma unroll
-            for (int q8 = 0; q8 < 16; q8 += 8) {
-              uint4 w4;
-              w4.x = pack_bf16x2(acc[16 * mm + q8] * inv, acc[16 * mm + q8 + 1] * inv);
-              w4.y = pack_bf16x2(acc[16 * mm + q8 + 2] * inv, acc[16 * mm + q8 + 3] * inv);
-              w4.z = pack_bf16x2(acc[16 * mm + q8 + 4] * inv, acc[16 * mm + q8 + 5] * inv);
-              w4.w = pack_bf16x2(acc[16 * mm + q8 + 6] * inv, acc[16 * mm + q8 + 7] * inv);
-              *reinterpret_cast<uint4*>(dst + q8) = w4;
-            }
-          }
-        }
-      }
+      const float inv = l > 0.f ? 1.0f / l : 0.f;
+      store_o_row<HD, OUT_F32>(o, g.o_stride, g.o_rows_32b != 0, tok, tc.head, half, lane, acc, inv);
     }
     if (aborted) {
       if (lane == 0) record_error(err, kStatusTimeout);

@@ -562,30 +562,6 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
     int prev_it = 0, prev_head = 0, prev_tok = -1;
     bool aborted = false;
 
-    auto store8 = [&](int tk, int head, int col, const float* vals, float scl) {
-      // 8 consecutive outputs of one row starting at column `col`.
-      if constexpr (OUT_F32) {
-        float* dst = static_cast<float*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD + col;
-        if (g.o_rows_32b) {
-          uint32_t u[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) u[e] = __float_as_uint(vals[e] * scl);
-          st_global_v8(dst, u);
-        } else {
-          *reinterpret_cast<float4*>(dst) = make_float4(vals[0] * scl, vals[1] * scl, vals[2] * scl, vals[3] * scl);
-          *reinterpret_cast<float4*>(dst + 4) = make_float4(vals[4] * scl, vals[5] * scl, vals[6] * scl, vals[7] * scl);
-        }
-      } else {
-        __nv_bfloat16* dst =
-            static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tk) * g.o_stride + head * HD + col;
-        uint4 u;
-        u.x = pack_bf16x2(vals[0] * scl, vals[1] * scl);
-        u.y = pack_bf16x2(vals[2] * scl, vals[3] * scl);
-        u.z = pack_bf16x2(vals[4] * scl, vals[5] * scl);
-        u.w = pack_bf16x2(vals[6] * scl, vals[7] * scl);
-        *reinterpret_cast<uint4*>(dst) = u;
-      }
-    };
 
     // Epilogue of a finished tile: this thread's O columns and the row sum (column 64 of O)
     // from TMEM, scaled by 1/rowsum, stored to the grid position of the query slot
@@ -628,48 +604,7 @@ window_attn_tc_kernel(const __grid_constant__ WinGeom g, const __grid_constant__
         }
         return true;
       }
-      if constexpr (HD == 64 && !OUT_F32) {
-        if (g.o_rows_32b && !is_tail) {
-          // The thread holds two 32-byte pieces of its row, 64 bytes apart in the same 128-byte
-          // line (columns 16 half .. +15 and 32 + 16 half .. +15).  Lanes 2i and 2i+1 swap one
-          // piece each, so that every store instruction writes both pieces of one row per lane
-          // pair: 16 lines per warp instruction instead of 32 (the store path's cost is per line).
-          uint32_t u0[8], u1[8], x[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            u0[e] = pack_bf16x2(ov[2 * e] * inv, ov[2 * e + 1] * inv);
-            u1[e] = pack_bf16x2(ov[16 + 2 * e] * inv, ov[16 + 2 * e + 1] * inv);
-          }
-          const bool odd = lane & 1;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = __shfl_xor_sync(0xffffffffu, odd ? u0[e] : u1[e], 1);
-          const int ptok = __shfl_xor_sync(0xffffffffu, tok, 1);
-          // first store: the even lane's row (even lane: piece 0, odd lane: piece 1); second:
-          // the odd lane's row
-          const int t1 = odd ? ptok : tok, t2 = odd ? tok : ptok;
-          __nv_bfloat16* base = static_cast<__nv_bfloat16*>(o) + head * HD + (odd ? 32 : 0) + 16 * half;
-          if (t1 >= 0) st_global_v8(base + static_cast<long long>(t1) * g.o_stride, odd ? x : u0);
-          if (t2 >= 0) st_global_v8(base + static_cast<long long>(t2) * g.o_stride, odd ? u1 : x);
-          return true;
-        }
-      }
-      if (tok >= 0) {
-#pragma unroll
-        for (int m = 0; m < HD / 32; ++m) {
-          const int col = 32 * m + 16 * half;
-          if constexpr (!OUT_F32) {
-            if (g.o_rows_32b) {   // 16 bf16 = one 32-byte store
-              uint32_t u[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) u[e] = pack_bf16x2(ov[16 * m + 2 * e] * inv, ov[16 * m + 2 * e + 1] * inv);
-              st_global_v8(static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tok) * g.o_stride + head * HD + col, u);
-              continue;
-            }
-          }
-          store8(tok, head, col, ov + 16 * m, inv);
-          store8(tok, head, col + 8, ov + 16 * m + 8, inv);
-        }
-      }
+      store_o_row<HD, OUT_F32>(o, g.o_stride, g.o_rows_32b != 0, tok, head, half, lane, ov, inv);
       return true;
     };
 

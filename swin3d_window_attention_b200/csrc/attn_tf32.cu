@@ -334,31 +334,7 @@ window_attn_tf32_kernel(const __grid_constant__ WinGeom g, const __grid_constant
       tc_fence_before();
       mbar_arrive(o_empty);
       const float inv = l > 0.f ? 1.0f / l : 0.f;
-      if (tok >= 0) {
-#pragma unroll
-        for (int m = 0; m < (HD + 31) / 32; ++m) {
-          const int col = 32 * m + 16 * half;
-          if constexpr (OUT_F32) {
-            float* dst = static_cast<float*>(o) + static_cast<long long>(tok) * g.o_stride + head * HD + col;
-#pragma unroll
-            for (int q = 0; q < 16; q += 4)
-              *reinterpret_cast<float4*>(dst + q) = make_float4(ov[16 * m + q] * inv, ov[16 * m + q + 1] * inv,
-                                                                ov[16 * m + q + 2] * inv, ov[16 * m + q + 3] * inv);
-          } else {
-            __nv_bfloat16* dst =
-                static_cast<__nv_bfloat16*>(o) + static_cast<long long>(tok) * g.o_stride + head * HD + col;
-#pragma unroll
-            for (int q = 0; q < 16; q += 8) {
-              uint4 u;
-              u.x = pack_bf16x2(ov[16 * m + q] * inv, ov[16 * m + q + 1] * inv);
-              u.y = pack_bf16x2(ov[16 * m + q + 2] * inv, ov[16 * m + q + 3] * inv);
-              u.z = pack_bf16x2(ov[16 * m + q + 4] * inv, ov[16 * m + q + 5] * inv);
-              u.w = pack_bf16x2(ov[16 * m + q + 6] * inv, ov[16 * m + q + 7] * inv);
-              *reinterpret_cast<uint4*>(dst + q) = u;
-            }
-          }
-        }
-      }
+      store_o_row<HD, OUT_F32>(o, g.o_stride, g.o_rows_32b != 0, tok, head, half, lane, ov, inv);
       return true;
     };
 
