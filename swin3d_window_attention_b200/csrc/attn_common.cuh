@@ -74,8 +74,30 @@ __device__ __forceinline__ void build_mask(const Table& tb, const SlotConst& sc,
 // Per-CTA slot constants, written by threads 0..143, 160..174 and 192..196.
 __device__ __forceinline__ void init_slot_consts(const WinGeom& g, SlotConst* slotc, int tid) {
   auto split_at = [&](int a) { return a == 0 ? g.wt - g.st : (a == 1 ? g.wh - g.sh : g.ww - g.sw); };
-  auto slot_off = [&](int r, int a) {   // offset of slot r along axis a
-    return a == 2 ? r % g.ww : (a == 1 ? (r / g.ww) % g.wh : r / (g.ww * g.wh));
+  // offset of slot r along axis a.  Slots run T-slab by T-slab; inside a slab, h-major rows of
+  // w, except that with a W shift each slab holds first the rows of the w offsets before the
+  // wrap-around split (win_w - shift_w of them), then the rows of the rest.  The split is where
+  // a window cut by the W seam wraps, so every slab loads in whole boxes (see the loader).
+  auto slot_off = [&](int r, int a) {
+    const int per_slab = g.ww * g.wh;
+    const int rt = r / per_slab, i = r - rt * per_slab;
+    if (a == 0) return rt;
+    int rh, rw;
+    if (g.sw > 0) {
+      const int n1 = g.ww - g.sw;
+      if (i < g.wh * n1) {
+        rh = i / n1;
+        rw = i - rh * n1;
+      } else {
+        const int j = i - g.wh * n1;
+        rh = j / g.sw;
+        rw = n1 + (j - rh * g.sw);
+      }
+    } else {
+      rh = i / g.ww;
+      rw = i - rh * g.ww;
+    }
+    return a == 1 ? rh : rw;
   };
   if (tid < kN) slotc->coord[tid] = tid < g.N ? (slot_off(tid, 0) | slot_off(tid, 1) << 8 | slot_off(tid, 2) << 16) : 0u;
   if (tid >= 160 && tid < 160 + 3 * kMaskWords) {
@@ -120,14 +142,26 @@ __device__ __forceinline__ TileCoord tile_coord(const WinGeom& g, long long tile
 }
 
 // Tensor maps of Q, K and V over the grid as a 5-D tensor (channel, W, H, T, sample),
-// one per box shape.  A window is loaded one T-slab (win_h x win_w tokens) at a time:
-// a whole slab in one box where the window does not wrap around a seam; a slab cut at
-// the H seam in two boxes (win_h - shift_h rows, then shift_h rows); and where the window
-// wraps around the W seam, one box per (t, h) run cut in two (win_w - shift_w, then
-// shift_w tokens), since a box narrower than the window would pack its rows too densely.
+// one per box shape.  A window is loaded one T-slab (win_h x win_w tokens) at a time.
+// Without a W shift: the whole slab in one box, or, where the window wraps around the H
+// seam, in two (win_h - shift_h rows, then shift_h rows).  With a W shift the slab's slots
+// hold part A (the first n1 = win_w - shift_w offsets of every row) and then part B (the
+// other shift_w), each h-major; A and B are one box each (two each at the H seam).  The
+// W seam of a window always falls between A and B, so no window needs more boxes.
 // Every box is one 128-byte channel chunk wide (64 bf16 or 32 fp32 channels), 128-byte
 // swizzle, out-of-bounds elements (padding) read as zero.
-enum : int { kBoxSlab = 0, kBoxSeamH1 = 1, kBoxSeamH2 = 2, kBoxSeamW1 = 3, kBoxSeamW2 = 4, kBoxShapes = 5 };
+enum : int {
+  kBoxSlab = 0,     // win_w x win_h
+  kBoxSeamH1 = 1,   // win_w x (win_h - shift_h)
+  kBoxSeamH2 = 2,   // win_w x shift_h
+  kBoxA = 3,        // n1 x win_h
+  kBoxB = 4,        // shift_w x win_h
+  kBoxA1 = 5,       // n1 x (win_h - shift_h)
+  kBoxA2 = 6,       // n1 x shift_h
+  kBoxB1 = 7,       // shift_w x (win_h - shift_h)
+  kBoxB2 = 8,       // shift_w x shift_h
+  kBoxShapes = 9
+};
 struct TmaMaps {
   CUtensorMap m[3][kBoxShapes];   // [tensor q/k/v][box shape]
 };
@@ -158,15 +192,13 @@ inline cudaError_t make_maps(const WinGeom& g, const void* const ptrs[3], bool f
                               static_cast<cuuint64_t>(g.T), static_cast<cuuint64_t>(g.B)};
   const cuuint64_t row = static_cast<cuuint64_t>(g.qkv_stride) * es;
   const cuuint64_t strides[4] = {row, row * g.W, row * g.W * g.H, row * g.W * g.H * g.T};
-  // box (W, H) extents per shape; a seam shape of an unshifted axis is never used and
-  // gets the whole window instead
+  // box (W, H) extents per shape; a shape of an unshifted axis is never used and gets the
+  // whole window's extent instead
   const cuuint32_t ww = static_cast<cuuint32_t>(g.ww), wh = static_cast<cuuint32_t>(g.wh);
   const cuuint32_t sw = static_cast<cuuint32_t>(g.sw), sh = static_cast<cuuint32_t>(g.sh);
-  const cuuint32_t boxwh[kBoxShapes][2] = {{ww, wh},
-                                           {ww, wh - sh},
-                                           {ww, sh > 0 ? sh : wh},
-                                           {ww - sw, 1},
-                                           {sw > 0 ? sw : ww, 1}};
+  const cuuint32_t n1 = ww - sw, n2 = sw > 0 ? sw : ww, h1 = wh - sh, h2 = sh > 0 ? sh : wh;
+  const cuuint32_t boxwh[kBoxShapes][2] = {{ww, wh}, {ww, h1}, {ww, h2}, {n1, wh}, {n2, wh},
+                                           {n1, h1}, {n1, h2}, {n2, h1}, {n2, h2}};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   const cuuint32_t box_c = static_cast<cuuint32_t>(kRowBytes / es);
   for (int t = 0; t < 3; ++t)
@@ -240,47 +272,45 @@ __device__ __forceinline__ void tma_loader(const WinGeom& g, const TmaMaps& maps
     mbar_arrive_expect_tx(bar, tile_bytes);
     // The window's first slot sits at (bt, bh, bw), inside the padded grid on every
     // axis; a window wraps around an axis's seam only if it is the last one along a
-    // shifted axis.
-    const bool wrap_w = tc.bw + g.ww > g.Pw;
+    // shifted axis.  n1h rows come before the H seam, the rest after it.
     const bool wrap_h = tc.bh + g.wh > g.Ph;
-    const int n1w = g.Pw - tc.bw, n1h = g.Ph - tc.bh;
+    const int n1h = g.Ph - tc.bh;
+    const int n1 = g.ww - g.sw;
+    int xb = tc.bw + n1;          // part B's first w (0 where the window wraps around the W seam)
+    xb -= xb >= g.Pw ? g.Pw : 0;
 #pragma unroll 1
     for (int rt = 0; rt < g.wt; ++rt) {
       int t = tc.bt + rt;
       t -= t >= g.Pt ? g.Pt : 0;
       const uint32_t slab = stage + rt * g.wh * run_bytes;
-      if (!wrap_w) {
 #pragma unroll 1
-        for (int tsr = 0; tsr < 3; ++tsr) {
+      for (int tsr = 0; tsr < 3; ++tsr) {
 #pragma unroll
-          for (int c = 0; c < CHUNKS; ++c) {
-            const uint32_t d = slab + tsr * kTensorBytes + c * kChunkTileBytes;
-            const int c0 = tc.head * head_dim + c * CHUNK_CH;
+        for (int c = 0; c < CHUNKS; ++c) {
+          const uint32_t d = slab + tsr * kTensorBytes + c * kChunkTileBytes;
+          const int c0 = tc.head * head_dim + c * CHUNK_CH;
+          const CUtensorMap* m = maps.m[tsr];
+          if (g.sw == 0) {
             if (!wrap_h) {
-              tma_load_5d(d, &maps.m[tsr][kBoxSlab], c0, tc.bw, tc.bh, t, tc.bsmp, bar);
+              tma_load_5d(d, &m[kBoxSlab], c0, tc.bw, tc.bh, t, tc.bsmp, bar);
             } else {
-              tma_load_5d(d, &maps.m[tsr][kBoxSeamH1], c0, tc.bw, tc.bh, t, tc.bsmp, bar);
-              tma_load_5d(d + n1h * run_bytes, &maps.m[tsr][kBoxSeamH2], c0, tc.bw, 0, t, tc.bsmp, bar);
+              tma_load_5d(d, &m[kBoxSeamH1], c0, tc.bw, tc.bh, t, tc.bsmp, bar);
+              tma_load_5d(d + n1h * run_bytes, &m[kBoxSeamH2], c0, tc.bw, 0, t, tc.bsmp, bar);
+            }
+          } else {
+            const uint32_t db = d + static_cast<uint32_t>(g.wh * n1) * kRowBytes;   // part B
+            if (!wrap_h) {
+              tma_load_5d(d, &m[kBoxA], c0, tc.bw, tc.bh, t, tc.bsmp, bar);
+              tma_load_5d(db, &m[kBoxB], c0, xb, tc.bh, t, tc.bsmp, bar);
+            } else {
+              tma_load_5d(d, &m[kBoxA1], c0, tc.bw, tc.bh, t, tc.bsmp, bar);
+              tma_load_5d(d + static_cast<uint32_t>(n1h * n1) * kRowBytes, &m[kBoxA2], c0, tc.bw, 0, t, tc.bsmp,
+                          bar);
+              tma_load_5d(db, &m[kBoxB1], c0, xb, tc.bh, t, tc.bsmp, bar);
+              tma_load_5d(db + static_cast<uint32_t>(n1h * g.sw) * kRowBytes, &m[kBoxB2], c0, xb, 0, t, tc.bsmp,
+                          bar);
             }
           }
-        }
-      } else {
-        int h = tc.bh;
-#pragma unroll 1
-        for (int rh = 0; rh < g.wh; ++rh) {
-          const uint32_t dst = slab + rh * run_bytes;
-#pragma unroll 1
-          for (int tsr = 0; tsr < 3; ++tsr) {
-#pragma unroll
-            for (int c = 0; c < CHUNKS; ++c) {
-              const uint32_t d = dst + tsr * kTensorBytes + c * kChunkTileBytes;
-              const int c0 = tc.head * head_dim + c * CHUNK_CH;
-              tma_load_5d(d, &maps.m[tsr][kBoxSeamW1], c0, tc.bw, h, t, tc.bsmp, bar);
-              tma_load_5d(d + n1w * kRowBytes, &maps.m[tsr][kBoxSeamW2], c0, 0, h, t, tc.bsmp, bar);
-            }
-          }
-          ++h;
-          h -= h >= g.Ph ? g.Ph : 0;
         }
       }
     }
