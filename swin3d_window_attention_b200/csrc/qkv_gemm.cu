@@ -13,7 +13,7 @@
 //
 // Per CTA (persistent, one per SM), 10 warps:
 //   warp 0   TMA: per output tile (128 tokens x 256 features) and K step of 64 channels, the
-//            x box (64 x 128) and the w box (64 x 256) into a 4-stage ring, 128B swizzle.
+//            x box (64 x 128) and the w box (64 x 256) into a 3-stage ring, 128B swizzle.
 //   warp 1   MMA: D (128 x 256, fp32, TMEM) += A B^T over 4 MMAs of K = 16 per stage; two
 //            accumulators (512 TMEM columns) so tile i+1 accumulates while tile i drains.
 //   warps 2-9 epilogue: warp w reads rows 32 (w % 4) .. of the accumulator (its TMEM lane
@@ -35,7 +35,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kBM = 128, kBN = 256, kBK = 64;      // tile: tokens x features x channels per stage
-constexpr int kStagesG = 4;
+constexpr int kStagesG = 3;
 constexpr int kABytes = kBM * kBK * 2;             // 16 KB
 constexpr int kBBytes = kBN * kBK * 2;             // 32 KB
 constexpr int kStageBytesG = kABytes + kBBytes;    // 48 KB
