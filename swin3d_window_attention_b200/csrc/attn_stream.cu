@@ -25,7 +25,7 @@
 //                       TMEM (the A operand of the TS form) and V plus a block of ones from
 //                       shared memory: O's columns 64.. are the row sums of the bf16 P.
 //   TMA warp 9          the unit's Q block (two buffers) and every K/V block through a
-//                       three-stage ring: per run of rows inside one T-slab and one side of
+//                       four-stage ring: per run of rows inside one T-slab and one side of
 //                       the H seam, boxes of 2^k rows; one row at a time (cut in two) where
 //                       the window wraps around the W seam.  Padded coordinates read as zero.
 //   table warp 10       per K/V block, the visible keys for each of the 8 combinations of a
@@ -47,7 +47,7 @@ using namespace attn;
 
 constexpr int kBlk = 128;                     // slots per block at most (query rows, keys)
 constexpr int kBlkBytes = kBlk * kRowBytes;   // one tensor's block: 16 KB
-constexpr int kStagesS = 3;
+constexpr int kStagesS = 4;
 constexpr int kThreadsS = 352;
 constexpr int kMmaWarpS = 8, kTmaWarpS = 9, kTableWarpS = 10;
 

@@ -274,14 +274,14 @@ def test_tf32_protocol_holds_under_random_schedules():
             model_tf32(ntiles=1 + seed % 11, has_tail=tail, seed=seed)
 
 
-def model_stream(nunits, nblk, seed=0, variant="kernel", max_steps=2_000_000):
+def model_stream(nunits, nblk, seed=0, variant="kernel", max_steps=2_000_000, stages=4):
     """The streaming kernel (windows of more than 144 slots): Q blocks by unit parity, K/V
-    blocks through a 3-stage ring, S double-buffered by block parity in TMEM with P written
+    blocks through a ring of `stages` stages (4 in the kernel), S double-buffered by block parity in TMEM with P written
     back over it (S(j + 2) waits for PV(j)), P handed over on a barrier per block parity, one
     O accumulator read out by every softmax thread before the next PV.  variant="single_p_full"
     hands P over on one barrier, which a fast row can lap."""
     rng = random.Random(seed)
-    S = 3
+    S = stages
     B = {}
 
     def mk(name, count):
@@ -366,7 +366,7 @@ def model_stream(nunits, nblk, seed=0, variant="kernel", max_steps=2_000_000):
 
 def test_stream_protocol_holds_under_random_schedules():
     for seed in range(100):
-        model_stream(nunits=1 + seed % 5, nblk=1 + seed % 4, seed=seed)
+        model_stream(nunits=1 + seed % 5, nblk=1 + seed % 4, seed=seed, stages=3 + seed % 2)
 
 
 def test_stream_single_p_full_is_caught():
