@@ -20,8 +20,9 @@
 //                      bf16 into shared memory.  One tile later (the PV MMA overlaps the next
 //                      softmax) it loads half of the row's O columns and the row sum (an MMA
 //                      output column, see below), scales by 1/rowsum, rounds to nearest even
-//                      and stores them to the query's original grid position; padded slots
-//                      are dropped.
+//                      and stores them to the query's original grid position in 32-byte
+//                      pieces, lane pairs swapping one so that each store writes both of a
+//                      row's pieces; padded slots are dropped.
 //   tail warp 8        the same for the 16 tail rows (S1 = Q[128:144] K^T in TMEM lanes
 //                      0..15, reachable from warp 8 like from warp 0), read with the 16x32bx2
 //                      shape: threads 0..15 hold half 0 of rows 128..143, threads 16..31
@@ -33,12 +34,13 @@
 //                      columns from 64 on are the row sums of the bf16 P; completion is
 //                      signalled by tcgen05.commit.
 //   TMA warp 10        (attn_common.cuh, shared with the TF32 kernel)
-//                      one thread loads the tile's Q, K and V with TMA: one box per T-slab
-//                      of the window (win_h x win_w tokens) per tensor, cut where the window
-//                      wraps around a seam of the shifted grid, straight from grid layout into
-//                      a 3-stage ring in the tensor core's 128-byte swizzled K-major layout;
-//                      padded coordinates are out of bounds and read as zero.  It runs ahead
-//                      as far as the ring allows.
+//                      one thread loads the tile's Q, K and V with TMA, a T-slab (win_h x
+//                      win_w tokens) at a time: one box per slab, or with a W shift two
+//                      (the w offsets before the wrap-around split, then the rest, which is
+//                      also the slots' order), each cut in two at the H seam; straight from
+//                      grid layout into a 3-stage ring in the tensor core's 128-byte swizzled
+//                      K-major layout; padded coordinates are out of bounds and read as zero.
+//                      It runs ahead as far as the ring allows.
 //   table warp 11      (attn_common.cuh) writes the slot -> grid-token table, a bitmask of the real slots, the
 //                      window's "last along a shifted axis" flags and, from these, the key
 //                      masks per region combination and key half, for the stage being loaded.
@@ -58,8 +60,8 @@ namespace {
 using namespace sm100;
 using namespace attn;
 
-// Stages of the Q/K/V ring: three for the attention kernel; two in the fused kernel, whose
-// AdaLN warps stream their rows through the shared memory the third stage would take.
+// Stages of the Q/K/V ring: three for the attention kernel (two are 60% slower); two in the
+// fused kernel, where three measure the same because its AdaLN warps set the pace.
 constexpr int kStagesPlain = 3;
 constexpr int kStagesFused = 2;
 constexpr int kTileBytes = kChunkTileBytes;         // 18432: one of Q / K / V
