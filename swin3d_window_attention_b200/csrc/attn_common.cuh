@@ -240,10 +240,10 @@ struct Ring {
 
 // TMA loader (one thread).  Per tile: wait until the stage is free, then load Q, K and V of
 // the tile's (sample, window, head), CHUNKS channel chunks of 128 bytes (CHUNK_CH channels)
-// per token row, one
-// box per T-slab (or per seam-cut piece), straight from grid layout into the stage: tensor
-// x, chunk c at stage + x * CHUNKS * kChunkTileBytes + c * kChunkTileBytes, rows in slot
-// order.  Padded coordinates are out of bounds and read as zero.  On an abort, or after the
+// per token row, in the boxes of the tensor maps above (per T-slab: one, or two parts A and
+// B with a W shift, each cut in two at the H seam), straight from grid layout into the
+// stage: tensor x, chunk c at stage + x * CHUNKS * kChunkTileBytes + c * kChunkTileBytes,
+// rows in slot order.  Padded coordinates are out of bounds and read as zero.  On an abort, or after the
 // last tile, waits (bounded) for the loads still in flight before returning.
 template <int CHUNKS, int CHUNK_CH, int STAGES, int STAGE_BYTES, bool WINDOW_MAJOR = false>
 __device__ __forceinline__ void tma_loader(const WinGeom& g, const TmaMaps& maps, const Ring& ring, int head_dim,
