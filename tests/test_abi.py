@@ -167,3 +167,47 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(api, "HERE", str(tmp_path))
     with pytest.raises(RuntimeError, match="missing"):
         api.load_library()
+
+
+def _qkv(**over):
+    # defaults: qkv over x (rejected last), so a call with them returns on the host everywhere
+    a = dict(x=FAKE, w=FAKE_QKV, b=None, qkv=FAKE, tokens=1152, C=512)
+    a.update(over)
+    return s3w.load_library().swin3d_qkv_proj_fwd(a["x"], a["w"], a["b"], a["qkv"], a["tokens"], a["C"], None)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(x=None), api.S3W_ERR_INVALID_ARG),
+    (dict(tokens=0), api.S3W_ERR_INVALID_ARG),
+    (dict(C=0), api.S3W_ERR_INVALID_ARG),
+    (dict(C=48), api.S3W_ERR_UNSUPPORTED),                    # not a multiple of 32
+    (dict(C=16416), api.S3W_ERR_UNSUPPORTED),                 # above 16,384
+    (dict(tokens=2 ** 31), api.S3W_ERR_UNSUPPORTED),          # TMA row coordinates are 32-bit
+    (dict(x=FAKE + 8), api.S3W_ERR_MISALIGNED),
+    (dict(qkv=FAKE + 16), api.S3W_ERR_MISALIGNED),            # qkv needs 32-byte alignment
+    (dict(), api.S3W_ERR_INVALID_ARG),                        # qkv over x
+    (dict(qkv=FAKE_QKV + 3 * 512 * 512 * 2 - 64), api.S3W_ERR_INVALID_ARG),   # qkv over the end of w
+])
+def test_qkv_proj_rejects_bad_arguments_on_host(over, expect):
+    assert _qkv(**over) == expect
+
+
+def _qkv_attn(**over):
+    a = dict(x=FAKE, w=FAKE_QKV, b=None, qkv=2 * FAKE_QKV, o=2 * FAKE_QKV + 4096, outd=0, B=1, T=4, H=12, W=24,
+             wt=2, wh=6, ww=12, st=1, sh=3, sw=6, heads=8, hd=64, scale=0.0)
+    a.update(over)
+    return s3w.load_library().swin3d_qkv_window_attn_fwd(
+        a["x"], a["w"], a["b"], a["qkv"], a["o"], a["outd"], a["B"], a["T"], a["H"], a["W"], a["wt"], a["wh"],
+        a["ww"], a["st"], a["sh"], a["sw"], a["heads"], a["hd"], a["scale"], None)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(o=None), api.S3W_ERR_INVALID_ARG),
+    (dict(heads=0), api.S3W_ERR_INVALID_ARG),
+    (dict(heads=300), api.S3W_ERR_UNSUPPORTED),               # C = 19,200 > 16,384
+    (dict(hd=48), api.S3W_ERR_UNSUPPORTED),                   # head_dim 32 or 64 only
+    (dict(st=2), api.S3W_ERR_INVALID_ARG),                    # shift == window
+    (dict(), api.S3W_ERR_INVALID_ARG),                        # o over the projection's output
+])
+def test_qkv_window_attn_rejects_bad_arguments_on_host(over, expect):
+    assert _qkv_attn(**over) == expect
