@@ -81,7 +81,8 @@ typedef enum { S3W_BF16 = 0, S3W_F32 = 1 } s3w_dtype;
  *           may be three slices of one fused [tokens][3C] buffer).  16-byte aligned.
  * o         device pointer, out_dtype elements (S3W_BF16 or S3W_F32), grid layout with
  *           o_token_stride elements between tokens (>= heads*head_dim, 16-byte rows).
- *           Must not overlap q, k or v.  Channels beyond heads*head_dim are not written.
+ *           Must not overlap q, k or v (S3W_ERR_INVALID_ARG).  Channels beyond heads*head_dim
+ *           are not written.
  * B,T,H,W   batch and unpadded grid sizes, each >= 1.
  * win_*     window extents, each >= 1, N = win_t*win_h*win_w.  1 <= N <= 144: one tile per
  *           (window, head).  144 < N <= 65536 (BF16 inputs, win_w <= 128): the streaming
