@@ -201,8 +201,20 @@ inline cudaError_t make_maps(const WinGeom& g, const void* const ptrs[3], bool f
                                            {n1, h1}, {n1, h2}, {n2, h1}, {n2, h2}};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   const cuuint32_t box_c = static_cast<cuuint32_t>(kRowBytes / es);
-  for (int t = 0; t < 3; ++t)
+  // Only the shapes the loader can use for this geometry are encoded (host time per call);
+  // the others are copies of the first one used, valid maps that no load names.
+  bool used[kBoxShapes] = {};
+  if (sw == 0) {
+    used[kBoxSlab] = true;
+    used[kBoxSeamH1] = used[kBoxSeamH2] = sh > 0;
+  } else {
+    used[kBoxA] = used[kBoxB] = true;
+    used[kBoxA1] = used[kBoxA2] = used[kBoxB1] = used[kBoxB2] = sh > 0;
+  }
+  const int first = sw == 0 ? kBoxSlab : kBoxA;
+  for (int t = 0; t < 3; ++t) {
     for (int b = 0; b < kBoxShapes; ++b) {
+      if (!used[b]) continue;
       const cuuint32_t box[5] = {box_c, boxwh[b][0], boxwh[b][1], 1, 1};
       CUresult r = enc(&maps->m[t][b], fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
                        const_cast<void*>(ptrs[t]), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -211,6 +223,9 @@ inline cudaError_t make_maps(const WinGeom& g, const void* const ptrs[3], bool f
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
       if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     }
+    for (int b = 0; b < kBoxShapes; ++b)
+      if (!used[b]) maps->m[t][b] = maps->m[t][first];
+  }
   return cudaSuccess;
 }
 
